@@ -1,0 +1,264 @@
+/*
+ * atlas_oracle.c -- plain, slow, fp64 CPU oracle for the detail branch's
+ * hierarchical locality-preserving attention of AtlasVid.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library. The CUDA library never
+ * calls it and shares no code, header, table or constant with it.
+ *
+ * Sources (page title, then section):
+ *   [TS]  "Technische Samenvatting: AtlasVid" (gist.science, Dutch), with
+ *         the same text as "Resume Technique : AtlasVid" (French) and
+ *         "Resumo Tecnico: AtlasVid" (Portuguese):
+ *           Methodologie 1, Fase 1 -- RoPE with temporal indices scaled by r_t;
+ *           Methodologie 1, Fase 2 -- latent volume cut into spatiotemporal
+ *               cubes, tokens reordered so each cube is contiguous, window
+ *               attention over the reordered sequence;
+ *           Methodologie 2 -- asymmetric hierarchical attention over the
+ *               concatenated [X_global; X_detail] set (global sees only
+ *               global; detail sees its own neighbourhood plus the global
+ *               tokens; global->detail masked with -inf) and position
+ *               alignment (global RoPE coordinates scaled by W/w, H/h, T/t).
+ *   [AB]  "AtlasVid: Efficient Ultra-High-Resolution Long Video Generation
+ *         via Decoupled Global-Local Modeling", abstract (arxivdaily.com):
+ *         reordered spatiotemporal windows, asymmetric global-local
+ *         attention, temporally scaled RoPE.
+ *
+ * The pages give no formulas for any of these steps. Where they are silent
+ * this file takes the plainest reading, stated at each function:
+ *   - tokens are stored in raster order r = (t*H + h)*W + w, one row of
+ *     heads*head_dim values per token;
+ *   - cubes are numbered in raster order over the cube grid, and the tokens
+ *     of one cube in raster order over the cube's own extent;
+ *   - RoPE splits head_dim into contiguous [t | h | w] segments and rotates
+ *     interleaved channel pairs (2k, 2k+1) of a segment of width d by the
+ *     angle p * theta^(-2k/d), p = index * scale for that axis;
+ *   - one joint softmax per query row over every allowed key; a detail
+ *     query is allowed the keys of its own cube and every global key; a
+ *     global query is allowed every global key and no detail key.
+ *
+ * Arithmetic is fp64 throughout, with no intermediate rounding.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* Cube reorder ([TS] Methodologie 1, Fase 2; [AB] "reordered windows")     */
+/* ------------------------------------------------------------------------ */
+
+/* Position j, in the cube-contiguous sequence, of the token at raster index
+ * r of a T x H x W grid cut into ct x ch x cw cubes. Each cube's
+ * L = ct*ch*cw tokens occupy positions cube*L .. cube*L + L - 1. */
+int64_t atlas_oracle_cube_position(int64_t T, int64_t H, int64_t W,
+                                   int64_t ct, int64_t ch, int64_t cw,
+                                   int64_t r)
+{
+    (void)T;
+    int64_t t = r / (H * W);
+    int64_t h = (r / W) % H;
+    int64_t w = r % W;
+    int64_t cubes_h = H / ch, cubes_w = W / cw;
+    int64_t cube = ((t / ct) * cubes_h + (h / ch)) * cubes_w + (w / cw);
+    int64_t local = ((t % ct) * ch + (h % ch)) * cw + (w % cw);
+    return cube * (ct * ch * cw) + local;
+}
+
+/* Fill pos[r] = cube position of raster token r, for every r < T*H*W. */
+void atlas_oracle_cube_positions(int64_t T, int64_t H, int64_t W,
+                                 int64_t ct, int64_t ch, int64_t cw,
+                                 int64_t *pos)
+{
+    int64_t n = T * H * W;
+    for (int64_t r = 0; r < n; ++r)
+        pos[r] = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+}
+
+/* dst[position(r)] = src[r], row by row, as a byte copy: every bit pattern
+ * survives, so the inverse below restores the input exactly. */
+void atlas_oracle_cube_reorder(const unsigned char *src, unsigned char *dst,
+                               int64_t T, int64_t H, int64_t W,
+                               int64_t ct, int64_t ch, int64_t cw,
+                               int64_t row_bytes)
+{
+    int64_t n = T * H * W;
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        memcpy(dst + j * row_bytes, src + r * row_bytes, (size_t)row_bytes);
+    }
+}
+
+/* The exact inverse: dst[r] = src[position(r)]. */
+void atlas_oracle_cube_unorder(const unsigned char *src, unsigned char *dst,
+                               int64_t T, int64_t H, int64_t W,
+                               int64_t ct, int64_t ch, int64_t cw,
+                               int64_t row_bytes)
+{
+    int64_t n = T * H * W;
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        memcpy(dst + r * row_bytes, src + j * row_bytes, (size_t)row_bytes);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 3D RoPE ([TS] Methodologie 1, Fase 1: temporal index times r_t;          */
+/*          [TS] Methodologie 2, position alignment: global coordinates     */
+/*          scaled by the resolution ratios)                                */
+/* ------------------------------------------------------------------------ */
+
+/* Rotate one segment of one head: channels [off, off + d) of x, as pairs
+ * (2k, 2k+1), by angle p * theta^(-2k/d). */
+static void rope_segment(const double *x, double *y, int64_t off, int64_t d,
+                         double p, double theta)
+{
+    for (int64_t k = 0; k < d / 2; ++k) {
+        double omega = pow(theta, -2.0 * (double)k / (double)d);
+        double phi = p * omega;
+        double c = cos(phi), s = sin(phi);
+        double x0 = x[off + 2 * k], x1 = x[off + 2 * k + 1];
+        y[off + 2 * k] = x0 * c - x1 * s;
+        y[off + 2 * k + 1] = x0 * s + x1 * c;
+    }
+}
+
+/* Apply 3D RoPE to n_rows token rows. Row i of x (heads*head_dim values)
+ * is the token at raster index raster_idx[i] of a T x H x W grid; its
+ * position is p = (t*s_t, h*s_h, w*s_w). head_dim = d_t + d_h + d_w, each
+ * even; the t segment comes first, then h, then w. */
+void atlas_oracle_rope3d_rows(const double *x, double *y, int64_t n_rows,
+                              const int64_t *raster_idx,
+                              int64_t T, int64_t H, int64_t W,
+                              int64_t heads, int64_t head_dim, double theta,
+                              int64_t d_t, int64_t d_h, int64_t d_w,
+                              double s_t, double s_h, double s_w)
+{
+    (void)T;
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t r = raster_idx[i];
+        double p_t = (double)(r / (H * W)) * s_t;
+        double p_h = (double)((r / W) % H) * s_h;
+        double p_w = (double)(r % W) * s_w;
+        for (int64_t hd = 0; hd < heads; ++hd) {
+            const double *xr = x + (i * heads + hd) * head_dim;
+            double *yr = y + (i * heads + hd) * head_dim;
+            rope_segment(xr, yr, 0, d_t, p_t, theta);
+            rope_segment(xr, yr, d_t, d_h, p_h, theta);
+            rope_segment(xr, yr, d_t + d_h, d_w, p_w, theta);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Asymmetric global-local attention ([TS] Methodologie 1 Fase 2 and 2)     */
+/* ------------------------------------------------------------------------ */
+
+/* Key ids run over the concatenated set: 0 .. N-1 are the detail tokens in
+ * cube-contiguous order, N .. N+G-1 the global tokens. Query ids likewise.
+ * A detail query sees the keys of its own cube (window of L consecutive
+ * positions) and every global key; a global query sees every global key and
+ * no detail key (mask value -inf). */
+static int allowed(int64_t q, int64_t k, int64_t N, int64_t L)
+{
+    int q_detail = q < N, k_detail = k < N;
+    if (q_detail && k_detail) return (q / L) == (k / L);
+    if (q_detail && !k_detail) return 1;
+    if (!q_detail && k_detail) return 0;
+    return 1;
+}
+
+/* One head. For each of the n_q queries (ids q_ids[i], vectors q[i]),
+ * evaluate allowed() against all N+G keys, take logits scale*<q,k> on the
+ * allowed ones, then a two-pass softmax (max, then sum of exp) and the
+ * weighted sum of V. Outputs o[i] (head_dim values) and lse[i] (natural
+ * log of the softmax denominator, logits included, i.e. max + log(sum)).
+ *
+ * k_d/v_d hold detail rows kd_lo .. kd_hi-1 only (row stride head_dim);
+ * k_g/v_g hold all G global rows. If an allowed detail key falls outside
+ * the rows supplied the function returns 1 (caller error); 2 on allocation
+ * failure; 0 on success. */
+int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
+                                int64_t n_global, int64_t head_dim,
+                                double scale,
+                                const double *k_d, const double *v_d,
+                                int64_t kd_lo, int64_t kd_hi,
+                                const double *k_g, const double *v_g,
+                                int64_t n_q, const int64_t *q_ids,
+                                const double *q, double *o, double *lse,
+                                int n_threads)
+{
+    int64_t N = n_detail, G = n_global, D = head_dim;
+    int status = 0;
+    if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+    for (int64_t i = 0; i < n_q; ++i) {
+        int64_t qid = q_ids[i];
+        const double *qi = q + i * D;
+        double *oi = o + i * D;
+        double *logit = (double *)malloc((size_t)(N + G) * sizeof(double));
+        const double **vrow = (const double **)malloc((size_t)(N + G) * sizeof(double *));
+        if (!logit || !vrow) {
+            free(logit); free(vrow);
+#pragma omp atomic write
+            status = 2;
+            continue;
+        }
+        int64_t n_allowed = 0;
+        int bad = 0;
+        for (int64_t kid = 0; kid < N + G; ++kid) {
+            if (!allowed(qid, kid, N, window_len)) continue;
+            const double *kr, *vr;
+            if (kid < N) {
+                if (kid < kd_lo || kid >= kd_hi) { bad = 1; break; }
+                kr = k_d + (kid - kd_lo) * D;
+                vr = v_d + (kid - kd_lo) * D;
+            } else {
+                kr = k_g + (kid - N) * D;
+                vr = v_g + (kid - N) * D;
+            }
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += qi[d] * kr[d];
+            logit[n_allowed] = scale * dot;
+            vrow[n_allowed] = vr;
+            ++n_allowed;
+        }
+        if (bad) {
+            free(logit); free(vrow);
+#pragma omp atomic write
+            status = 1;
+            continue;
+        }
+        /* pass 1: row maximum */
+        double m = -INFINITY;
+        for (int64_t a = 0; a < n_allowed; ++a)
+            if (logit[a] > m) m = logit[a];
+        /* pass 2: denominator and weighted sum of V */
+        double sum = 0.0;
+        for (int64_t d = 0; d < D; ++d) oi[d] = 0.0;
+        for (int64_t a = 0; a < n_allowed; ++a) {
+            double p = exp(logit[a] - m);
+            sum += p;
+            for (int64_t d = 0; d < D; ++d) oi[d] += p * vrow[a][d];
+        }
+        for (int64_t d = 0; d < D; ++d) oi[d] /= sum;
+        lse[i] = m + log(sum);
+        free(logit);
+        free(vrow);
+    }
+    return status;
+}
+
+/* Number of threads an OpenMP parallel region of this library would use by
+ * default (reported beside CPU timings). */
+int atlas_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

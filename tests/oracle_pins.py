@@ -1,0 +1,418 @@
+"""Pins that tie the fp64 oracle to facts fixed outside the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with a fact that the pages or the mathematics fix:
+an independent construction (numpy reshape/transpose for the cube order,
+torch's dense scaled-dot-product attention with an explicit boolean mask for
+the attention), a closed form (literal RoPE angles, O = V for 1-token
+windows, mean of V when all logits tie), an invariant (bijection, exact
+inverse, pair norms, relative-position property, rows summing to 1), or a
+special case that reduces to textbook full attention. The test modules run
+them against the real oracle (all must pass) and against copies of the
+oracle with a planted mistake (each mutant must fail at least one).
+
+Passages: "Technische Samenvatting: AtlasVid" (gist.science), Methodologie 1
+Fase 1 (temporal RoPE scale r_t), Fase 2 (cube reorder, window attention), 2
+(asymmetric hierarchical attention; position alignment).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([float(v) for v in line.split()])
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# Cube reorder
+# ---------------------------------------------------------------------------
+
+CUBE_CASES = [
+    ((4, 8, 8), (2, 4, 4)),
+    ((3, 6, 10), (3, 2, 5)),
+    ((2, 4, 6), (1, 2, 3)),
+    ((6, 4, 4), (2, 4, 2)),
+    ((5, 3, 7), (1, 1, 1)),
+    ((2, 3, 4), (2, 3, 4)),
+]
+
+
+def rearrange_order(grid, cube):
+    """order[j] = raster index of the token at cube position j, built with a
+    reshape/transpose: (T/ct, ct, H/ch, ch, W/cw, cw) -> cube axes first."""
+    T, H, W = grid
+    ct, ch, cw = cube
+    idx = np.arange(T * H * W, dtype=np.int64).reshape(
+        T // ct, ct, H // ch, ch, W // cw, cw)
+    return idx.transpose(0, 2, 4, 1, 3, 5).reshape(-1)
+
+
+def pin_cube_matches_rearrange(o):
+    for grid, cube in CUBE_CASES:
+        pos = o.cube_positions(grid, cube)
+        order = rearrange_order(grid, cube)
+        assert np.array_equal(pos[order], np.arange(pos.size)), (grid, cube)
+
+
+def pin_cube_bijection(o):
+    for grid, cube in CUBE_CASES:
+        pos = o.cube_positions(grid, cube)
+        assert np.array_equal(np.sort(pos), np.arange(pos.size)), (grid, cube)
+
+
+def pin_cube_worked_example(o):
+    for row in _golden_rows("cube_positions_example.txt"):
+        T, H, W, ct, ch, cw, t, h, w, r, j = (int(v) for v in row)
+        assert (t * H + h) * W + w == r
+        assert o.cube_position((T, H, W), (ct, ch, cw), r) == j, row
+
+
+def pin_cube_locality(o):
+    """Every block of L consecutive positions is one geometric cube."""
+    for grid, cube in CUBE_CASES:
+        T, H, W = grid
+        ct, ch, cw = cube
+        L = ct * ch * cw
+        pos = o.cube_positions(grid, cube)
+        inv = np.empty_like(pos)
+        inv[pos] = np.arange(pos.size)
+        t, h, w = inv // (H * W), (inv // W) % H, inv % W
+        for b in range(pos.size // L):
+            sl = slice(b * L, (b + 1) * L)
+            for coord, c in ((t, ct), (h, ch), (w, cw)):
+                lo = coord[sl].min()
+                assert lo % c == 0 and coord[sl].max() - lo == c - 1, (grid, cube, b)
+
+
+def pin_cube_roundtrip_bytes(o):
+    rng = np.random.default_rng(1)
+    for grid, cube in CUBE_CASES:
+        n = grid[0] * grid[1] * grid[2]
+        x = rng.integers(0, 256, size=(n, 3, 10), dtype=np.uint8)
+        # include NaN payload patterns when viewed as float32 / bfloat16
+        x[::3, 0, :4] = np.frombuffer(np.array([0x7FC00001], np.uint32).tobytes(), np.uint8)
+        y = o.cube_reorder(x, grid, cube)
+        z = o.cube_unorder(y, grid, cube)
+        assert z.tobytes() == x.tobytes(), (grid, cube)
+        order = rearrange_order(grid, cube)
+        assert y.tobytes() == x[order].tobytes(), (grid, cube)
+
+
+def pin_cube_special_cases(o):
+    for grid in ((3, 5, 7), (2, 2, 2)):
+        n = grid[0] * grid[1] * grid[2]
+        assert np.array_equal(o.cube_positions(grid, (1, 1, 1)), np.arange(n))
+        assert np.array_equal(o.cube_positions(grid, grid), np.arange(n))
+
+
+CUBE_PINS = [pin_cube_matches_rearrange, pin_cube_bijection,
+             pin_cube_worked_example, pin_cube_locality,
+             pin_cube_roundtrip_bytes, pin_cube_special_cases]
+
+
+# ---------------------------------------------------------------------------
+# 3D RoPE
+# ---------------------------------------------------------------------------
+
+def pin_rope_literal_angles(o):
+    """theta=100, 4 channels per axis: frequencies are exactly 1 and 0.1."""
+    for row in _golden_rows("rope_literal_angles.txt"):
+        theta, dt, dh, dw, T, H, W, t, h, w, st, sh, sw = row[:13]
+        angles = row[13:]
+        grid = (int(T), int(H), int(W))
+        r = (int(t) * grid[1] + int(h)) * grid[2] + int(w)
+        D = int(dt + dh + dw)
+        rng = np.random.default_rng(7)
+        x = rng.standard_normal((1, 2, D))
+        y = o.rope3d_rows(x, [r], grid, theta, (int(dt), int(dh), int(dw)),
+                          (st, sh, sw))
+        for head in range(2):
+            for k, phi in enumerate(angles):
+                x0, x1 = x[0, head, 2 * k], x[0, head, 2 * k + 1]
+                c, s = math.cos(phi), math.sin(phi)
+                assert abs(y[0, head, 2 * k] - (x0 * c - x1 * s)) < 1e-13, (row, k)
+                assert abs(y[0, head, 2 * k + 1] - (x0 * s + x1 * c)) < 1e-13, (row, k)
+
+
+def pin_rope_zero_scale_identity(o):
+    grid = (3, 4, 5)
+    n = 60
+    x = np.random.default_rng(2).standard_normal((n, 3, 16))
+    y = o.rope3d_grid(x, grid, 10000.0, (4, 6, 6), (0.0, 0.0, 0.0))
+    assert np.array_equal(x, y)
+    # origin token is never rotated, whatever the scales
+    y = o.rope3d_rows(x[:1], [0], grid, 10000.0, (4, 6, 6), (4.0, 8.0, 8.0))
+    assert np.array_equal(x[:1], y)
+
+
+def pin_rope_pair_norms(o):
+    grid = (4, 6, 8)
+    x = np.random.default_rng(3).standard_normal((192, 2, 128))
+    y = o.rope3d_grid(x, grid, 10000.0, (44, 42, 42), (4.0, 8.0, 8.0))
+    nx = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    ny = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    assert np.max(np.abs(nx - ny)) < 1e-12
+
+
+def pin_rope_relative_position(o):
+    """<R(p)q, R(p')k> depends only on p - p' (axis by axis)."""
+    grid = (6, 7, 9)
+    H, W = grid[1], grid[2]
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 1, 64))
+    k = rng.standard_normal((1, 1, 64))
+    split, scales = (16, 24, 24), (4.0, 2.0, 3.0)
+
+    def dot_at(pq, pk):
+        rq = (pq[0] * H + pq[1]) * W + pq[2]
+        rk = (pk[0] * H + pk[1]) * W + pk[2]
+        a = o.rope3d_rows(q, [rq], grid, 10000.0, split, scales)
+        b = o.rope3d_rows(k, [rk], grid, 10000.0, split, scales)
+        return float(np.sum(a * b))
+
+    base = dot_at((1, 2, 3), (0, 0, 1))
+    for shift in ((1, 0, 0), (0, 3, 0), (0, 0, 4), (4, 4, 5)):
+        pq = (1 + shift[0], 2 + shift[1], 3 + shift[2])
+        pk = (0 + shift[0], 0 + shift[1], 1 + shift[2])
+        assert abs(dot_at(pq, pk) - base) < 1e-11, shift
+    # and a different offset gives a different value (the angle is not lost)
+    assert abs(dot_at((2, 2, 3), (0, 0, 1)) - base) > 1e-6
+
+
+def pin_rope_temporal_scale(o):
+    """Scaling the temporal index by r_t equals placing the token at t*r_t."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, 2, 64))
+    split = (16, 24, 24)
+    for r_t in (2.0, 4.0):
+        for (t, h, w) in ((1, 2, 3), (3, 0, 5)):
+            small = (4, 4, 8)
+            tall = (4 * 4, 4, 8)
+            a = o.rope3d_rows(x, [(t * 4 + h) * 8 + w], small, 10000.0, split,
+                              (r_t, 1.0, 1.0))
+            tt = int(t * r_t)
+            b = o.rope3d_rows(x, [(tt * 4 + h) * 8 + w], tall, 10000.0, split,
+                              (1.0, 1.0, 1.0))
+            assert np.max(np.abs(a - b)) < 1e-12
+
+
+def pin_rope_complex_form(o):
+    """At unit scales the result equals the complex-multiplication form of
+    rotary embedding, per axis: (x0 + i x1) * exp(i * p * theta^(-2k/d))."""
+    grid = (3, 4, 5)
+    n = 60
+    x = torch.randn(n, 2, 64, dtype=torch.float64,
+                    generator=torch.Generator().manual_seed(6))
+    y = o.rope3d_grid(x.numpy(), grid, 10000.0, (16, 24, 24), (1.0, 1.0, 1.0))
+    pos = torch.stack(torch.meshgrid(torch.arange(3), torch.arange(4),
+                                     torch.arange(5), indexing="ij"), -1).reshape(n, 3)
+    parts = []
+    off = 0
+    for axis, d in enumerate((16, 24, 24)):
+        freqs = 10000.0 ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+        ang = pos[:, axis:axis + 1].double() * freqs[None, :]          # [n, d/2]
+        xc = torch.view_as_complex(x[..., off:off + d].reshape(n, 2, d // 2, 2).contiguous())
+        rot = xc * torch.polar(torch.ones_like(ang), ang)[:, None, :]
+        parts.append(torch.view_as_real(rot).reshape(n, 2, d))
+        off += d
+    ref = torch.cat(parts, -1).numpy()
+    assert np.max(np.abs(ref - y)) < 1e-12
+
+
+def pin_rope_heads_identical(o):
+    grid = (2, 3, 4)
+    x1 = np.random.default_rng(8).standard_normal((24, 1, 32))
+    x = np.repeat(x1, 4, axis=1)
+    y = o.rope3d_grid(x, grid, 10000.0, (8, 12, 12), (4.0, 2.0, 2.0))
+    for hd in range(4):
+        assert np.array_equal(y[:, hd], y[:, 0])
+
+
+ROPE_PINS = [pin_rope_literal_angles, pin_rope_zero_scale_identity,
+             pin_rope_pair_norms, pin_rope_relative_position,
+             pin_rope_temporal_scale, pin_rope_complex_form,
+             pin_rope_heads_identical]
+
+
+# ---------------------------------------------------------------------------
+# Asymmetric global-local attention
+# ---------------------------------------------------------------------------
+
+def geometric_mask(grid, cube, G):
+    """Boolean allowed-matrix over [detail (cube order); global], built from
+    cube ids that a reshape assigns to each token: a detail query may see
+    keys with its own cube id and every global key; a global query may see
+    only global keys."""
+    T, H, W = grid
+    ct, ch, cw = cube
+    N = T * H * W
+    if N:
+        ids = np.arange(N // (ct * ch * cw)).reshape(T // ct, H // ch, W // cw)
+        cube_of_raster = np.broadcast_to(
+            ids[:, None, :, None, :, None],
+            (T // ct, ct, H // ch, ch, W // cw, cw)).reshape(-1)
+        cube_of_pos = cube_of_raster[rearrange_order(grid, cube)]
+    else:
+        cube_of_pos = np.zeros(0, dtype=np.int64)
+    allowed = np.zeros((N + G, N + G), dtype=bool)
+    allowed[:N, :N] = cube_of_pos[:, None] == cube_of_pos[None, :]
+    allowed[:N, N:] = True
+    allowed[N:, N:] = True
+    return allowed
+
+
+ATTN_CASES = [
+    # grid, cube, G, heads, D
+    ((4, 8, 8), (2, 4, 4), 32, 2, 64),
+    ((2, 4, 6), (1, 2, 3), 5, 2, 16),
+    ((2, 4, 4), (2, 2, 2), 1, 1, 8),
+    ((3, 4, 4), (3, 4, 4), 0, 2, 16),
+    ((2, 2, 4), (1, 1, 1), 0, 1, 8),
+    ((0, 0, 0), (1, 1, 1), 40, 2, 16),
+    ((2, 6, 4), (2, 3, 2), 7, 3, 32),
+]
+
+
+def _rand_case(grid, G, heads, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    N = grid[0] * grid[1] * grid[2]
+    mk = lambda n: torch.randn(n, heads, D, dtype=torch.float64, generator=g).numpy()
+    return N, mk(N), mk(N), mk(N), mk(G), mk(G), mk(G)
+
+
+def pin_attention_dense_sdpa(o):
+    """Equal to dense masked softmax attention over all N+G tokens."""
+    for ci, (grid, cube, G, heads, D) in enumerate(ATTN_CASES):
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 100 + ci)
+        L = cube[0] * cube[1] * cube[2]
+        scale = 1.0 / math.sqrt(D)
+        od, og, lse = o.attention_full(qd, kd, vd, L, qg, kg, vg, scale)
+        mask = torch.from_numpy(geometric_mask(grid, cube, G))
+        q = torch.from_numpy(np.concatenate([qd, qg])).permute(1, 0, 2)
+        k = torch.from_numpy(np.concatenate([kd, kg])).permute(1, 0, 2)
+        v = torch.from_numpy(np.concatenate([vd, vg])).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k, v, attn_mask=mask, scale=scale).permute(1, 0, 2).numpy()
+        got = np.concatenate([od, og])
+        assert np.max(np.abs(ref - got)) < 1e-12, (grid, cube, G)
+        logits = (q @ k.transpose(1, 2)).numpy() * scale
+        logits = np.where(mask.numpy()[None], logits, -np.inf)
+        mx = logits.max(-1, keepdims=True)
+        ref_lse = (mx + np.log(np.exp(logits - mx).sum(-1, keepdims=True)))[..., 0]
+        assert np.max(np.abs(ref_lse - lse)) < 1e-12, (grid, cube, G)
+
+
+def pin_attention_full_when_one_cube(o):
+    """One cube covering the volume and no global tokens: full attention."""
+    grid, heads, D = (2, 4, 4), 2, 16
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, 0, heads, D, 11)
+    od, _, _ = o.attention_full(qd, kd, vd, N, qg, kg, vg, 0.3)
+    q, k, v = (torch.from_numpy(a).permute(1, 0, 2) for a in (qd, kd, vd))
+    ref = torch.softmax(q @ k.transpose(1, 2) * 0.3, -1) @ v
+    assert np.max(np.abs(ref.permute(1, 0, 2).numpy() - od)) < 1e-12
+
+
+def pin_attention_single_token_windows(o):
+    """1x1x1 cubes and no global tokens: each row sees only itself, O = V."""
+    grid, heads, D = (2, 3, 4), 2, 8
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, 0, heads, D, 12)
+    od, _, lse = o.attention_full(qd, kd, vd, 1, qg, kg, vg, 0.25)
+    assert np.array_equal(od, vd)
+    ref_lse = 0.25 * np.einsum("nhd,nhd->hn", qd, kd)
+    assert np.max(np.abs(ref_lse - lse)) < 1e-12
+
+
+def pin_attention_zero_keys_mean(o):
+    """K = 0: every allowed logit ties, O = mean of the allowed V rows."""
+    grid, cube, G, heads, D = (2, 4, 4), (1, 2, 2), 6, 2, 8
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 13)
+    kd[:] = 0.0
+    kg[:] = 0.0
+    L = 4
+    od, og, lse = o.attention_full(qd, kd, vd, L, qg, kg, vg, 0.5)
+    for i in range(N):
+        w = i // L
+        allowed_v = np.concatenate([vd[w * L:(w + 1) * L], vg])
+        assert np.max(np.abs(od[i] - allowed_v.mean(0))) < 1e-12
+    assert np.max(np.abs(og - vg.mean(0, keepdims=True))) < 1e-12
+    assert np.max(np.abs(lse[:, :N] - math.log(L + G))) < 1e-12
+    assert np.max(np.abs(lse[:, N:] - math.log(G))) < 1e-12
+
+
+def pin_attention_rows_sum_to_one(o):
+    for grid, cube, G, heads, D in ATTN_CASES:
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 14)
+        vd[:] = 1.0
+        vg[:] = 1.0
+        L = cube[0] * cube[1] * cube[2]
+        od, og, _ = o.attention_full(qd, kd, vd, L, qg, kg, vg, 1.0)
+        assert np.max(np.abs(np.concatenate([od, og]) - 1.0)) < 1e-12
+
+
+def pin_attention_global_ignores_detail(o):
+    """Global rows see no detail key: changing detail K/V changes nothing."""
+    grid, cube, G, heads, D = (2, 4, 4), (2, 2, 2), 9, 2, 16
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 15)
+    _, og1, l1 = o.attention_full(qd, kd, vd, 8, qg, kg, vg, 0.25)
+    _, og2, l2 = o.attention_full(qd, kd * 3.0 + 1.0, -vd, 8, qg, kg, vg, 0.25)
+    assert np.array_equal(og1, og2) and np.array_equal(l1[:, N:], l2[:, N:])
+
+
+def pin_attention_probe_mass(o):
+    """V columns = indicators of (own window, other windows, global): the
+    output columns are the attention mass on each group; the mass outside
+    the own window and the global set is exactly 0."""
+    grid, cube, G, heads, D = (2, 4, 8), (1, 2, 4), 5, 1, 8
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 16)
+    L = 8
+    nwin = N // L
+    for w in range(nwin):
+        vd[:] = 0.0
+        vg[:] = 0.0
+        vd[w * L:(w + 1) * L, :, 0] = 1.0
+        vd[:w * L, :, 1] = 1.0
+        vd[(w + 1) * L:, :, 1] = 1.0
+        vg[:, :, 2] = 1.0
+        od, og, _ = o.attention_full(qd, kd, vd, L, qg, kg, vg, 0.35)
+        rows = slice(w * L, (w + 1) * L)
+        assert np.all(od[rows, :, 1] == 0.0)
+        assert np.all(od[rows, :, 0] > 0.0) and np.all(od[rows, :, 2] > 0.0)
+        assert np.max(np.abs(od[rows, :, 0] + od[rows, :, 2] - 1.0)) < 1e-12
+        assert np.all(og[:, :, 0] == 0.0) and np.all(og[:, :, 1] == 0.0)
+
+
+def pin_attention_rejects_missing_rows(o):
+    """A detail query whose window rows are not supplied is an error."""
+    D = 8
+    q = np.ones((1, D))
+    k = np.zeros((4, D))
+    try:
+        o.attention_head(16, 8, 0, 1.0, k, k, 0, None, None, [9], q)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("missing window rows not detected")
+    out, _ = o.attention_head(16, 8, 0, 1.0, np.zeros((8, D)), np.ones((8, D)),
+                              8, None, None, [9], q)
+    assert np.array_equal(out, np.ones((1, D)))
+
+
+ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_full_when_one_cube,
+             pin_attention_single_token_windows, pin_attention_zero_keys_mean,
+             pin_attention_rows_sum_to_one, pin_attention_global_ignores_detail,
+             pin_attention_probe_mass, pin_attention_rejects_missing_rows]
+
+ALL_PINS = CUBE_PINS + ROPE_PINS + ATTN_PINS

@@ -1,0 +1,50 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check
+that the pins catch every one. The mistakes are planted in the oracle, on the
+CPU; the real oracle is untouched."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in atlas_oracle.c, replacement)
+MUTANTS = [
+    ("window_off_by_one", "return (q / L) == (k / L);", "return (q / L) == ((k + 1) / L);"),
+    ("global_sees_detail", "if (!q_detail && k_detail) return 0;", "if (!q_detail && k_detail) return 1;"),
+    ("detail_misses_global", "if (q_detail && !k_detail) return 1;", "if (q_detail && !k_detail) return 0;"),
+    ("rope_sign", "y[off + 2 * k] = x0 * c - x1 * s;", "y[off + 2 * k] = x0 * c + x1 * s;"),
+    ("rope_freq_width", "pow(theta, -2.0 * (double)k / (double)d)", "pow(theta, -2.0 * (double)k / (double)(d + 2))"),
+    ("rope_wrong_axis", "rope_segment(xr, yr, d_t + d_h, d_w, p_w, theta);", "rope_segment(xr, yr, d_t + d_h, d_w, p_h, theta);"),
+    ("rope_scale_mixup", "double p_h = (double)((r / W) % H) * s_h;", "double p_h = (double)((r / W) % H) * s_w;"),
+    ("rope_pair_layout", "double x0 = x[off + 2 * k], x1 = x[off + 2 * k + 1];", "double x0 = x[off + k], x1 = x[off + k + d / 2];"),
+    ("cube_local_transposed", "int64_t local = ((t % ct) * ch + (h % ch)) * cw + (w % cw);",
+     "int64_t local = ((h % ch) * ct + (t % ct)) * cw + (w % cw);"),
+    ("cube_order_transposed", "int64_t cube = ((t / ct) * cubes_h + (h / ch)) * cubes_w + (w / cw);",
+     "int64_t cube = ((w / cw) * cubes_h + (h / ch)) * (T / ct) + (t / ct);"),
+    ("dropped_scale", "logit[n_allowed] = scale * dot;", "logit[n_allowed] = dot;"),
+    ("lse_missing_max", "lse[i] = m + log(sum);", "lse[i] = log(sum);"),
+    ("unorder_not_inverse", "memcpy(dst + r * row_bytes, src + j * row_bytes, (size_t)row_bytes);",
+     "memcpy(dst + j * row_bytes, src + r * row_bytes, (size_t)row_bytes);"),
+    ("dot_drops_last_channel", "for (int64_t d = 0; d < D; ++d) dot += qi[d] * kr[d];",
+     "for (int64_t d = 0; d + 1 < D; ++d) dot += qi[d] * kr[d];"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    mutant_c = tmp_path / f"{name}.c"
+    mutant_c.write_text(src.replace(old, new))
+    so = oracle.build(str(mutant_c), str(tmp_path / f"lib{name}.so"))
+    orc = oracle.Oracle(oracle.load(so))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+        except Exception:  # a crash or an error also counts as caught
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutant {name}"
