@@ -1,0 +1,462 @@
+"""Benchmark of the detail-branch attention path (one JSON line on rank 0).
+
+A step is one pass of the whole path over one synthetic input resident in
+HBM: reorder+RoPE of detail Q and K, reorder of detail V, RoPE of global Q
+and K, the asymmetric local-global attention, and the unorder of the detail
+output -- seven launches of this repository's kernels through the C-ABI.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload 720p]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
+
+Metric: TFLOP/s of unmasked attention FLOPs (4*D per allowed query-key pair
+per head) over the whole step; the attention kernel's own TFLOP/s and the
+reorder+RoPE kernels' GB/s (one read + one write of detail Q, K, V and global
+Q, K) are reported beside it with their fractions of the measured peaks.
+Multi-GPU (torchrun): every rank runs its own copy of the workload (weak
+scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from video_dit_windowed_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "local-global attn TFLOP/s (unmasked) & % BF16 peak; reorder+RoPE GB/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU path
+# ---------------------------------------------------------------------------
+class Path:
+    """Device buffers and the seven C-ABI calls of one step."""
+
+    def __init__(self, w, device, stream):
+        from video_dit_windowed_b200 import atlas
+        self.atlas = atlas
+        self.w = w
+        self.dev = device
+        self.stream = stream
+        x = make_inputs(w, device=device)
+        self.x = x
+        self.rd = atlas.make_rope(w.theta, w.split, w.detail_scales)
+        self.rg = atlas.make_rope(w.theta, w.split, w.global_scales)
+        e = lambda t: torch.empty_like(t)
+        self.q_d, self.k_d, self.v_d = e(x["q_d"]), e(x["k_d"]), e(x["v_d"])
+        self.q_g, self.k_g = e(x["q_g"]), e(x["k_g"])
+        self.o_d, self.o_g = e(x["q_d"]), e(x["q_g"])
+        self.o_raster = e(x["q_d"])
+
+    def step(self, ev=None):
+        """One pass; ``ev`` (5 CUDA events) brackets the phases if given."""
+        a, w, s, x = self.atlas, self.w, self.stream, self.x
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec(0)
+        if w.n_detail:
+            a.cube_reorder(x["q_d"], self.q_d, w.grid, w.cube, self.rd, stream=s)
+            a.cube_reorder(x["k_d"], self.k_d, w.grid, w.cube, self.rd, stream=s)
+            a.cube_reorder(x["v_d"], self.v_d, w.grid, w.cube, None, stream=s)
+        rec(1)
+        if w.n_global:
+            a.rope3d(x["q_g"], self.q_g, w.global_grid, self.rg, stream=s)
+            a.rope3d(x["k_g"], self.k_g, w.global_grid, self.rg, stream=s)
+        rec(2)
+        a.local_global_attn(self.q_d, self.k_d, self.v_d, w.window_len, self.q_g, self.k_g,
+                            x["v_g"], self.o_d, self.o_g, None, stream=s)
+        rec(3)
+        if w.n_detail:
+            a.cube_unorder(self.o_d, self.o_raster, w.grid, w.cube, stream=s)
+        rec(4)
+
+    def launches_per_step(self):
+        w = self.w
+        return (3 if w.n_detail else 0) + (2 if w.n_global else 0) + 1 + (1 if w.n_detail else 0)
+
+    @staticmethod
+    def phase_ms(ev):
+        return {"reorder": ev[0].elapsed_time(ev[1]), "rope_g": ev[1].elapsed_time(ev[2]),
+                "attn": ev[2].elapsed_time(ev[3]), "unorder": ev[3].elapsed_time(ev[4])}
+
+
+def bytes_reorder_rope(w):
+    row = w.heads * w.head_dim * w.elem_bytes
+    return 2 * 3 * w.n_detail * row, 2 * 2 * w.n_global * row
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "video_dit_windowed_b200", "csrc")
+    for name in ("attn_tc.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU)
+# ---------------------------------------------------------------------------
+def oracle_sample_flops(w, n_det_rows, n_glob_rows):
+    D = w.head_dim
+    return 4 * D * (n_det_rows * (w.window_len + w.n_global) + n_glob_rows * w.n_global)
+
+
+def time_oracle(w, budget_s=15.0, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload (one head):
+    whole windows of detail rows plus 128-row blocks of global rows, added
+    until about ``budget_s`` of CPU work. Returns (TFLOP/s, cores, sample)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    orc = oracle.Oracle()
+    cores = orc.max_threads()
+    rng = np.random.default_rng(seed)
+    D, L, G, N = w.head_dim, w.window_len, w.n_global, w.n_detail
+    kg = rng.standard_normal((G, D))
+    vg = rng.standard_normal((G, D))
+    flops = 0
+    t_total = 0.0
+    det_rows = glob_rows = 0
+    while t_total < budget_s:
+        if N:
+            k = rng.standard_normal((L, D))
+            v = rng.standard_normal((L, D))
+            q = rng.standard_normal((L, D))
+            ids = np.arange(L, dtype=np.int64)
+            t0 = time.perf_counter()
+            orc.attention_head(N, L, G, w.softmax_scale, k, v, 0, kg, vg, ids, q, cores)
+            t_total += time.perf_counter() - t0
+            det_rows += L
+        if G:
+            q = rng.standard_normal((128, D))
+            ids = N + np.arange(128, dtype=np.int64)
+            t0 = time.perf_counter()
+            orc.attention_head(N, max(L, 1), G, w.softmax_scale, None, None, 0, kg, vg, ids,
+                               q, cores)
+            t_total += time.perf_counter() - t0
+            glob_rows += 128
+        if t_total > 2 * budget_s:
+            break
+    flops = oracle_sample_flops(w, det_rows, glob_rows)
+    sample = (f"{det_rows} detail rows (whole windows) + {glob_rows} global rows of one head, "
+              f"{t_total:.1f} s of fp64 oracle work")
+    return flops / t_total / 1e12, cores, sample, t_total
+
+
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def config_of(w, world):
+    c = {"workload": w.name, "detail_grid": list(w.grid), "cube": list(w.cube),
+         "global_grid": list(w.global_grid), "n_detail": w.n_detail, "window_len": w.window_len,
+         "n_global": w.n_global, "heads": w.heads, "head_dim": w.head_dim,
+         "rope_split": list(w.split), "detail_scales": list(w.detail_scales),
+         "global_scales": list(w.global_scales), "batch_per_gpu": 1,
+         "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"}
+    per_tensor = max(w.n_detail, w.n_global) * w.heads * w.head_dim * w.elem_bytes
+    c["l2"] = (f"inputs larger than L2 ({per_tensor / 1e6:.0f} MB per tensor)"
+               if per_tensor > 126e6 else "inputs smaller than L2; no flush")
+    return c
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    times, flops_total = [], 0
+    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        tf, cores, sample, t = time_oracle(w, budget_s=budget, seed=i)
+        if i >= args.warmup:
+            times.append(tf)
+    value = statistics.mean(times)
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference", "config": config_of(w, world),
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": sample + " per step"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(out), flush=True)
+
+
+def run_atlas(args, world, rank, local):
+    from video_dit_windowed_b200 import atlas, build
+    if not os.path.exists(atlas.LIB_PATH):
+        build.build()
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        path = Path(w, dev, stream)
+    torch.cuda.synchronize(dev)
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize(dev)
+    code = atlas.last_device_error(stream)
+    if code:
+        raise RuntimeError(f"device error word 0x{code:x} after warm-up")
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start.record(stream)
+    for i in range(args.steps):
+        path.step(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    elapsed = start.elapsed_time(stop)
+    phases = {"reorder": [], "rope_g": [], "attn": [], "unorder": []}
+    for ev in evs:
+        for k, v in Path.phase_ms(ev).items():
+            phases[k].append(v)
+    elapsed = max_over_ranks(elapsed, world)
+    code = atlas.last_device_error(stream)
+    if code:
+        raise RuntimeError(f"device error word 0x{code:x} in the timed region")
+
+    # end to end through the C-ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(path, w, dev, stream, args, world)
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    ms = elapsed / args.steps
+    flops = w.unmasked_flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    attn_ms = statistics.median(phases["attn"])
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    b_d, b_g = bytes_reorder_rope(w)
+    rr_ms = statistics.median(phases["reorder"]) + statistics.median(phases["rope_g"])
+    rr_gbs = (b_d + b_g) / (rr_ms * 1e-3) / 1e9 if rr_ms > 0 else None
+    un_ms = statistics.median(phases["unorder"])
+    un_bytes = 2 * w.n_detail * w.heads * w.head_dim * w.elem_bytes
+    traffic = measured_traffic()
+    peak_tf = pk["bf16_tflops_sustained"]
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, world),
+        "attn_tflops": attn_tf, "attn_ms": attn_ms,
+        "attn_frac_of_bf16_peak": {"sustained": attn_tf / pk["bf16_tflops_sustained"],
+                                   "burst": attn_tf / pk["bf16_tflops"], "peaks": pk_kind},
+        "reorder_rope_gbs": rr_gbs, "reorder_rope_ms": rr_ms,
+        "reorder_rope_frac_of_hbm": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
+        "unorder_gbs": un_bytes / (un_ms * 1e-3) / 1e9 if un_ms > 0 else None,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": attn_tf,
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
+                     "peak_kind": f"{pk_kind} bf16 sustained",
+                     "traffic": traffic["bytes_per_launch"] if traffic else None},
+        "roofline_reorder_rope": {"bound": "hbm", "achieved": rr_gbs, "peak": pk["hbm_gbs"],
+                                  "unit": "GB/s",
+                                  "frac": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
+                                  "peak_kind": f"{pk_kind} copy"},
+        "gpu_launches": path.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        out["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        tf, cores, sample, _ = time_oracle(w, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    print(json.dumps(out), flush=True)
+
+
+def run_e2e(path, w, dev, stream, args, world):
+    """Same step, but inputs start in pinned host memory and the outputs end
+    there: H2D of the six raster tensors, the seven calls, D2H of O_d and O_g."""
+    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+            for k, v in path.x.items()}
+    for k in host:
+        host[k].copy_(path.x[k].cpu())
+    out_d = torch.empty(path.o_raster.shape, dtype=path.o_raster.dtype, pin_memory=True)
+    out_g = torch.empty(path.o_g.shape, dtype=path.o_g.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_d.numel() * out_d.element_size() + out_g.numel() * out_g.element_size()
+
+    def one():
+        with torch.cuda.stream(stream):
+            for k in host:
+                path.x[k].copy_(host[k], non_blocking=True)
+            path.step()
+            out_d.copy_(path.o_raster, non_blocking=True)
+            out_g.copy_(path.o_g, non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 10))
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    return {"value": world * w.unmasked_flops() / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="atlas", choices=["atlas", "reference"])
+    ap.add_argument("--workload", default="720p", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_atlas(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * atlas.h -- C-ABI of libatlas.so: the B200 (sm_100a) hot path of AtlasVid's
+ * detail-branch hierarchical locality-preserving attention.
+ *
+ * The path has four steps (page titles and sections cited at each call):
+ *   (1) cube reorder of the latent token grid, and its exact inverse;
+ *   (2) 3D rotary position embedding with per-axis position scales (the
+ *       temporal scale r_t; global-proxy coordinates mapped onto the detail
+ *       grid);
+ *   (3) window attention over the reordered sequence, and
+ *   (4) the asymmetric global-local attention,
+ * where (3) and (4) are one call sharing one softmax per query row.
+ *
+ * Conventions for every call:
+ *   - Tensors are row-major [rows, heads, head_dim], batch 1, contiguous.
+ *     A detail grid T x H x W is stored in raster order, row
+ *     r = (t*H + h)*W + w, unless the call says "cube order".
+ *   - Every pointer is a device pointer owned by the caller, 16-byte
+ *     aligned. The library allocates no tensor memory. It caches RoPE
+ *     cos/sin tables in device memory (freed by atlas_release_caches) and
+ *     keeps one device error word.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *     A status other than ATLAS_OK means nothing was launched, except
+ *     ATLAS_ERR_CUDA, which reports a failed launch or copy.
+ *   - The library runs on compute capability 10.0 (B200, sm_100a) only.
+ */
+#ifndef ATLAS_H
+#define ATLAS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *atlas_stream_t;
+
+typedef enum {
+    ATLAS_OK = 0,
+    ATLAS_ERR_NULL = 1,        /* a required pointer is NULL                      */
+    ATLAS_ERR_SHAPE = 2,       /* sizes inconsistent (cube does not divide grid,  */
+                               /* n_detail not a multiple of window_len, <0 ...)  */
+    ATLAS_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                */
+    ATLAS_ERR_UNSUPPORTED = 4, /* dtype / head_dim / RoPE split not supported     */
+    ATLAS_ERR_ALIAS = 5,       /* input and output overlap where not allowed      */
+    ATLAS_ERR_CUDA = 6,        /* a CUDA runtime call or a launch failed          */
+    ATLAS_ERR_TIMEOUT = 7,     /* a kernel's bounded wait expired (device word)   */
+    ATLAS_ERR_DEVICE = 8       /* no usable device, or not compute capability 10.0 */
+} atlas_status;
+
+typedef enum {
+    ATLAS_BF16 = 0,            /* bfloat16 I/O, fp32 arithmetic                   */
+    ATLAS_FP32 = 1             /* float32 I/O, fp32 arithmetic                    */
+} atlas_dtype;
+
+/* Extents of a token grid: T frames, H rows, W columns. */
+typedef struct { int64_t T, H, W; } atlas_grid3;
+
+/* Extents of one spatiotemporal cube (window). */
+typedef struct { int32_t ct, ch, cw; } atlas_cube3;
+
+/* 3D RoPE parameters. head_dim = d_t + d_h + d_w, each even and > 0 or 0.
+ * The segments are contiguous in that order. A token at grid index (t,h,w)
+ * has position (t*scale_t, h*scale_h, w*scale_w). Channel pair (2k, 2k+1)
+ * of a segment of width d rotates by angle position * theta^(-2k/d). */
+typedef struct {
+    double theta;
+    int32_t d_t, d_h, d_w;
+    double scale_t, scale_h, scale_w;
+} atlas_rope;
+
+/*
+ * atlas_cube_reorder -- step (1), with step (2) fused when rope != NULL.
+ *
+ * Passage: "Technische Samenvatting: AtlasVid" (gist.science; same text in
+ * the French and Portuguese editions), Methodologie 1, Fase 2: the latent
+ * video volume is cut into spatiotemporal cubes and the tokens are reordered
+ * so the tokens of one cube are contiguous. With rope != NULL the rows are
+ * also rotated by 3D RoPE (Methodologie 1, Fase 1: temporal index times
+ * r_t; Methodologie 2, position alignment: coordinates times the resolution
+ * ratios), at the token's grid position.
+ *
+ * src: [T*H*W, heads, head_dim] in raster order. dst: same size, cube order:
+ * cubes in raster order over the (T/ct) x (H/ch) x (W/cw) cube grid, the
+ * L = ct*ch*cw tokens of a cube in raster order over the cube, position
+ * j = cube*L + local. Without rope the copy is bit-exact. With rope the
+ * rotation runs in fp32 on fp64-built, fp32-rounded cos/sin and rounds once
+ * to dtype (round to nearest even).
+ * Errors: NULL pointers; a cube extent that does not divide the grid or is
+ * < 1 (SHAPE); head_dim not even or the RoPE split not summing to head_dim
+ * or odd (UNSUPPORTED); rows not a multiple of 16 bytes, or misaligned
+ * pointers (ALIGN); src and dst overlapping (ALIAS).
+ */
+atlas_status atlas_cube_reorder(const void *src, void *dst, atlas_grid3 grid,
+                                atlas_cube3 cube, int32_t heads,
+                                int32_t head_dim, atlas_dtype dtype,
+                                const atlas_rope *rope, atlas_stream_t stream);
+
+/*
+ * atlas_cube_unorder -- the exact inverse of step (1).
+ *
+ * Passage: as atlas_cube_reorder (the permutation is undone after the
+ * attention so the output is back in raster order).
+ * src: cube order, dst: raster order, both [T*H*W, heads, head_dim]. A
+ * byte copy: unorder(reorder(x)) == x for every bit pattern.
+ * Errors: as atlas_cube_reorder (no RoPE).
+ */
+atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
+                                atlas_cube3 cube, int32_t heads,
+                                int32_t head_dim, atlas_dtype dtype,
+                                atlas_stream_t stream);
+
+/*
+ * atlas_rope3d -- step (2) on raster-ordered tokens (the global proxy).
+ *
+ * Passage: "Technische Samenvatting: AtlasVid", Methodologie 1, Fase 1
+ * (temporally scaled RoPE, factor r_t) and Methodologie 2, position
+ * alignment (global-proxy RoPE coordinates scaled by W/w, H/h, T/t onto the
+ * high-resolution grid); abstract of "AtlasVid: Efficient Ultra-High-
+ * Resolution Long Video Generation via Decoupled Global-Local Modeling".
+ *
+ * src, dst: [T*H*W, heads, head_dim], raster order. dst may equal src
+ * (in place); partial overlap is ALIAS. Numerics as atlas_cube_reorder.
+ */
+atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid,
+                          int32_t heads, int32_t head_dim, atlas_dtype dtype,
+                          const atlas_rope *rope, atlas_stream_t stream);
+
+/*
+ * atlas_local_global_attn -- steps (3) and (4) in one pass.
+ *
+ * Passages: "Technische Samenvatting: AtlasVid", Methodologie 1, Fase 2
+ * (window attention over the reordered sequence, windows = geometric
+ * neighbourhoods) and Methodologie 2, asymmetric hierarchical attention
+ * (X_global and X_detail concatenated; X_global attends only to itself;
+ * X_detail attends to its own neighbourhood and to the global tokens;
+ * global -> detail masked with -inf).
+ *
+ * One softmax per query row over its allowed keys:
+ *   detail row q (0 <= q < n_detail, cube order): detail keys of its own
+ *     window [floor(q/window_len)*window_len, +window_len) and all
+ *     n_global global keys;
+ *   global row g: all n_global global keys, no detail key.
+ * q_d, k_d, v_d: [n_detail, heads, head_dim] in cube order (n_detail may be
+ *   0; the pointers are then ignored). n_detail % window_len == 0.
+ * q_g, k_g, v_g: [n_global, heads, head_dim] (n_global may be 0).
+ * o_d, o_g: outputs, same shapes and order as q_d, q_g.
+ * lse: optional (NULL to skip), fp32 [heads, n_detail + n_global]: natural
+ *   log of each row's softmax denominator over logits scale*<q,k>; detail
+ *   rows first (cube order), then global rows.
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ * dtype BF16: tcgen05 tensor-core kernel; S and O accumulate in fp32, P is
+ *   rounded to bf16 before the P*V product, O rounded to bf16 RNE.
+ * dtype FP32: SIMT fp32 kernel.
+ * head_dim must be 64 or 128.
+ * Errors: NULL (required pointer), SHAPE, ALIGN, UNSUPPORTED; a kernel
+ * whose bounded internal wait expires sets the device error word (read it
+ * with atlas_last_device_error) and finishes without completing the rows.
+ */
+atlas_status atlas_local_global_attn(
+    const void *q_d, const void *k_d, const void *v_d, int64_t n_detail,
+    int64_t window_len, const void *q_g, const void *k_g, const void *v_g,
+    int64_t n_global, int32_t heads, int32_t head_dim, float softmax_scale,
+    atlas_dtype dtype, void *o_d, void *o_g, float *lse,
+    atlas_stream_t stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char *atlas_status_string(atlas_status status);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word of the
+ * current device into *code (0 = no kernel reported an error). Returns
+ * ATLAS_ERR_TIMEOUT when the word is non-zero, ATLAS_ERR_CUDA when the
+ * synchronisation itself failed, ATLAS_OK otherwise.
+ */
+atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *code);
+
+/* Free the cached RoPE tables of every device (synchronises the device). */
+atlas_status atlas_release_caches(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t atlas_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATLAS_H */

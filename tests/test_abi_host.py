@@ -1,0 +1,136 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must build, load, export exactly the symbols ``include/atlas.h``
+declares, and reject bad arguments on the host before any CUDA call. Fake
+pointer values are never dereferenced: every case below fails validation
+first.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from video_dit_windowed_b200 import atlas, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "atlas.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return atlas.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(atlas_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for want in ("atlas_cube_reorder", "atlas_cube_unorder", "atlas_rope3d",
+                 "atlas_local_global_attn", "atlas_status_string"):
+        assert want in names
+
+
+def test_exports_match_header(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", atlas.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = sorted({l.split()[-1] for l in out.splitlines()
+                       if l.split()[-2:-1] == ["T"] and l.split()[-1].startswith("atlas_")})
+    assert exported == declared_functions()
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        s = atlas.status_string(code)
+        assert s.startswith("ATLAS_")
+    assert "UNKNOWN" in atlas.status_string(99)
+    assert atlas.version() >= 100
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+G = atlas.Grid3(4, 8, 8)
+C = atlas.Cube3(2, 4, 4)
+
+
+def reorder(lib, src, dst, grid=G, cube=C, heads=2, hd=64, dt=atlas.FP32, rope=None):
+    return lib.atlas_cube_reorder(src, dst, grid, cube, heads, hd, dt,
+                                  ctypes.byref(rope) if rope else None, None)
+
+
+def test_reorder_validation(lib):
+    big = FAKE + (1 << 30)
+    assert reorder(lib, None, big) == atlas.ERR_NULL
+    assert reorder(lib, FAKE, None) == atlas.ERR_NULL
+    assert reorder(lib, FAKE, big, cube=atlas.Cube3(3, 4, 4)) == atlas.ERR_SHAPE
+    assert reorder(lib, FAKE, big, cube=atlas.Cube3(0, 4, 4)) == atlas.ERR_SHAPE
+    assert reorder(lib, FAKE, big, grid=atlas.Grid3(0, 8, 8)) == atlas.ERR_SHAPE
+    assert reorder(lib, FAKE + 8, big) == atlas.ERR_ALIGN
+    assert reorder(lib, FAKE, big, hd=6, dt=atlas.BF16) == atlas.ERR_ALIGN
+    assert reorder(lib, FAKE, FAKE + 64) == atlas.ERR_ALIAS
+    assert reorder(lib, FAKE, FAKE) == atlas.ERR_ALIAS
+    assert reorder(lib, FAKE, big, dt=7) == atlas.ERR_UNSUPPORTED
+    bad_split = atlas.make_rope(10000, (16, 24, 22), (1, 1, 1))
+    assert reorder(lib, FAKE, big, rope=bad_split) == atlas.ERR_UNSUPPORTED
+    odd_split = atlas.make_rope(10000, (15, 25, 24), (1, 1, 1))
+    assert reorder(lib, FAKE, big, rope=odd_split) == atlas.ERR_UNSUPPORTED
+    bad_theta = atlas.make_rope(0.0, (16, 24, 24), (1, 1, 1))
+    assert reorder(lib, FAKE, big, rope=bad_theta) == atlas.ERR_UNSUPPORTED
+    huge = atlas.Grid3(1 << 16, 1 << 16, 1)
+    assert reorder(lib, FAKE, big, grid=huge, cube=atlas.Cube3(1, 1, 1)) == atlas.ERR_SHAPE
+
+
+def test_unorder_and_rope_validation(lib):
+    big = FAKE + (1 << 30)
+    assert lib.atlas_cube_unorder(None, big, G, C, 2, 64, atlas.FP32, None) == atlas.ERR_NULL
+    assert lib.atlas_cube_unorder(FAKE, big, G, atlas.Cube3(2, 3, 4), 2, 64, atlas.FP32,
+                                  None) == atlas.ERR_SHAPE
+    assert lib.atlas_cube_unorder(FAKE, FAKE + 16, G, C, 2, 64, atlas.FP32,
+                                  None) == atlas.ERR_ALIAS
+    rope = atlas.make_rope(10000, (16, 24, 24), (1, 1, 1))
+    assert lib.atlas_rope3d(FAKE, big, G, 2, 64, atlas.FP32, None, None) == atlas.ERR_NULL
+    assert lib.atlas_rope3d(FAKE, FAKE + 16, G, 2, 64, atlas.FP32, ctypes.byref(rope),
+                            None) == atlas.ERR_ALIAS
+    assert lib.atlas_rope3d(FAKE + 4, FAKE + 4, G, 2, 64, atlas.FP32, ctypes.byref(rope),
+                            None) == atlas.ERR_ALIGN
+
+
+def attn(lib, q_d=FAKE, k_d=FAKE + (1 << 28), v_d=FAKE + (2 << 28), n_d=256, L=32,
+         q_g=FAKE + (3 << 28), k_g=FAKE + (4 << 28), v_g=FAKE + (5 << 28), n_g=32, heads=2,
+         hd=64, dt=atlas.BF16, o_d=FAKE + (6 << 28), o_g=FAKE + (7 << 28), lse=None):
+    return lib.atlas_local_global_attn(q_d, k_d, v_d, n_d, L, q_g, k_g, v_g, n_g, heads, hd,
+                                       0.0, dt, o_d, o_g, lse, None)
+
+
+def test_attention_validation(lib):
+    assert attn(lib, q_d=None) == atlas.ERR_NULL
+    assert attn(lib, o_g=None) == atlas.ERR_NULL
+    assert attn(lib, n_d=250) == atlas.ERR_SHAPE          # not a multiple of L
+    assert attn(lib, L=0) == atlas.ERR_SHAPE
+    assert attn(lib, n_d=-1) == atlas.ERR_SHAPE
+    assert attn(lib, heads=0) == atlas.ERR_SHAPE
+    assert attn(lib, hd=96) == atlas.ERR_UNSUPPORTED
+    assert attn(lib, dt=5) == atlas.ERR_UNSUPPORTED
+    assert attn(lib, k_g=FAKE + (4 << 28) + 8) == atlas.ERR_ALIGN
+    assert attn(lib, lse=FAKE + 2) == atlas.ERR_ALIGN
+    assert attn(lib, o_d=FAKE + (1 << 28)) == atlas.ERR_ALIAS   # o_d over k_d
+    assert attn(lib, o_g=FAKE + (6 << 28)) == atlas.ERR_ALIAS   # o_g over o_d
+    # Absent sides: their pointers are not required.
+    assert attn(lib, n_d=0, q_d=None, k_d=None, v_d=None, o_d=None, n_g=0,
+                q_g=None, k_g=None, v_g=None, o_g=None) == atlas.OK
+
+
+def test_valid_call_without_gpu_reports_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert attn(lib) == atlas.ERR_DEVICE
+    big = FAKE + (1 << 30)
+    assert reorder(lib, FAKE, big) == atlas.ERR_DEVICE

@@ -1,0 +1,200 @@
+"""ctypes binding of ``libatlas.so`` (declared in ``include/atlas.h``).
+
+Argument marshalling only: shapes, dtypes and device pointers are read off
+torch tensors (torch is used for device memory and streams) and passed to the
+C-ABI; every step of the path runs in the library's CUDA kernels. There is no
+CPU fallback: if the library has not been built, the first call raises.
+
+Passages (page title, section) for each call are given in the header; in
+short: "Technische Samenvatting: AtlasVid" (gist.science), Methodologie 1
+Fase 1 (temporally scaled RoPE), Fase 2 (cube reorder, window attention) and
+Methodologie 2 (asymmetric hierarchical attention, position alignment).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libatlas.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_ALIAS, ERR_CUDA, \
+    ERR_TIMEOUT, ERR_DEVICE = range(9)
+BF16, FP32 = 0, 1
+
+
+class Grid3(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64)]
+
+
+class Cube3(ctypes.Structure):
+    _fields_ = [("ct", ctypes.c_int32), ("ch", ctypes.c_int32), ("cw", ctypes.c_int32)]
+
+
+class Rope(ctypes.Structure):
+    _fields_ = [("theta", ctypes.c_double), ("d_t", ctypes.c_int32), ("d_h", ctypes.c_int32),
+                ("d_w", ctypes.c_int32), ("scale_t", ctypes.c_double),
+                ("scale_h", ctypes.c_double), ("scale_w", ctypes.c_double)]
+
+
+def make_rope(theta, split, scales) -> Rope:
+    d_t, d_h, d_w = (int(v) for v in split)
+    s_t, s_h, s_w = (float(v) for v in scales)
+    return Rope(float(theta), d_t, d_h, d_w, s_t, s_h, s_w)
+
+
+class AtlasError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+
+
+def _declare(lib):
+    lib.atlas_cube_reorder.restype = ctypes.c_int
+    lib.atlas_cube_reorder.argtypes = [_vp, _vp, Grid3, Cube3, _i32, _i32, ctypes.c_int,
+                                       ctypes.POINTER(Rope), _vp]
+    lib.atlas_cube_unorder.restype = ctypes.c_int
+    lib.atlas_cube_unorder.argtypes = [_vp, _vp, Grid3, Cube3, _i32, _i32, ctypes.c_int, _vp]
+    lib.atlas_rope3d.restype = ctypes.c_int
+    lib.atlas_rope3d.argtypes = [_vp, _vp, Grid3, _i32, _i32, ctypes.c_int,
+                                 ctypes.POINTER(Rope), _vp]
+    lib.atlas_local_global_attn.restype = ctypes.c_int
+    lib.atlas_local_global_attn.argtypes = [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64,
+                                            _i32, _i32, ctypes.c_float, ctypes.c_int, _vp, _vp,
+                                            _vp, _vp]
+    lib.atlas_status_string.restype = ctypes.c_char_p
+    lib.atlas_status_string.argtypes = [ctypes.c_int]
+    lib.atlas_last_device_error.restype = ctypes.c_int
+    lib.atlas_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.atlas_release_caches.restype = ctypes.c_int
+    lib.atlas_release_caches.argtypes = []
+    lib.atlas_version.restype = ctypes.c_int32
+    lib.atlas_version.argtypes = []
+    return lib
+
+
+def lib():
+    """The loaded library. Raises if ``libatlas.so`` has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m video_dit_windowed_b200.build` (no CPU fallback exists)")
+            _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().atlas_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise AtlasError(status, where)
+
+
+# ---------------------------------------------------------------------------
+# torch-facing wrappers (torch only supplies pointers, shapes and streams)
+# ---------------------------------------------------------------------------
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t, stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(t.device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def cube_reorder(src, dst, grid, cube, rope: Rope | None = None, stream=None):
+    """Raster -> cube order of ``src`` [T*H*W, heads, head_dim] into ``dst``;
+    with ``rope`` the rows are also rotated by 3D RoPE at their grid position."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_reorder(
+        _ptr(src), _ptr(dst), Grid3(*grid), Cube3(*cube), heads, hd, _dtype_code(src),
+        ctypes.byref(rope) if rope is not None else None, _stream(src, stream))
+    _check(st, "atlas_cube_reorder")
+    return dst
+
+
+def cube_unorder(src, dst, grid, cube, stream=None):
+    """Cube order -> raster order (exact inverse of ``cube_reorder``)."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_unorder(_ptr(src), _ptr(dst), Grid3(*grid), Cube3(*cube), heads, hd,
+                                  _dtype_code(src), _stream(src, stream))
+    _check(st, "atlas_cube_unorder")
+    return dst
+
+
+def rope3d(src, dst, grid, rope: Rope, stream=None):
+    """3D RoPE of raster-ordered tokens (``dst`` may be ``src``)."""
+    n, heads, hd = src.shape
+    st = lib().atlas_rope3d(_ptr(src), _ptr(dst), Grid3(*grid), heads, hd, _dtype_code(src),
+                            ctypes.byref(rope), _stream(src, stream))
+    _check(st, "atlas_rope3d")
+    return dst
+
+
+def local_global_attn(q_d, k_d, v_d, window_len, q_g, k_g, v_g, o_d, o_g, lse=None,
+                      softmax_scale: float = 0.0, stream=None):
+    """Asymmetric global-local attention; detail tensors in cube order.
+    ``q_d`` (or ``q_g``) may have 0 rows. Returns (o_d, o_g, lse)."""
+    ref = q_d if q_d is not None and q_d.shape[0] > 0 else q_g
+    heads, hd = ref.shape[1], ref.shape[2]
+    n_d = q_d.shape[0] if q_d is not None else 0
+    n_g = q_g.shape[0] if q_g is not None else 0
+    nz = lambda t, n: _ptr(t) if (t is not None and n > 0) else None
+    st = lib().atlas_local_global_attn(
+        nz(q_d, n_d), nz(k_d, n_d), nz(v_d, n_d), n_d, int(window_len),
+        nz(q_g, n_g), nz(k_g, n_g), nz(v_g, n_g), n_g, heads, hd, float(softmax_scale),
+        _dtype_code(ref), nz(o_d, n_d), nz(o_g, n_g), _ptr(lse), _stream(ref, stream))
+    _check(st, "atlas_local_global_attn")
+    return o_d, o_g, lse
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise and read/clear the device error word (0 = clean)."""
+    import torch
+    s = ctypes.c_void_p(stream.cuda_stream if stream is not None
+                        else torch.cuda.current_stream().cuda_stream)
+    code = ctypes.c_uint32(0)
+    st = lib().atlas_last_device_error(s, ctypes.byref(code))
+    if st not in (OK, ERR_TIMEOUT):
+        raise AtlasError(st, "atlas_last_device_error")
+    return int(code.value)
+
+
+def release_caches():
+    _check(lib().atlas_release_caches(), "atlas_release_caches")
+
+
+def version() -> int:
+    return int(lib().atlas_version())

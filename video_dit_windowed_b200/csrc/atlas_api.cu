@@ -1,0 +1,217 @@
+// atlas_api.cu -- the C-ABI of libatlas.so: argument validation and dispatch.
+//
+// Every entry point checks its arguments on the host and returns a status
+// without launching anything when they are bad. See include/atlas.h for the
+// contract of each call and the passages it implements.
+#include <cmath>
+#include <mutex>
+
+#include "atlas_internal.cuh"
+
+namespace atlas {
+
+__device__ uint32_t g_device_error = 0;
+
+uint32_t *device_error_word() {
+    static std::mutex mu;
+    static uint32_t *addr[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<uint32_t *>(p);
+    }
+    return addr[dev];
+}
+
+bool current_device(DeviceInfo *out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo &c = cache[dev];
+    if (c.device != dev) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return false;
+        c.device = dev;
+        c.sm_count = prop.multiProcessorCount;
+        c.major = prop.major;
+        c.minor = prop.minor;
+        c.smem_optin = prop.sharedMemPerBlockOptin;
+    }
+    *out = c;
+    return c.major == 10 && c.minor == 0;
+}
+
+namespace {
+
+int elem_bytes(atlas_dtype dt) {
+    switch (dt) {
+        case ATLAS_BF16: return 2;
+        case ATLAS_FP32: return 4;
+    }
+    return 0;
+}
+
+// Row-index arithmetic in the kernels is 32-bit: the token count and every
+// intermediate index stay below 2^31.
+constexpr int64_t kMaxRows = (1ll << 31) - 1;
+
+atlas_status check_grid(atlas_grid3 g, int32_t heads, int32_t head_dim, atlas_dtype dt) {
+    if (g.T < 1 || g.H < 1 || g.W < 1 || heads < 1 || head_dim < 1) return ATLAS_ERR_SHAPE;
+    if (g.T > kMaxRows || g.H > kMaxRows || g.W > kMaxRows) return ATLAS_ERR_SHAPE;
+    if (g.T * g.H > kMaxRows || g.T * g.H * g.W > kMaxRows) return ATLAS_ERR_SHAPE;
+    const int eb = elem_bytes(dt);
+    if (eb == 0) return ATLAS_ERR_UNSUPPORTED;
+    if ((static_cast<int64_t>(head_dim) * eb) % 16 != 0) return ATLAS_ERR_ALIGN;
+    return ATLAS_OK;
+}
+
+atlas_status check_cube(atlas_grid3 g, atlas_cube3 c) {
+    if (c.ct < 1 || c.ch < 1 || c.cw < 1) return ATLAS_ERR_SHAPE;
+    if (g.T % c.ct || g.H % c.ch || g.W % c.cw) return ATLAS_ERR_SHAPE;
+    return ATLAS_OK;
+}
+
+atlas_status check_rope(const atlas_rope &r, int32_t head_dim, atlas_dtype dt) {
+    if (r.d_t < 0 || r.d_h < 0 || r.d_w < 0) return ATLAS_ERR_UNSUPPORTED;
+    if ((r.d_t | r.d_h | r.d_w) & 1) return ATLAS_ERR_UNSUPPORTED;
+    if (r.d_t + r.d_h + r.d_w != head_dim) return ATLAS_ERR_UNSUPPORTED;
+    if (!(r.theta > 0.0) || !std::isfinite(r.theta)) return ATLAS_ERR_UNSUPPORTED;
+    if (!std::isfinite(r.scale_t) || !std::isfinite(r.scale_h) || !std::isfinite(r.scale_w))
+        return ATLAS_ERR_UNSUPPORTED;
+    // The kernel gives each thread one 16-byte slot of a head: the slots of a
+    // head must tile a 128-thread group.
+    const int vph = head_dim * elem_bytes(dt) / 16;
+    if (vph < 1 || vph > 128 || (vph & (vph - 1))) return ATLAS_ERR_UNSUPPORTED;
+    return ATLAS_OK;
+}
+
+}  // namespace
+}  // namespace atlas
+
+using namespace atlas;
+
+ATLAS_API atlas_status atlas_cube_reorder(const void *src, void *dst, atlas_grid3 grid,
+                                          atlas_cube3 cube, int32_t heads, int32_t head_dim,
+                                          atlas_dtype dtype, const atlas_rope *rope,
+                                          atlas_stream_t stream) {
+    if (!src || !dst) return ATLAS_ERR_NULL;
+    atlas_status st = check_grid(grid, heads, head_dim, dtype);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
+    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
+                         elem_bytes(dtype);
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), 0, rope};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ATLAS_API atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
+                                          atlas_cube3 cube, int32_t heads, int32_t head_dim,
+                                          atlas_dtype dtype, atlas_stream_t stream) {
+    if (!src || !dst) return ATLAS_ERR_NULL;
+    atlas_status st = check_grid(grid, heads, head_dim, dtype);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
+    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
+                         elem_bytes(dtype);
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), 1, nullptr};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ATLAS_API atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid, int32_t heads,
+                                    int32_t head_dim, atlas_dtype dtype, const atlas_rope *rope,
+                                    atlas_stream_t stream) {
+    if (!src || !dst || !rope) return ATLAS_ERR_NULL;
+    atlas_status st = check_grid(grid, heads, head_dim, dtype);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
+    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
+                         elem_bytes(dtype);
+    if (src != dst && ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, 1, 1, 1,
+                  heads, head_dim, elem_bytes(dtype), 2, rope};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d, const void *v_d,
+                                               int64_t n_detail, int64_t window_len,
+                                               const void *q_g, const void *k_g, const void *v_g,
+                                               int64_t n_global, int32_t heads, int32_t head_dim,
+                                               float softmax_scale, atlas_dtype dtype, void *o_d,
+                                               void *o_g, float *lse, atlas_stream_t stream) {
+    if (n_detail < 0 || n_global < 0 || heads < 1) return ATLAS_ERR_SHAPE;
+    if (n_detail > 0 && (window_len < 1 || n_detail % window_len != 0)) return ATLAS_ERR_SHAPE;
+    if (n_detail + n_global > kMaxRows || static_cast<int64_t>(heads) > 65535)
+        return ATLAS_ERR_SHAPE;
+    if (n_detail > 0 && (!q_d || !k_d || !v_d || !o_d)) return ATLAS_ERR_NULL;
+    if (n_global > 0 && (!q_g || !k_g || !v_g || !o_g)) return ATLAS_ERR_NULL;
+    if (elem_bytes(dtype) == 0) return ATLAS_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q_d, k_d, v_d, o_d, q_g, k_g, v_g, o_g};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return ATLAS_ERR_ALIGN;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATLAS_ERR_ALIGN;
+    // Outputs must not overlap inputs.
+    const size_t eb = static_cast<size_t>(elem_bytes(dtype)) * heads * head_dim;
+    const size_t bd = eb * static_cast<size_t>(n_detail), bg = eb * static_cast<size_t>(n_global);
+    const void *ins[] = {q_d, k_d, v_d, q_g, k_g, v_g};
+    const size_t in_bytes[] = {bd, bd, bd, bg, bg, bg};
+    for (int i = 0; i < 6; ++i) {
+        if (!ins[i] || !in_bytes[i]) continue;
+        if (o_d && bd && ranges_overlap(ins[i], in_bytes[i], o_d, bd)) return ATLAS_ERR_ALIAS;
+        if (o_g && bg && ranges_overlap(ins[i], in_bytes[i], o_g, bg)) return ATLAS_ERR_ALIAS;
+    }
+    if (o_d && o_g && bd && bg && ranges_overlap(o_d, bd, o_g, bg)) return ATLAS_ERR_ALIAS;
+    if (n_detail + n_global == 0) return ATLAS_OK;
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    float scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(head_dim));
+    AttnArgs a{q_d, k_d, v_d, n_detail, window_len, q_g, k_g, v_g, n_global,
+               heads, head_dim, scale, o_d, o_g, lse};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dtype == ATLAS_BF16 ? launch_attn_tc_bf16(a, s) : launch_attn_simt_f32(a, s);
+}
+
+ATLAS_API const char *atlas_status_string(atlas_status status) {
+    switch (status) {
+        case ATLAS_OK: return "ATLAS_OK";
+        case ATLAS_ERR_NULL: return "ATLAS_ERR_NULL: a required pointer is NULL";
+        case ATLAS_ERR_SHAPE: return "ATLAS_ERR_SHAPE: inconsistent sizes";
+        case ATLAS_ERR_ALIGN: return "ATLAS_ERR_ALIGN: pointer or row not 16-byte aligned";
+        case ATLAS_ERR_UNSUPPORTED: return "ATLAS_ERR_UNSUPPORTED: dtype, head_dim or RoPE split";
+        case ATLAS_ERR_ALIAS: return "ATLAS_ERR_ALIAS: input and output overlap";
+        case ATLAS_ERR_CUDA: return "ATLAS_ERR_CUDA: a CUDA call or launch failed";
+        case ATLAS_ERR_TIMEOUT: return "ATLAS_ERR_TIMEOUT: a kernel's bounded wait expired";
+        case ATLAS_ERR_DEVICE: return "ATLAS_ERR_DEVICE: no compute capability 10.0 device";
+    }
+    return "ATLAS_ERR_UNKNOWN";
+}
+
+ATLAS_API atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *code) {
+    if (!code) return ATLAS_ERR_NULL;
+    *code = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATLAS_ERR_CUDA;
+    uint32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return ATLAS_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess)
+        return ATLAS_ERR_CUDA;
+    *code = v;
+    return v ? ATLAS_ERR_TIMEOUT : ATLAS_OK;
+}
+
+ATLAS_API atlas_status atlas_release_caches(void) { return release_rope_tables(); }
+
+ATLAS_API int32_t atlas_version(void) { return 100; }

@@ -1,0 +1,89 @@
+// atlas_internal.cuh -- shared declarations of libatlas.so (not installed).
+//
+// Device helpers here are thin inline-PTX wrappers around sm_100a
+// instructions (mbarrier, TMA, tcgen05) written for this library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/atlas.h"
+
+#define ATLAS_API extern "C" __attribute__((visibility("default")))
+
+namespace atlas {
+
+// ---------------------------------------------------------------------------
+// Device error word: kernels OR bits into it instead of trapping.
+// ---------------------------------------------------------------------------
+enum DeviceError : uint32_t {
+    kErrTimeoutProducer = 1u << 0,   // TMA producer wait expired
+    kErrTimeoutMma = 1u << 1,        // MMA issuer wait expired
+    kErrTimeoutSoftmax = 1u << 2,    // softmax / epilogue wait expired
+    kErrTimeoutTeardown = 1u << 3,   // teardown wait for in-flight work expired
+    kErrTmemAlloc = 1u << 4,         // tensor-memory allocation returned bad base
+};
+
+// Device address of the error word on the current device (host call; the
+// word is a __device__ variable of atlas_api.cu, reached by kernels of other
+// translation units through this pointer). NULL if it cannot be resolved.
+uint32_t *device_error_word();
+
+// Wall-clock limit of one bounded wait in a kernel, in nanoseconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side helpers shared by the launchers.
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int major = 0, minor = 0;
+    size_t smem_optin = 0;
+};
+
+// Current device's properties (cached per device). Returns false if no
+// usable device or not compute capability 10.0.
+bool current_device(DeviceInfo *out);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
+    uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Launchers (defined in the kernel files). Arguments are validated by the
+// C-ABI layer before these run.
+struct PermuteArgs {
+    const void *src;
+    void *dst;
+    int64_t T, H, W;
+    int32_t ct, ch, cw;
+    int32_t heads, head_dim, elem_bytes;
+    int mode;               // 0 reorder (raster -> cube), 1 unorder, 2 raster RoPE
+    const atlas_rope *rope; // may be NULL (pure permutation)
+};
+atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
+atlas_status release_rope_tables();
+
+struct AttnArgs {
+    const void *q_d, *k_d, *v_d;
+    int64_t n_detail, window_len;
+    const void *q_g, *k_g, *v_g;
+    int64_t n_global;
+    int32_t heads, head_dim;
+    float scale;
+    void *o_d, *o_g;
+    float *lse;
+};
+atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
+atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream);
+
+}  // namespace atlas

@@ -1,0 +1,111 @@
+// attn_simt.cu -- asymmetric local-global attention, fp32 I/O, SIMT fp32.
+//
+// Passages: as attn_tc.cu ("Technische Samenvatting: AtlasVid", Methodologie
+// 1 Fase 2 and Methodologie 2). This kernel serves fp32 tensors, whose
+// workloads here are small and launch-bound: one warp per (query row, head),
+// exact fp32 products, an online softmax with expf, keys streamed in order
+// (own window first, then the global keys).
+#include "atlas_internal.cuh"
+
+namespace atlas {
+namespace {
+
+constexpr int kWarps = 8;
+
+struct Params {
+    const float *q_d, *k_d, *v_d, *q_g, *k_g, *v_g;
+    float *o_d, *o_g, *lse;
+    int64_t N, L, G;
+    int32_t heads;
+    float scale;
+};
+
+template <int HD>
+__device__ __forceinline__ void accumulate_keys(const float *k, const float *v, int64_t k0,
+                                                int64_t k1, int64_t row_stride,
+                                                const float (&q)[HD / 32], float scale,
+                                                float &m, float &l, float (&o)[HD / 32]) {
+    const int lane = threadIdx.x & 31;
+    for (int64_t key = k0; key < k1; ++key) {
+        const float *kr = k + key * row_stride;
+        const float *vr = v + key * row_stride;
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < HD / 32; ++e) dot = fmaf(q[e], kr[lane + 32 * e], dot);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float s = dot * scale;
+        const float m_new = fmaxf(m, s);
+        const float corr = expf(m - m_new);
+        const float p = expf(s - m_new);
+        l = l * corr + p;
+#pragma unroll
+        for (int e = 0; e < HD / 32; ++e) o[e] = fmaf(p, vr[lane + 32 * e], o[e] * corr);
+        m = m_new;
+    }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const Params p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + threadIdx.x / 32;
+    const int head = blockIdx.y;
+    if (row >= p.N + p.G) return;
+    const bool detail = row < p.N;
+    const int64_t stride = static_cast<int64_t>(p.heads) * HD;
+    const float *qr = (detail ? p.q_d + row * stride : p.q_g + (row - p.N) * stride) + head * HD;
+    float q[HD / 32], o[HD / 32];
+#pragma unroll
+    for (int e = 0; e < HD / 32; ++e) {
+        q[e] = qr[lane + 32 * e];
+        o[e] = 0.f;
+    }
+    float m = -__builtin_huge_valf(), l = 0.f;
+    if (detail) {
+        const int64_t lo = (row / p.L) * p.L;
+        accumulate_keys<HD>(p.k_d + head * HD, p.v_d + head * HD, lo, lo + p.L, stride, q,
+                            p.scale, m, l, o);
+    }
+    if (p.G > 0)
+        accumulate_keys<HD>(p.k_g + head * HD, p.v_g + head * HD, 0, p.G, stride, q, p.scale, m,
+                            l, o);
+    float *out = (detail ? p.o_d + row * stride : p.o_g + (row - p.N) * stride) + head * HD;
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int e = 0; e < HD / 32; ++e) out[lane + 32 * e] = o[e] * inv;
+    if (p.lse != nullptr && lane == 0) p.lse[head * (p.N + p.G) + row] = m + logf(l);
+}
+
+template <int HD>
+atlas_status launch_hd(const Params &p, cudaStream_t stream) {
+    const int64_t rows = p.N + p.G;
+    if (rows == 0) return ATLAS_OK;
+    dim3 grid(static_cast<unsigned>((rows + kWarps - 1) / kWarps), static_cast<unsigned>(p.heads));
+    attn_simt_kernel<HD><<<grid, kWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+}  // namespace
+
+atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream) {
+    Params p{};
+    p.q_d = static_cast<const float *>(a.q_d);
+    p.k_d = static_cast<const float *>(a.k_d);
+    p.v_d = static_cast<const float *>(a.v_d);
+    p.q_g = static_cast<const float *>(a.q_g);
+    p.k_g = static_cast<const float *>(a.k_g);
+    p.v_g = static_cast<const float *>(a.v_g);
+    p.o_d = static_cast<float *>(a.o_d);
+    p.o_g = static_cast<float *>(a.o_g);
+    p.lse = a.lse;
+    p.N = a.n_detail;
+    p.L = a.n_detail > 0 ? a.window_len : 1;
+    p.G = a.n_global;
+    p.heads = a.heads;
+    p.scale = a.scale;
+    if (a.head_dim == 64) return launch_hd<64>(p, stream);
+    if (a.head_dim == 128) return launch_hd<128>(p, stream);
+    return ATLAS_ERR_UNSUPPORTED;
+}
+
+}  // namespace atlas

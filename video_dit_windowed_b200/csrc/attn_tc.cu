@@ -1,0 +1,538 @@
+// attn_tc.cu -- asymmetric local-global attention, bf16, tcgen05 + TMA + TMEM.
+//
+// Passages: "Technische Samenvatting: AtlasVid" (gist.science), Methodologie
+// 1, Fase 2 (window attention over the cube-reordered sequence) and
+// Methodologie 2 (asymmetric hierarchical attention: a detail query sees the
+// keys of its own cube and every global-proxy key; a global query sees only
+// global keys; global -> detail is masked with -inf).
+//
+// One softmax per query row over its allowed keys, flash style:
+//   * a work unit is one head and 256 consecutive query rows (two 128-row Q
+//     tiles), either detail rows (cube order) or global rows;
+//   * its key list is the detail rows of the windows its queries belong to
+//     (128-key tiles from the first window's start), then all global keys;
+//     detail units of windows that are multiples of 256 rows see exactly
+//     their own window, otherwise per-row masks cut the tile;
+//   * persistent CTAs (one per SM) walk the units head-major, so the CTAs in
+//     flight share one head's global K/V in L2.
+// Warp roles per CTA (320 threads):
+//   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread = one row =
+//                    one TMEM lane),
+//   warp 8           TMA producer (Q tiles, then K and V tiles into a ring of
+//                    shared-memory slots),
+//   warp 9           tensor-memory owner and MMA issuer (one thread).
+// Tensor memory (512 columns): S0 | S1 | O0 | O1. P (bf16) is written over
+// the first half of S and read from TMEM by the P*V MMA.
+// Every wait is bounded: on expiry a bit is set in the device error word,
+// the CTA drains its in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "atlas_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace atlas {
+namespace {
+
+constexpr int kBM = 128;          // query rows per Q tile
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kQTiles = 2;        // Q tiles per CTA (one per softmax warpgroup)
+constexpr int kUnitRows = kBM * kQTiles;
+constexpr int kSlots = 4;         // K/V shared-memory ring slots
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
+
+template <int HD>
+struct Smem {
+    static constexpr int kTileBytes = kBM * HD * 2;  // one 128-row bf16 tile
+    alignas(1024) uint8_t q[kQTiles][kTileBytes];
+    alignas(1024) uint8_t kv[kSlots][kTileBytes];
+    uint64_t q_full[kQTiles];
+    uint64_t q_empty;
+    uint64_t kv_full[kSlots];
+    uint64_t kv_empty[kSlots];
+    uint64_t s_full[kQTiles];
+    uint64_t p_full[kQTiles];
+    uint64_t pv_done[kQTiles];
+    uint64_t o_final[kQTiles];
+    uint64_t drain;
+    uint32_t tmem_base;
+    volatile int abort;
+    uint32_t *err_word;
+};
+
+struct Params {
+    CUtensorMap tm_qd, tm_kd, tm_vd, tm_qg, tm_kg, tm_vg;
+    __nv_bfloat16 *o_d, *o_g;
+    float *lse;
+    uint32_t *err_word;
+    int32_t N, L, G, heads;
+    float scale_log2;
+    int32_t n_dunits, n_gunits, units_per_head, n_units, n_gtiles;
+};
+
+struct Unit {
+    int32_t head, detail, q0, rows, kw0, n_wtiles, n_tiles;
+};
+
+__device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
+    Unit U;
+    U.head = u / p.units_per_head;
+    int32_t lu = u - U.head * p.units_per_head;
+    U.detail = lu < p.n_dunits;
+    if (U.detail) {
+        U.q0 = lu * kUnitRows;
+        U.rows = p.N;
+        int32_t q_last = min(U.q0 + kUnitRows, p.N) - 1;
+        U.kw0 = (U.q0 / p.L) * p.L;
+        int32_t kw1 = min(p.N, (q_last / p.L + 1) * p.L);
+        U.n_wtiles = (kw1 - U.kw0 + kBN - 1) / kBN;
+    } else {
+        U.q0 = (lu - p.n_dunits) * kUnitRows;
+        U.rows = p.G;
+        U.kw0 = 0;
+        U.n_wtiles = 0;
+    }
+    U.n_tiles = U.n_wtiles + p.n_gtiles;
+    return U;
+}
+
+// Bounded wait. Returns false (after flagging `err`) if the phase did not
+// complete within the limit or another role of this CTA aborted.
+template <int HD>
+__device__ __forceinline__ bool wait_phase(Smem<HD> &sm, uint64_t &bar, uint32_t parity,
+                                           uint32_t err, bool honor_abort = true) {
+    const uint32_t a = ptx::smem_addr(&bar);
+    if (ptx::mbar_try_wait(a, parity)) return true;
+    uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ptx::mbar_try_wait(a, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (honor_abort && sm.abort) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(sm.err_word, err);
+                sm.abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Producer: Q tiles once per unit, then K and V tiles of every key tile.
+// ---------------------------------------------------------------------------
+template <int HD>
+__device__ void producer(const Params &p, Smem<HD> &sm) {
+    constexpr uint32_t kBytes = Smem<HD>::kTileBytes;
+    uint32_t it = 0, unit_iter = 0;
+    uint32_t q_armed = 0;
+    uint32_t armed[kSlots] = {0};
+    bool ok = true;
+    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit(p, u);
+        if (unit_iter > 0 && !(ok = wait_phase(sm, sm.q_empty, (unit_iter - 1) & 1,
+                                               kErrTimeoutProducer)))
+            break;
+        const CUtensorMap *tq = U.detail ? &p.tm_qd : &p.tm_qg;
+        for (int i = 0; i < kQTiles; ++i) {
+            uint32_t bar = ptx::smem_addr(&sm.q_full[i]);
+            ptx::mbar_arrive_expect_tx(bar, kBytes);
+            for (int db = 0; db < HD / 64; ++db)
+                ptx::tma_load_3d(ptx::smem_addr(sm.q[i] + db * kBM * 128), tq, bar, db * 64,
+                                 U.head, U.q0 + i * kBM);
+        }
+        q_armed = unit_iter + 1;
+        for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
+            const bool win = j < U.n_wtiles;
+            const int32_t row = win ? U.kw0 + j * kBN : (j - U.n_wtiles) * kBN;
+            const CUtensorMap *maps[2] = {win ? &p.tm_kd : &p.tm_kg, win ? &p.tm_vd : &p.tm_vg};
+            for (int which = 0; which < 2; ++which, ++it) {
+                const uint32_t slot = it % kSlots, round = it / kSlots;
+                if (round > 0 && !(ok = wait_phase(sm, sm.kv_empty[slot], (round - 1) & 1,
+                                                   kErrTimeoutProducer)))
+                    break;
+                uint32_t bar = ptx::smem_addr(&sm.kv_full[slot]);
+                ptx::mbar_arrive_expect_tx(bar, kBytes);
+                for (int db = 0; db < HD / 64; ++db)
+                    ptx::tma_load_3d(ptx::smem_addr(sm.kv[slot] + db * kBN * 128), maps[which],
+                                     bar, db * 64, U.head, row);
+                armed[slot] = round + 1;
+            }
+        }
+    }
+    if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        if (q_armed)
+            for (int i = 0; i < kQTiles; ++i)
+                wait_phase(sm, sm.q_full[i], (q_armed - 1) & 1, kErrTimeoutTeardown, false);
+        for (int s = 0; s < kSlots; ++s)
+            if (armed[s])
+                wait_phase(sm, sm.kv_full[s], (armed[s] - 1) & 1, kErrTimeoutTeardown, false);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one thread).
+// ---------------------------------------------------------------------------
+template <int HD>
+__device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+    constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(kBM, kBN, 0);
+    constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, HD, 1);
+    const uint32_t tmem_s[2] = {tmem, tmem + kBN};
+    const uint32_t tmem_o[2] = {tmem + 2 * kBN, tmem + 2 * kBN + HD};
+    uint32_t it = 0, unit_iter = 0;
+    uint32_t pv_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+    bool ok = true;
+    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit(p, u);
+        for (int i = 0; i < kQTiles && ok; ++i)
+            ok = wait_phase(sm, sm.q_full[i], unit_iter & 1, kErrTimeoutMma);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
+            // S_i = Q_i K^T
+            uint32_t slot = it % kSlots;
+            if (!(ok = wait_phase(sm, sm.kv_full[slot], (it / kSlots) & 1, kErrTimeoutMma))) break;
+            ++it;
+            ptx::tc_fence_after();
+            const uint32_t k_base = ptx::smem_addr(sm.kv[slot]);
+            for (int i = 0; i < kQTiles; ++i) {
+                if (pv_cnt[i] > 0 &&
+                    !(ok = wait_phase(sm, sm.pv_done[i], (pv_cnt[i] - 1) & 1, kErrTimeoutMma)))
+                    break;
+                ptx::tc_fence_after();
+                const uint32_t q_base = ptx::smem_addr(sm.q[i]);
+#pragma unroll
+                for (int ks = 0; ks < HD / 16; ++ks) {
+                    const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
+                    ptx::mma_ss(tmem_s[i], ptx::smem_desc_sw128(q_base + off, 16, 1024),
+                                ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
+                }
+                ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
+            }
+            if (!ok) break;
+            ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+            // O_i += P_i V
+            slot = it % kSlots;
+            if (!(ok = wait_phase(sm, sm.kv_full[slot], (it / kSlots) & 1, kErrTimeoutMma))) break;
+            ++it;
+            const uint32_t v_base = ptx::smem_addr(sm.kv[slot]);
+            for (int i = 0; i < kQTiles; ++i) {
+                if (!(ok = wait_phase(sm, sm.p_full[i], p_cnt[i] & 1, kErrTimeoutMma))) break;
+                ++p_cnt[i];
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks) {
+                    ptx::mma_ts(tmem_o[i], tmem_s[i] + ks * 8,
+                                ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
+                                kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                ptx::mma_commit(ptx::smem_addr(&sm.pv_done[i]));
+                ++pv_cnt[i];
+            }
+            if (!ok) break;
+            ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+        }
+        if (!ok) break;
+        for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
+        ptx::mma_commit(ptx::smem_addr(&sm.q_empty));
+    }
+    // Drain: every MMA issued must finish before tensor memory is freed.
+    ptx::mma_commit(ptx::smem_addr(&sm.drain));
+    wait_phase(sm, sm.drain, 0, kErrTimeoutTeardown, false);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax + epilogue of Q tile `qt`; 128 threads, thread = row = TMEM lane.
+// ---------------------------------------------------------------------------
+template <int HD>
+__device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, int qt) {
+    const uint32_t warp = (threadIdx.x / 32) & 3;
+    const uint32_t r = threadIdx.x & 127;                 // row within the tile
+    const uint32_t lane_sel = (warp * 32u) << 16;         // TMEM lane field
+    const uint32_t t_s = tmem + qt * kBN + lane_sel;
+    const uint32_t t_o = tmem + 2 * kBN + qt * HD + lane_sel;
+    const uint32_t err = kErrTimeoutSoftmax;
+    uint32_t s_cnt = 0, unit_iter = 0;
+    for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit(p, u);
+        const int32_t q = U.q0 + qt * kBM + static_cast<int32_t>(r);
+        const bool row_valid = q < U.rows;
+        int32_t lo = 0, hi = p.N;
+        if (U.detail) {
+            lo = (min(q, p.N - 1) / p.L) * p.L;
+            hi = min(lo + p.L, p.N);
+        }
+        float m_run = kNegInf, l_run = 0.f;
+        for (int32_t j = 0; j < U.n_tiles; ++j) {
+            if (!__all_sync(0xffffffffu, wait_phase(sm, sm.s_full[qt], s_cnt & 1, err))) return;
+            ++s_cnt;
+            ptx::tc_fence_after();
+            float s[kBN];
+            {
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
+                    ptx::tmem_ld32(t_s + c * 32, raw);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+                }
+            }
+            // Mask keys outside this row's allowed range.
+            int32_t k0, klo, khi;
+            if (j < U.n_wtiles) {
+                k0 = U.kw0 + j * kBN;
+                klo = lo;
+                khi = hi;
+            } else {
+                k0 = (j - U.n_wtiles) * kBN;
+                klo = 0;
+                khi = p.G;
+            }
+            if (k0 < klo || k0 + kBN > khi) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (k0 + c < klo || k0 + c >= khi) s[c] = kNegInf;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+            const float mx2 = mx * p.scale_log2;
+            // Lazy rescale: move the running max only when the tile's max
+            // exceeds it by more than the threshold (results are exact either
+            // way, because O and l share the same reference).
+            const bool need = (m_run == kNegInf) ? (mx2 != kNegInf)
+                                                 : (mx2 > m_run + kRescaleThreshold);
+            float alpha = 1.f;
+            if (need) {
+                alpha = (m_run == kNegInf) ? 0.f : ptx::ex2(m_run - mx2);
+                m_run = mx2;
+            }
+            l_run *= alpha;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    ptx::tmem_st32(t_o + c * 32, o);
+                }
+            }
+            const float m_use = (m_run == kNegInf) ? 0.f : m_run;
+            float sum = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = half * 64 + 2 * e;
+                    const float p0 = ptx::ex2(fmaf(s[c], p.scale_log2, -m_use));
+                    const float p1 = ptx::ex2(fmaf(s[c + 1], p.scale_log2, -m_use));
+                    sum += p0 + p1;
+                    pk[e] = ptx::pack_bf16x2(p0, p1);
+                }
+                ptx::tmem_st32(t_s + half * 32, pk);
+            }
+            l_run += sum;
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
+        }
+        // Epilogue: O / l -> bf16 rows; LSE.
+        if (!__all_sync(0xffffffffu, wait_phase(sm, sm.o_final[qt], unit_iter & 1, err)))
+            return;
+        ptx::tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16 *out = U.detail ? p.o_d : p.o_g;
+        uint4 *dst = reinterpret_cast<uint4 *>(
+            out + (static_cast<int64_t>(row_valid ? q : 0) * p.heads + U.head) * HD);
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            ptx::tmem_ld32(t_o + c * 32, o);
+            if (row_valid) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 w;
+                    w.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                           __uint_as_float(o[8 * v + 1]) * inv_l);
+                    w.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                           __uint_as_float(o[8 * v + 3]) * inv_l);
+                    w.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                           __uint_as_float(o[8 * v + 5]) * inv_l);
+                    w.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                           __uint_as_float(o[8 * v + 7]) * inv_l);
+                    dst[c * 4 + v] = w;
+                }
+            }
+        }
+        if (p.lse != nullptr && row_valid) {
+            const int64_t col = U.detail ? q : static_cast<int64_t>(p.N) + q;
+            p.lse[static_cast<int64_t>(U.head) * (p.N + p.G) + col] =
+                (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        }
+        ptx::tc_fence_before();
+    }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem<HD> &sm = *reinterpret_cast<Smem<HD> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQTiles; ++i) {
+            ptx::mbar_init(ptx::smem_addr(&sm.q_full[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.s_full[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.p_full[i]), kBM);
+            ptx::mbar_init(ptx::smem_addr(&sm.pv_done[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.o_final[i]), 1);
+        }
+        ptx::mbar_init(ptx::smem_addr(&sm.q_empty), 1);
+        for (int s = 0; s < kSlots; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&sm.kv_full[s]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.kv_empty[s]), 1);
+        }
+        ptx::mbar_init(ptx::smem_addr(&sm.drain), 1);
+        sm.abort = 0;
+        sm.err_word = p.err_word;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_addr(&sm.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        ptx::prefetch_tmap(&p.tm_qd);
+        ptx::prefetch_tmap(&p.tm_kd);
+        ptx::prefetch_tmap(&p.tm_vd);
+        ptx::prefetch_tmap(&p.tm_qg);
+        ptx::prefetch_tmap(&p.tm_kg);
+        ptx::prefetch_tmap(&p.tm_vg);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    // A 512-column allocation always starts at column 0 of lane 0.
+    const bool tmem_ok = tmem == 0;
+    if (!tmem_ok && threadIdx.x == 0) {
+        atomicOr(p.err_word, kErrTmemAlloc);
+    }
+
+    if (tmem_ok) {
+        if (warp < 8) {
+            softmax_epilogue<HD>(p, sm, tmem, warp / 4);
+        } else if (warp == kProducerWarp) {
+            if (lane == 0) producer<HD>(p, sm);
+        } else if (warp == kMmaWarp) {
+            if (lane == 0) mma_issuer<HD>(p, sm, tmem);
+        }
+    }
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// [rows, heads, hd] bf16 viewed as a 3-D tensor (hd, heads, rows); box of
+// 64 channels x 1 head x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(hd) * 2,
+                             static_cast<cuuint64_t>(heads) * hd * 2};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBM)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int HD>
+atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
+    Params p{};
+    const bool has_d = a.n_detail > 0, has_g = a.n_global > 0;
+    // Maps for an absent side point at the other side; they are never used.
+    const void *qd = has_d ? a.q_d : a.q_g, *kd = has_d ? a.k_d : a.k_g,
+               *vd = has_d ? a.v_d : a.v_g;
+    const void *qg = has_g ? a.q_g : a.q_d, *kg = has_g ? a.k_g : a.k_d,
+               *vg = has_g ? a.v_g : a.v_d;
+    const int64_t nd = has_d ? a.n_detail : a.n_global, ng = has_g ? a.n_global : a.n_detail;
+    if (!make_map(&p.tm_qd, qd, nd, a.heads, HD) || !make_map(&p.tm_kd, kd, nd, a.heads, HD) ||
+        !make_map(&p.tm_vd, vd, nd, a.heads, HD) || !make_map(&p.tm_qg, qg, ng, a.heads, HD) ||
+        !make_map(&p.tm_kg, kg, ng, a.heads, HD) || !make_map(&p.tm_vg, vg, ng, a.heads, HD))
+        return ATLAS_ERR_CUDA;
+    p.o_d = static_cast<__nv_bfloat16 *>(a.o_d);
+    p.o_g = static_cast<__nv_bfloat16 *>(a.o_g);
+    p.lse = a.lse;
+    p.err_word = device_error_word();
+    if (!p.err_word) return ATLAS_ERR_CUDA;
+    p.N = static_cast<int32_t>(a.n_detail);
+    p.L = static_cast<int32_t>(has_d ? a.window_len : 1);
+    p.G = static_cast<int32_t>(a.n_global);
+    p.heads = a.heads;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.n_dunits = static_cast<int32_t>((a.n_detail + kUnitRows - 1) / kUnitRows);
+    p.n_gunits = static_cast<int32_t>((a.n_global + kUnitRows - 1) / kUnitRows);
+    p.units_per_head = p.n_dunits + p.n_gunits;
+    p.n_units = p.units_per_head * a.heads;
+    p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
+    if (p.n_units == 0) return ATLAS_OK;
+    const size_t smem = sizeof(Smem<HD>) + 1024;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [&] {
+        attr_err = cudaFuncSetAttribute(attn_tc_kernel<HD>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem));
+    });
+    if (attr_err != cudaSuccess) return ATLAS_ERR_CUDA;
+    const int grid = std::min(p.n_units, dev.sm_count);
+    attn_tc_kernel<HD><<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+}  // namespace
+
+atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream) {
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    if (a.head_dim == 128) return launch_hd<128>(a, dev, stream);
+    if (a.head_dim == 64) return launch_hd<64>(a, dev, stream);
+    return ATLAS_ERR_UNSUPPORTED;
+}
+
+}  // namespace atlas

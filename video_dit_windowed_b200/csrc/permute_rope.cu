@@ -1,0 +1,380 @@
+// permute_rope.cu -- cube reorder / unorder and 3D RoPE: one row-gather pass.
+//
+// Passages: "Technische Samenvatting: AtlasVid" (gist.science), Methodologie
+// 1, Fase 2 (tokens of one spatiotemporal cube made contiguous), Fase 1
+// (temporal RoPE index times r_t) and Methodologie 2, position alignment
+// (global RoPE coordinates times the resolution ratios).
+//
+// The pass is HBM-bound: every destination row (heads*head_dim elements,
+// 10 KB for 40 heads x 128 bf16) is one contiguous read of its source row and
+// one contiguous write. Each 128-thread group owns one row at a time; a
+// thread owns a fixed 16-byte slot of the head (so its RoPE pairs, and hence
+// its cos/sin table entries, are the same for every head of the row) and
+// moves that slot for heads hg, hg + 128/vph, ... with all loads of a row in
+// flight before the first store. Row index arithmetic (cube <-> raster) is
+// done once per row per thread with multiply-shift division.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "atlas_internal.cuh"
+
+namespace atlas {
+namespace {
+
+// Unsigned division by a run-time constant for dividends below 2^31:
+// q = (n * m) >> s with m = ceil(2^s / d), s = 31 + ceil(log2 d). For
+// n < 2^31 the error term n*(m - 2^s/d)/2^s stays below 1/d, so the floor is
+// exact.
+struct FastDiv {
+    uint64_t m = 1ull << 31;
+    uint32_t s = 31;
+    uint32_t d = 1;
+    FastDiv() = default;
+    explicit FastDiv(uint32_t div) : d(div) {
+        uint32_t l = 0;
+        while ((1ull << l) < div) ++l;
+        s = 31 + l;
+        m = ((1ull << s) + div - 1) / div;
+    }
+    __host__ __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        return static_cast<uint32_t>((static_cast<uint64_t>(n) * m) >> s);
+    }
+};
+
+struct Geom {
+    uint32_t H, W, ct, ch, cw, cubes_h, cubes_w, L;
+    FastDiv by_W, by_H, by_ct, by_ch, by_cw, by_cubes_w, by_cubes_h, by_L;
+};
+
+struct Params {
+    const uint8_t *src;
+    uint8_t *dst;
+    uint32_t rows;          // tokens
+    uint32_t row_vecs;      // 16-byte vectors per row
+    uint32_t vph;           // 16-byte vectors per head (power of two <= 128)
+    uint32_t heads;
+    Geom g;
+    const float2 *tab;      // RoPE cos/sin table, NULL without RoPE
+    uint32_t tab_base[3];   // first entry of each axis section
+    uint32_t half[3];       // d_axis / 2 for t, h, w
+};
+
+constexpr int kThreads = 256;     // two 128-thread row groups per block
+constexpr int kGroup = 128;
+constexpr int kMaxInFlight = 8;   // 16-byte loads in flight per thread per row
+
+__device__ __forceinline__ uint4 ld_stream(const uint8_t *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// Coherent streaming load, for the in-place RoPE pass (src may equal dst).
+__device__ __forceinline__ uint4 ld_stream_coherent(const uint8_t *p) {
+    uint4 v;
+    asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint8_t *p, const uint4 &v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Raster coordinates of a raster row.
+__device__ __forceinline__ void raster_coords(const Geom &g, uint32_t r, uint32_t &t,
+                                              uint32_t &h, uint32_t &w) {
+    uint32_t tw = g.by_W.div(r);
+    w = r - tw * g.W;
+    t = g.by_H.div(tw);
+    h = tw - t * g.H;
+}
+
+// Cube-order position of the token at (t, h, w).
+__device__ __forceinline__ uint32_t cube_position(const Geom &g, uint32_t t, uint32_t h,
+                                                  uint32_t w) {
+    uint32_t bt = g.by_ct.div(t), bh = g.by_ch.div(h), bw = g.by_cw.div(w);
+    uint32_t cube = (bt * g.cubes_h + bh) * g.cubes_w + bw;
+    uint32_t local = ((t - bt * g.ct) * g.ch + (h - bh * g.ch)) * g.cw + (w - bw * g.cw);
+    return cube * g.L + local;
+}
+
+// Raster coordinates of the token at cube-order position j.
+__device__ __forceinline__ void cube_coords(const Geom &g, uint32_t j, uint32_t &t,
+                                            uint32_t &h, uint32_t &w) {
+    uint32_t cube = g.by_L.div(j);
+    uint32_t local = j - cube * g.L;
+    uint32_t c1 = g.by_cubes_w.div(cube);
+    uint32_t bw = cube - c1 * g.cubes_w;
+    uint32_t bt = g.by_cubes_h.div(c1);
+    uint32_t bh = c1 - bt * g.cubes_h;
+    uint32_t l1 = g.by_cw.div(local);
+    uint32_t lw = local - l1 * g.cw;
+    uint32_t lt = g.by_ch.div(l1);
+    uint32_t lh = l1 - lt * g.ch;
+    t = bt * g.ct + lt;
+    h = bh * g.ch + lh;
+    w = bw * g.cw + lw;
+}
+
+// Rotate the pairs of one 16-byte vector. bf16: 4 pairs, fp32: 2 pairs.
+template <int EB>
+__device__ __forceinline__ uint4 rotate(uint4 v, const float2 *cs);
+
+template <>
+__device__ __forceinline__ uint4 rotate<2>(uint4 v, const float2 *cs) {
+    uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        float x0 = __uint_as_float(u[p] << 16);
+        float x1 = __uint_as_float(u[p] & 0xffff0000u);
+        float c = cs[p].x, s = cs[p].y;
+        float y0 = fmaf(x0, c, -(x1 * s));
+        float y1 = fmaf(x0, s, x1 * c);
+        __nv_bfloat162 b = __floats2bfloat162_rn(y0, y1);  // .x = y0 (low half)
+        u[p] = *reinterpret_cast<uint32_t *>(&b);
+    }
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+template <>
+__device__ __forceinline__ uint4 rotate<4>(uint4 v, const float2 *cs) {
+    float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                  __uint_as_float(v.w)};
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        float x0 = f[2 * p], x1 = f[2 * p + 1];
+        float c = cs[p].x, s = cs[p].y;
+        f[2 * p] = fmaf(x0, c, -(x1 * s));
+        f[2 * p + 1] = fmaf(x0, s, x1 * c);
+    }
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+}
+
+// MODE 0: dst in cube order, src raster (reorder). MODE 1: dst raster, src
+// cube order (unorder). MODE 2: dst and src raster (RoPE only).
+template <int EB, bool ROPE, int MODE>
+__global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) {
+    constexpr int kPairs = 16 / EB / 2;  // RoPE pairs in one 16-byte vector
+    const uint32_t tid = threadIdx.x & (kGroup - 1);
+    const uint32_t group = threadIdx.x / kGroup;
+    const uint64_t row_bytes = static_cast<uint64_t>(p.row_vecs) * 16u;
+
+    // This thread's fixed slot within a head, and its pairs' table layout.
+    const uint32_t slot = ROPE ? tid % p.vph : 0;
+    const uint32_t hg = ROPE ? tid / p.vph : 0;
+    const uint32_t n_hg = ROPE ? kGroup / p.vph : 0;
+    uint32_t pair_axis[kPairs], pair_off[kPairs], pair_stride[kPairs];
+    if (ROPE) {
+#pragma unroll
+        for (int q = 0; q < kPairs; ++q) {
+            uint32_t P = slot * kPairs + q;  // pair index within the head
+            uint32_t a = P < p.half[0] ? 0u : (P < p.half[0] + p.half[1] ? 1u : 2u);
+            uint32_t k = a == 0 ? P : (a == 1 ? P - p.half[0] : P - p.half[0] - p.half[1]);
+            pair_axis[q] = a;
+            pair_off[q] = (a == 0 ? p.tab_base[0] : (a == 1 ? p.tab_base[1] : p.tab_base[2])) + k;
+            pair_stride[q] = a == 0 ? p.half[0] : (a == 1 ? p.half[1] : p.half[2]);
+        }
+    }
+
+    for (uint32_t row = blockIdx.x * 2 + group; row < p.rows; row += gridDim.x * 2) {
+        uint32_t t = 0, h = 0, w = 0, src_row;
+        if (MODE == 0) {
+            cube_coords(p.g, row, t, h, w);
+            src_row = (t * p.g.H + h) * p.g.W + w;
+        } else if (MODE == 1) {
+            raster_coords(p.g, row, t, h, w);
+            src_row = cube_position(p.g, t, h, w);
+        } else {
+            raster_coords(p.g, row, t, h, w);
+            src_row = row;
+        }
+        const uint8_t *s = p.src + static_cast<uint64_t>(src_row) * row_bytes;
+        uint8_t *d = p.dst + static_cast<uint64_t>(row) * row_bytes;
+
+        if (!ROPE) {
+            for (uint32_t v0 = tid; v0 < p.row_vecs; v0 += kGroup * kMaxInFlight) {
+                uint4 buf[kMaxInFlight];
+#pragma unroll
+                for (int i = 0; i < kMaxInFlight; ++i) {
+                    uint32_t v = v0 + i * kGroup;
+                    if (v < p.row_vecs) buf[i] = ld_stream(s + v * 16u);
+                }
+#pragma unroll
+                for (int i = 0; i < kMaxInFlight; ++i) {
+                    uint32_t v = v0 + i * kGroup;
+                    if (v < p.row_vecs) st_stream(d + v * 16u, buf[i]);
+                }
+            }
+        } else {
+            float2 cs[kPairs];
+#pragma unroll
+            for (int q = 0; q < kPairs; ++q) {
+                const uint32_t c = pair_axis[q] == 0 ? t : (pair_axis[q] == 1 ? h : w);
+                cs[q] = __ldg(p.tab + pair_off[q] + c * pair_stride[q]);
+            }
+            for (uint32_t h0 = hg; h0 < p.heads; h0 += n_hg * kMaxInFlight) {
+                uint4 buf[kMaxInFlight];
+#pragma unroll
+                for (int i = 0; i < kMaxInFlight; ++i) {
+                    uint32_t hd = h0 + i * n_hg;
+                    if (hd < p.heads) {
+                        const uint8_t *a = s + (hd * p.vph + slot) * 16u;
+                        buf[i] = MODE == 2 ? ld_stream_coherent(a) : ld_stream(a);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kMaxInFlight; ++i) {
+                    uint32_t hd = h0 + i * n_hg;
+                    if (hd < p.heads)
+                        st_stream(d + (hd * p.vph + slot) * 16u, rotate<EB>(buf[i], cs));
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// RoPE table: fp64 angles rounded to fp32 cos/sin, cached per device.
+// Layout: axis t entries [t][k] (k < d_t/2), then axis h [h][k], then w.
+// ---------------------------------------------------------------------------
+using TableKey = std::tuple<int, int64_t, int64_t, int64_t, int32_t, int32_t, int32_t,
+                            uint64_t, uint64_t, uint64_t, uint64_t>;
+std::mutex g_tab_mutex;
+std::map<TableKey, float2 *> g_tables;
+
+uint64_t bits_of(double v) {
+    uint64_t b;
+    std::memcpy(&b, &v, sizeof b);
+    return b;
+}
+
+atlas_status rope_table(int device, int64_t T, int64_t H, int64_t W, const atlas_rope &r,
+                        float2 **out) {
+    TableKey key{device, T, H, W, r.d_t, r.d_h, r.d_w, bits_of(r.theta), bits_of(r.scale_t),
+                 bits_of(r.scale_h), bits_of(r.scale_w)};
+    std::lock_guard<std::mutex> lock(g_tab_mutex);
+    auto it = g_tables.find(key);
+    if (it != g_tables.end()) {
+        *out = it->second;
+        return ATLAS_OK;
+    }
+    const int64_t ext[3] = {T, H, W};
+    const int32_t width[3] = {r.d_t, r.d_h, r.d_w};
+    const double scale[3] = {r.scale_t, r.scale_h, r.scale_w};
+    std::vector<float2> host;
+    for (int a = 0; a < 3; ++a) {
+        for (int64_t c = 0; c < ext[a]; ++c) {
+            for (int32_t k = 0; k < width[a] / 2; ++k) {
+                double omega = std::pow(r.theta, -2.0 * k / static_cast<double>(width[a]));
+                double phi = (static_cast<double>(c) * scale[a]) * omega;
+                host.push_back(make_float2(static_cast<float>(std::cos(phi)),
+                                           static_cast<float>(std::sin(phi))));
+            }
+        }
+    }
+    if (host.empty()) host.push_back(make_float2(1.f, 0.f));
+    float2 *dev = nullptr;
+    if (cudaMalloc(&dev, host.size() * sizeof(float2)) != cudaSuccess) return ATLAS_ERR_CUDA;
+    if (cudaMemcpy(dev, host.data(), host.size() * sizeof(float2), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
+        cudaFree(dev);
+        return ATLAS_ERR_CUDA;
+    }
+    g_tables.emplace(key, dev);
+    *out = dev;
+    return ATLAS_OK;
+}
+
+template <int EB, bool ROPE, int MODE>
+atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream) {
+    uint32_t blocks_needed = (p.rows + 1) / 2;
+    uint32_t grid = std::min<uint32_t>(blocks_needed, static_cast<uint32_t>(dev.sm_count) * 8u);
+    if (grid == 0) return ATLAS_OK;
+    permute_rope_kernel<EB, ROPE, MODE><<<grid, kThreads, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+template <int EB>
+atlas_status dispatch(const Params &p, bool rope, int mode, const DeviceInfo &dev,
+                      cudaStream_t stream) {
+    if (rope) {
+        if (mode == 0) return launch<EB, true, 0>(p, dev, stream);
+        return launch<EB, true, 2>(p, dev, stream);
+    }
+    if (mode == 0) return launch<EB, false, 0>(p, dev, stream);
+    return launch<EB, false, 1>(p, dev, stream);
+}
+
+}  // namespace
+
+atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream) {
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    Params p{};
+    p.src = static_cast<const uint8_t *>(a.src);
+    p.dst = static_cast<uint8_t *>(a.dst);
+    p.rows = static_cast<uint32_t>(a.T * a.H * a.W);
+    p.heads = static_cast<uint32_t>(a.heads);
+    p.row_vecs = static_cast<uint32_t>(static_cast<int64_t>(a.heads) * a.head_dim *
+                                       a.elem_bytes / 16);
+    p.vph = static_cast<uint32_t>(a.head_dim * a.elem_bytes / 16);
+    Geom &g = p.g;
+    g.H = static_cast<uint32_t>(a.H);
+    g.W = static_cast<uint32_t>(a.W);
+    g.ct = static_cast<uint32_t>(a.ct);
+    g.ch = static_cast<uint32_t>(a.ch);
+    g.cw = static_cast<uint32_t>(a.cw);
+    g.cubes_h = g.H / g.ch;
+    g.cubes_w = g.W / g.cw;
+    g.L = g.ct * g.ch * g.cw;
+    g.by_W = FastDiv(g.W);
+    g.by_H = FastDiv(g.H);
+    g.by_ct = FastDiv(g.ct);
+    g.by_ch = FastDiv(g.ch);
+    g.by_cw = FastDiv(g.cw);
+    g.by_cubes_w = FastDiv(g.cubes_w);
+    g.by_cubes_h = FastDiv(g.cubes_h);
+    g.by_L = FastDiv(g.L);
+    const bool rope = a.rope != nullptr;
+    if (rope) {
+        float2 *tab = nullptr;
+        atlas_status st = rope_table(dev.device, a.T, a.H, a.W, *a.rope, &tab);
+        if (st != ATLAS_OK) return st;
+        p.tab = tab;
+        p.half[0] = static_cast<uint32_t>(a.rope->d_t / 2);
+        p.half[1] = static_cast<uint32_t>(a.rope->d_h / 2);
+        p.half[2] = static_cast<uint32_t>(a.rope->d_w / 2);
+        p.tab_base[0] = 0;
+        p.tab_base[1] = static_cast<uint32_t>(a.T) * p.half[0];
+        p.tab_base[2] = p.tab_base[1] + static_cast<uint32_t>(a.H) * p.half[1];
+    }
+    if (a.elem_bytes == 2) return dispatch<2>(p, rope, a.mode, dev, stream);
+    return dispatch<4>(p, rope, a.mode, dev, stream);
+}
+
+atlas_status release_rope_tables() {
+    std::lock_guard<std::mutex> lock(g_tab_mutex);
+    atlas_status st = ATLAS_OK;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto &kv : g_tables) {
+        cudaSetDevice(std::get<0>(kv.first));
+        if (cudaDeviceSynchronize() != cudaSuccess) st = ATLAS_ERR_CUDA;
+        if (cudaFree(kv.second) != cudaSuccess) st = ATLAS_ERR_CUDA;
+    }
+    g_tables.clear();
+    cudaSetDevice(cur);
+    return st;
+}
+
+}  // namespace atlas
