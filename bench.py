@@ -284,8 +284,8 @@ def config_of(w, world):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
-    times, flops_total = [], 0
+    w = workload(args)
+    times = []
     budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         tf, cores, sample, t = time_oracle(w, budget_s=budget, seed=i)
@@ -304,11 +304,19 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
+def workload(args):
+    w = WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
+    return w
+
+
 def run_atlas(args, world, rank, local):
     from video_dit_windowed_b200 import atlas, build
     if not os.path.exists(atlas.LIB_PATH):
         build.build()
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
@@ -445,6 +453,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads instead of its own "
+                         "(smaller cases for profiler captures; reported in config)")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
