@@ -15,12 +15,13 @@
 //     their own window, otherwise per-row masks cut the tile;
 //   * persistent CTAs (one per SM) walk the units head-major, so the CTAs in
 //     flight share one head's global K/V in L2.
-// Warp roles per CTA (320 threads):
+// Warp roles per CTA (384 threads):
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread = one row =
 //                    one TMEM lane),
 //   warp 8           TMA producer (Q tiles, then K and V tiles into a ring of
 //                    shared-memory slots),
-//   warp 9           tensor-memory owner and MMA issuer (one thread).
+//   warp 9           tensor-memory owner and MMA issuer (one thread),
+//   warps 10-11      idle (complete the third warpgroup for the register split).
 // Tensor memory (512 columns): S0 | S1 | O0 | O1. P (bf16) is written over
 // the first half of S and read from TMEM by the P*V MMA.
 // Every wait is bounded: on expiry a bit is set in the device error word,
@@ -44,7 +45,14 @@ constexpr int kUnitRows = kBM * kQTiles;
 constexpr int kSlots = 4;         // K/V shared-memory ring slots
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;      // three warpgroups
+// Register split (setmaxnreg): the launch gives 168 per thread (3 warps per
+// SM sub-partition x 168 <= 512); the two softmax warpgroups take 208 and the
+// third warpgroup (producer, MMA issuer, two idle warps) keeps 88:
+// 256*208 + 128*88 = 384*168, and per sub-partition 2*208 + 88 <= 512.
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsOther = 88;
+static_assert(256 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
@@ -275,16 +283,8 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             if (!__all_sync(0xffffffffu, wait_phase(sm, sm.s_full[qt], s_cnt & 1, err))) return;
             ++s_cnt;
             ptx::tc_fence_after();
-            float s[kBN];
-            {
-                uint32_t raw[32];
-#pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    ptx::tmem_ld32(t_s + c * 32, raw);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
-                }
-            }
+            uint32_t sr[kBN];
+            ptx::tmem_ld128(t_s, sr);
             // Mask keys outside this row's allowed range.
             int32_t k0, klo, khi;
             if (j < U.n_wtiles) {
@@ -299,11 +299,19 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             if (k0 < klo || k0 + kBN > khi) {
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
-                    if (k0 + c < klo || k0 + c >= khi) s[c] = kNegInf;
+                    if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
             }
-            float mx = s[0];
+            // Row maximum as a tree (8 independent chains, then 3 levels).
+            float m8[8];
 #pragma unroll
-            for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+            for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(sr[k]);
+#pragma unroll
+            for (int c = 8; c < kBN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sr[c]));
+#pragma unroll
+            for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int k = 0; k < w; ++k) m8[k] = fmaxf(m8[k], m8[k + w]);
+            const float mx = m8[0];
             const float mx2 = mx * p.scale_log2;
             // Lazy rescale: move the running max only when the tile's max
             // exceeds it by more than the threshold (results are exact either
@@ -328,20 +336,26 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
                 }
             }
             const float m_use = (m_run == kNegInf) ? 0.f : m_run;
-            float sum = 0.f;
+            // P = exp2(S*scale*log2e - m); the row sum comes from fp32 P,
+            // accumulated in 8 partial sums.
+            float sum8[8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
+            for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+            uint32_t pk[kBN / 2];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = half * 64 + 2 * e;
-                    const float p0 = ptx::ex2(fmaf(s[c], p.scale_log2, -m_use));
-                    const float p1 = ptx::ex2(fmaf(s[c + 1], p.scale_log2, -m_use));
-                    sum += p0 + p1;
-                    pk[e] = ptx::pack_bf16x2(p0, p1);
-                }
-                ptx::tmem_st32(t_s + half * 32, pk);
+            for (int e = 0; e < kBN / 2; ++e) {
+                const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -m_use));
+                const float p1 =
+                    ptx::ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -m_use));
+                sum8[e & 7] += p0 + p1;
+                pk[e] = ptx::pack_bf16x2(p0, p1);
             }
+            ptx::tmem_st64(t_s, pk);
+#pragma unroll
+            for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int k = 0; k < w; ++k) sum8[k] += sum8[k + w];
+            const float sum = sum8[0];
             l_run += sum;
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
@@ -430,13 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         atomicOr(p.err_word, kErrTmemAlloc);
     }
 
-    if (tmem_ok) {
-        if (warp < 8) {
-            softmax_epilogue<HD>(p, sm, tmem, warp / 4);
-        } else if (warp == kProducerWarp) {
-            if (lane == 0) producer<HD>(p, sm);
-        } else if (warp == kMmaWarp) {
-            if (lane == 0) mma_issuer<HD>(p, sm, tmem);
+    if (warp < 8) {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        if (tmem_ok) softmax_epilogue<HD>(p, sm, tmem, warp / 4);
+    } else {
+        ptx::setmaxnreg_dec<kRegsOther>();
+        if (tmem_ok && lane == 0) {
+            if (warp == kProducerWarp) producer<HD>(p, sm);
+            if (warp == kMmaWarp) mma_issuer<HD>(p, sm, tmem);
         }
     }
     __syncwarp();
