@@ -19,11 +19,14 @@
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread = one row =
 //                    one TMEM lane),
 //   warp 8           TMA producer (Q tiles, then K and V tiles into a ring of
-//                    shared-memory slots),
+//                    shared-memory slots, in the order the MMAs use them),
 //   warp 9           tensor-memory owner and MMA issuer (one thread),
 //   warps 10-11      idle (complete the third warpgroup for the register split).
-// Tensor memory (512 columns): S0 | S1 | O0 | O1. P (bf16) is written over
-// the first half of S and read from TMEM by the P*V MMA.
+// Tensor memory (512 columns): S0 | S1 | O0 | O1 (fp32). P (bf16) goes to
+// shared memory, so S of the next key tile can be computed as soon as the
+// softmax has loaded S of this one. The MMA issue order per key tile j is
+//   S0(j+1), S1(j+1), O0 += P0(j) V(j), O1 += P1(j) V(j),
+// which gives each softmax the time of about four MMAs to produce P(j).
 // Every wait is bounded: on expiry a bit is set in the device error word,
 // the CTA drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -42,16 +45,15 @@ constexpr int kBM = 128;          // query rows per Q tile
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kQTiles = 2;        // Q tiles per CTA (one per softmax warpgroup)
 constexpr int kUnitRows = kBM * kQTiles;
-constexpr int kSlots = 4;         // K/V shared-memory ring slots
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 384;      // three warpgroups
+constexpr int kThreads = 384;     // three warpgroups
 // Register split (setmaxnreg): the launch gives 168 per thread (3 warps per
-// SM sub-partition x 168 <= 512); the two softmax warpgroups take 208 and the
-// third warpgroup (producer, MMA issuer, two idle warps) keeps 88:
-// 256*208 + 128*88 = 384*168, and per sub-partition 2*208 + 88 <= 512.
-constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsOther = 88;
+// SM sub-partition x 168 <= 512); the two softmax warpgroups take 200 and the
+// third warpgroup (producer, MMA issuer, two idle warps) keeps 104:
+// 256*200 + 128*104 = 384*168, and per sub-partition 2*200 + 104 <= 512.
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsOther = 104;
 static_assert(256 * kRegsSoftmax + 128 * kRegsOther == kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -59,17 +61,21 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 
 template <int HD>
 struct Smem {
-    static constexpr int kTileBytes = kBM * HD * 2;  // one 128-row bf16 tile
+    static constexpr int kTileBytes = kBM * HD * 2;     // one 128-row bf16 Q/K/V tile
+    static constexpr int kPBytes = kBM * kBN * 2;       // one 128 x 128 bf16 P tile
+    static constexpr int kSlots = (96 * 1024) / kTileBytes;  // K/V ring: 96 KB
     alignas(1024) uint8_t q[kQTiles][kTileBytes];
+    alignas(1024) uint8_t pmat[kQTiles][kPBytes];
     alignas(1024) uint8_t kv[kSlots][kTileBytes];
     uint64_t q_full[kQTiles];
     uint64_t q_empty;
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];
-    uint64_t s_full[kQTiles];
-    uint64_t p_full[kQTiles];
-    uint64_t pv_done[kQTiles];
-    uint64_t o_final[kQTiles];
+    uint64_t s_full[kQTiles];    // S(j) is in TMEM               (MMA commit)
+    uint64_t s_free[kQTiles];    // softmax has loaded S(j)       (128 arrivals)
+    uint64_t p_full[kQTiles];    // P(j) in smem, O rescaled      (128 arrivals)
+    uint64_t pv_done[kQTiles];   // O += P(j) V(j) finished       (MMA commit)
+    uint64_t o_final[kQTiles];   // every MMA of the unit done    (MMA commit)
     uint64_t drain;
     uint32_t tmem_base;
     volatile int abort;
@@ -133,46 +139,66 @@ __device__ __forceinline__ bool wait_phase(Smem<HD> &sm, uint64_t &bar, uint32_t
     }
 }
 
+// Key tile j of unit U: first row and whether it is a window (detail) tile.
+__device__ __forceinline__ int32_t key_row(const Unit &U, int32_t j) {
+    return j < U.n_wtiles ? U.kw0 + j * kBN : (j - U.n_wtiles) * kBN;
+}
+
 // ---------------------------------------------------------------------------
-// Producer: Q tiles once per unit, then K and V tiles of every key tile.
+// Producer: Q tiles once per unit, then K/V tiles in MMA order:
+// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
 // ---------------------------------------------------------------------------
 template <int HD>
 __device__ void producer(const Params &p, Smem<HD> &sm) {
     constexpr uint32_t kBytes = Smem<HD>::kTileBytes;
+    constexpr int kSlots = Smem<HD>::kSlots;
     uint32_t it = 0, unit_iter = 0;
     uint32_t q_armed = 0;
-    uint32_t armed[kSlots] = {0};
+    uint32_t armed[kSlots];
+#pragma unroll
+    for (int s = 0; s < kSlots; ++s) armed[s] = 0;
     bool ok = true;
+
+    auto load = [&](const CUtensorMap *map, int32_t head, int32_t row) -> bool {
+        const uint32_t slot = it % kSlots, round = it / kSlots;
+        if (round > 0 &&
+            !wait_phase(sm, sm.kv_empty[slot], (round - 1) & 1, kErrTimeoutProducer))
+            return false;
+        const uint32_t bar = ptx::smem_addr(&sm.kv_full[slot]);
+        ptx::mbar_arrive_expect_tx(bar, kBytes);
+#pragma unroll
+        for (int db = 0; db < HD / 64; ++db)
+            ptx::tma_load_3d(ptx::smem_addr(sm.kv[slot] + db * kBN * 128), map, bar, db * 64,
+                             head, row);
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s)
+            if (s == static_cast<int>(slot)) armed[s] = round + 1;
+        ++it;
+        return true;
+    };
+
     for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const Unit U = decode_unit(p, u);
         if (unit_iter > 0 && !(ok = wait_phase(sm, sm.q_empty, (unit_iter - 1) & 1,
                                                kErrTimeoutProducer)))
             break;
         const CUtensorMap *tq = U.detail ? &p.tm_qd : &p.tm_qg;
+#pragma unroll
         for (int i = 0; i < kQTiles; ++i) {
             uint32_t bar = ptx::smem_addr(&sm.q_full[i]);
             ptx::mbar_arrive_expect_tx(bar, kBytes);
+#pragma unroll
             for (int db = 0; db < HD / 64; ++db)
                 ptx::tma_load_3d(ptx::smem_addr(sm.q[i] + db * kBM * 128), tq, bar, db * 64,
                                  U.head, U.q0 + i * kBM);
         }
         q_armed = unit_iter + 1;
+        auto kmap = [&](int32_t j) { return j < U.n_wtiles ? &p.tm_kd : &p.tm_kg; };
+        auto vmap = [&](int32_t j) { return j < U.n_wtiles ? &p.tm_vd : &p.tm_vg; };
+        ok = load(kmap(0), U.head, key_row(U, 0));
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
-            const bool win = j < U.n_wtiles;
-            const int32_t row = win ? U.kw0 + j * kBN : (j - U.n_wtiles) * kBN;
-            const CUtensorMap *maps[2] = {win ? &p.tm_kd : &p.tm_kg, win ? &p.tm_vd : &p.tm_vg};
-            for (int which = 0; which < 2; ++which, ++it) {
-                const uint32_t slot = it % kSlots, round = it / kSlots;
-                if (round > 0 && !(ok = wait_phase(sm, sm.kv_empty[slot], (round - 1) & 1,
-                                                   kErrTimeoutProducer)))
-                    break;
-                uint32_t bar = ptx::smem_addr(&sm.kv_full[slot]);
-                ptx::mbar_arrive_expect_tx(bar, kBytes);
-                for (int db = 0; db < HD / 64; ++db)
-                    ptx::tma_load_3d(ptx::smem_addr(sm.kv[slot] + db * kBN * 128), maps[which],
-                                     bar, db * 64, U.head, row);
-                armed[slot] = round + 1;
-            }
+            if (j + 1 < U.n_tiles && !(ok = load(kmap(j + 1), U.head, key_row(U, j + 1)))) break;
+            ok = load(vmap(j), U.head, key_row(U, j));
         }
     }
     if (!ok) {
@@ -191,62 +217,75 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 // ---------------------------------------------------------------------------
 template <int HD>
 __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+    constexpr int kSlots = Smem<HD>::kSlots;
     constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, HD, 1);
-    const uint32_t tmem_s[2] = {tmem, tmem + kBN};
-    const uint32_t tmem_o[2] = {tmem + 2 * kBN, tmem + 2 * kBN + HD};
     uint32_t it = 0, unit_iter = 0;
-    uint32_t pv_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+    uint32_t s_cnt = 0;   // S tiles issued per Q tile (same for both)
+    uint32_t p_cnt = 0;   // P tiles consumed per Q tile
     bool ok = true;
+
+    auto next_slot = [&](uint32_t &slot) -> bool {
+        slot = it % kSlots;
+        const bool r = wait_phase(sm, sm.kv_full[slot], (it / kSlots) & 1, kErrTimeoutMma);
+        ++it;
+        ptx::tc_fence_after();
+        return r;
+    };
+    // S_i = Q_i K^T for both Q tiles from the K tile in `slot`.
+    auto issue_s = [&](uint32_t slot) -> bool {
+        const uint32_t k_base = ptx::smem_addr(sm.kv[slot]);
+#pragma unroll
+        for (int i = 0; i < kQTiles; ++i) {
+            if (s_cnt > 0 &&
+                !wait_phase(sm, sm.s_free[i], (s_cnt - 1) & 1, kErrTimeoutMma))
+                return false;
+            ptx::tc_fence_after();
+            const uint32_t q_base = ptx::smem_addr(sm.q[i]);
+#pragma unroll
+            for (int ks = 0; ks < HD / 16; ++ks) {
+                const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
+                ptx::mma_ss(tmem + i * kBN, ptx::smem_desc_sw128(q_base + off, 16, 1024),
+                            ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
+            }
+            ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
+        }
+        ++s_cnt;
+        ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+        return true;
+    };
+    // O_i += P_i V for both Q tiles from the V tile in `slot`.
+    auto issue_pv = [&](uint32_t slot, bool first) -> bool {
+        const uint32_t v_base = ptx::smem_addr(sm.kv[slot]);
+#pragma unroll
+        for (int i = 0; i < kQTiles; ++i) {
+            if (!wait_phase(sm, sm.p_full[i], p_cnt & 1, kErrTimeoutMma)) return false;
+            ptx::tc_fence_after();
+            const uint32_t p_base = ptx::smem_addr(sm.pmat[i]);
+#pragma unroll
+            for (int ks = 0; ks < kBN / 16; ++ks) {
+                const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
+                ptx::mma_ss(tmem + 2 * kBN + i * HD, ptx::smem_desc_sw128(p_base + off, 16, 1024),
+                            ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
+                            kIdescPV, (!first || ks > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(ptx::smem_addr(&sm.pv_done[i]));
+        }
+        ++p_cnt;
+        ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+        return true;
+    };
+
     for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const Unit U = decode_unit(p, u);
         for (int i = 0; i < kQTiles && ok; ++i)
             ok = wait_phase(sm, sm.q_full[i], unit_iter & 1, kErrTimeoutMma);
         if (!ok) break;
-        ptx::tc_fence_after();
+        uint32_t slot;
+        if (!(ok = next_slot(slot) && issue_s(slot))) break;
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
-            // S_i = Q_i K^T
-            uint32_t slot = it % kSlots;
-            if (!(ok = wait_phase(sm, sm.kv_full[slot], (it / kSlots) & 1, kErrTimeoutMma))) break;
-            ++it;
-            ptx::tc_fence_after();
-            const uint32_t k_base = ptx::smem_addr(sm.kv[slot]);
-            for (int i = 0; i < kQTiles; ++i) {
-                if (pv_cnt[i] > 0 &&
-                    !(ok = wait_phase(sm, sm.pv_done[i], (pv_cnt[i] - 1) & 1, kErrTimeoutMma)))
-                    break;
-                ptx::tc_fence_after();
-                const uint32_t q_base = ptx::smem_addr(sm.q[i]);
-#pragma unroll
-                for (int ks = 0; ks < HD / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
-                    ptx::mma_ss(tmem_s[i], ptx::smem_desc_sw128(q_base + off, 16, 1024),
-                                ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
-                }
-                ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
-            }
-            if (!ok) break;
-            ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
-            // O_i += P_i V
-            slot = it % kSlots;
-            if (!(ok = wait_phase(sm, sm.kv_full[slot], (it / kSlots) & 1, kErrTimeoutMma))) break;
-            ++it;
-            const uint32_t v_base = ptx::smem_addr(sm.kv[slot]);
-            for (int i = 0; i < kQTiles; ++i) {
-                if (!(ok = wait_phase(sm, sm.p_full[i], p_cnt[i] & 1, kErrTimeoutMma))) break;
-                ++p_cnt[i];
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kBN / 16; ++ks) {
-                    ptx::mma_ts(tmem_o[i], tmem_s[i] + ks * 8,
-                                ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
-                                kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
-                }
-                ptx::mma_commit(ptx::smem_addr(&sm.pv_done[i]));
-                ++pv_cnt[i];
-            }
-            if (!ok) break;
-            ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+            if (j + 1 < U.n_tiles && !(ok = next_slot(slot) && issue_s(slot))) break;
+            ok = next_slot(slot) && issue_pv(slot, j == 0);
         }
         if (!ok) break;
         for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
@@ -268,7 +307,11 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
     const uint32_t t_s = tmem + qt * kBN + lane_sel;
     const uint32_t t_o = tmem + 2 * kBN + qt * HD + lane_sel;
     const uint32_t err = kErrTimeoutSoftmax;
-    uint32_t s_cnt = 0, unit_iter = 0;
+    // This row of the P tile: two 64-key column blocks of 128-byte rows with
+    // the 128-byte swizzle (16-byte chunk c of row r stored at c ^ (r & 7)).
+    uint8_t *p_row = sm.pmat[qt] + r * 128;
+    const uint32_t swz = r & 7;
+    uint32_t cnt = 0, unit_iter = 0;   // key tiles processed (all units)
     for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
         const Unit U = decode_unit(p, u);
         const int32_t q = U.q0 + qt * kBM + static_cast<int32_t>(r);
@@ -279,23 +322,18 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             hi = min(lo + p.L, p.N);
         }
         float m_run = kNegInf, l_run = 0.f;
-        for (int32_t j = 0; j < U.n_tiles; ++j) {
-            if (!__all_sync(0xffffffffu, wait_phase(sm, sm.s_full[qt], s_cnt & 1, err))) return;
-            ++s_cnt;
+        for (int32_t j = 0; j < U.n_tiles; ++j, ++cnt) {
+            if (!__all_sync(0xffffffffu, wait_phase(sm, sm.s_full[qt], cnt & 1, err))) return;
             ptx::tc_fence_after();
             uint32_t sr[kBN];
             ptx::tmem_ld128(t_s, sr);
+            // S is in registers: the MMA may overwrite it with the next tile.
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&sm.s_free[qt]));
             // Mask keys outside this row's allowed range.
-            int32_t k0, klo, khi;
-            if (j < U.n_wtiles) {
-                k0 = U.kw0 + j * kBN;
-                klo = lo;
-                khi = hi;
-            } else {
-                k0 = (j - U.n_wtiles) * kBN;
-                klo = 0;
-                khi = p.G;
-            }
+            const int32_t k0 = key_row(U, j);
+            const int32_t klo = j < U.n_wtiles ? lo : 0;
+            const int32_t khi = j < U.n_wtiles ? hi : p.G;
             if (k0 < klo || k0 + kBN > khi) {
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
@@ -311,8 +349,7 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int k = 0; k < w; ++k) m8[k] = fmaxf(m8[k], m8[k + w]);
-            const float mx = m8[0];
-            const float mx2 = mx * p.scale_log2;
+            const float mx2 = m8[0] * p.scale_log2;
             // Lazy rescale: move the running max only when the tile's max
             // exceeds it by more than the threshold (results are exact either
             // way, because O and l share the same reference).
@@ -324,20 +361,9 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
                 m_run = mx2;
             }
             l_run *= alpha;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    ptx::tmem_st32(t_o + c * 32, o);
-                }
-            }
             const float m_use = (m_run == kNegInf) ? 0.f : m_run;
-            // P = exp2(S*scale*log2e - m); the row sum comes from fp32 P,
-            // accumulated in 8 partial sums.
+            // P = exp2(S*scale*log2e - m) as bf16 pairs; the row sum comes
+            // from fp32 P, accumulated in 8 partial sums.
             float sum8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
@@ -350,13 +376,34 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
                 sum8[e & 7] += p0 + p1;
                 pk[e] = ptx::pack_bf16x2(p0, p1);
             }
-            ptx::tmem_st64(t_s, pk);
 #pragma unroll
             for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int k = 0; k < w; ++k) sum8[k] += sum8[k + w];
-            const float sum = sum8[0];
-            l_run += sum;
+            l_run += sum8[0];
+            // The previous P*V must be done before its P is overwritten and
+            // before O is rescaled.
+            if (cnt > 0 &&
+                !__all_sync(0xffffffffu, wait_phase(sm, sm.pv_done[qt], (cnt - 1) & 1, err)))
+                return;
+            ptx::tc_fence_after();
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    ptx::tmem_st32(t_o + c * 32, o);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < kBN / 8; ++c) {
+                uint8_t *dst = p_row + (c / 8) * (kBM * 128) + (((c & 7) ^ swz) << 4);
+                ptx::st_shared_v4(dst, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
+            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
         }
@@ -408,12 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int i = 0; i < kQTiles; ++i) {
             ptx::mbar_init(ptx::smem_addr(&sm.q_full[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.s_full[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.s_free[i]), kBM);
             ptx::mbar_init(ptx::smem_addr(&sm.p_full[i]), kBM);
             ptx::mbar_init(ptx::smem_addr(&sm.pv_done[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.o_final[i]), 1);
         }
         ptx::mbar_init(ptx::smem_addr(&sm.q_empty), 1);
-        for (int s = 0; s < kSlots; ++s) {
+        for (int s = 0; s < Smem<HD>::kSlots; ++s) {
             ptx::mbar_init(ptx::smem_addr(&sm.kv_full[s]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.kv_empty[s]), 1);
         }

@@ -173,6 +173,19 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
         : "memory");
 }
 
+// ---- shared memory stores and proxy fences -----------------------------------
+__device__ __forceinline__ void st_shared_v4(void *dst, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                 :: "r"(smem_addr(dst)), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---- register reallocation between warpgroups ------------------------------
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
