@@ -17,7 +17,8 @@ import os
 import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libatlas.so")
+# The in-tree build; ATLAS_LIBRARY may name another build of the same C-ABI.
+LIB_PATH = os.environ.get("ATLAS_LIBRARY") or os.path.join(HERE, "libatlas.so")
 
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_ALIAS, ERR_CUDA, \
     ERR_TIMEOUT, ERR_DEVICE = range(9)

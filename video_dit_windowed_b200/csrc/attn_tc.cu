@@ -339,17 +339,19 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
                 for (int c = 0; c < kBN; ++c)
                     if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
             }
-            // Row maximum as a tree (8 independent chains, then 3 levels).
+            // Row maximum: 8 independent chains of 3-input max, then a tree.
             float m8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(sr[k]);
 #pragma unroll
-            for (int c = 8; c < kBN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sr[c]));
+            for (int c = 8; c < kBN; c += 16)
 #pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                for (int k = 0; k < w; ++k) m8[k] = fmaxf(m8[k], m8[k + w]);
-            const float mx2 = m8[0] * p.scale_log2;
+                for (int k = 0; k < 8; ++k)
+                    m8[k] = ptx::max3(m8[k], __uint_as_float(sr[c + k]),
+                                      __uint_as_float(sr[c + 8 + k]));
+            const float mx2 = ptx::max3(ptx::max3(m8[0], m8[1], m8[2]),
+                                        ptx::max3(m8[3], m8[4], m8[5]),
+                                        fmaxf(m8[6], m8[7])) * p.scale_log2;
             // Lazy rescale: move the running max only when the tile's max
             // exceeds it by more than the threshold (results are exact either
             // way, because O and l share the same reference).
