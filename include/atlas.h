@@ -46,7 +46,9 @@ typedef enum {
     ATLAS_ERR_ALIAS = 5,       /* input and output overlap where not allowed      */
     ATLAS_ERR_CUDA = 6,        /* a CUDA runtime call or a launch failed          */
     ATLAS_ERR_TIMEOUT = 7,     /* a kernel's bounded wait expired (device word)   */
-    ATLAS_ERR_DEVICE = 8       /* no usable device, or not compute capability 10.0 */
+    ATLAS_ERR_DEVICE = 8,      /* no usable device, or not compute capability 10.0 */
+    ATLAS_ERR_CAPACITY = 9     /* a fixed-size internal buffer is too small (see  */
+                               /* atlas_cube_reorder_noalloc)                     */
 } atlas_status;
 
 typedef enum {
@@ -164,6 +166,40 @@ atlas_status atlas_local_global_attn(
     int64_t n_global, int32_t heads, int32_t head_dim, float softmax_scale,
     atlas_dtype dtype, void *o_d, void *o_g, float *lse,
     atlas_stream_t stream);
+
+/*
+ * atlas_cube_reorder_noalloc -- atlas_cube_reorder without any device
+ * memory allocation. The paper has no counterpart: this is a library
+ * concern. Some callers cannot let a library call cudaMalloc: a serving
+ * process whose device memory is reserved up front by its own allocator and
+ * budget, or a latency-critical loop where cudaMalloc's implicit device-wide
+ * synchronisation is not acceptable. atlas_cube_reorder caches its RoPE
+ * cos/sin table in memory it allocates on first use; this variant keeps the
+ * table in a fixed array compiled into the library instead.
+ *
+ * Arguments, layout, numerics and results are those of atlas_cube_reorder.
+ * Differences:
+ *   - The table lives in one file-scope device array of 32768 (cos, sin)
+ *     pairs (256 KB), held by every GPU that loads the library until the
+ *     process exits. A RoPE needs T*(d_t/2) + H*(d_h/2) + W*(d_w/2) pairs;
+ *     more than 32768 returns ATLAS_ERR_CAPACITY and launches nothing.
+ *   - Each call builds the table on the host and copies it into the array
+ *     on `stream` (from pageable memory: the call returns once the copy has
+ *     been staged), then launches the kernel on `stream`.
+ *   - Every call on a device shares the array and overwrites it: calls whose
+ *     work overlaps on the GPU (for example on two streams) race; issue
+ *     them on one stream or otherwise order them.
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and reads the device
+ *     properties; make that first call before any stream capture.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ * Without rope the call is a pure permutation and touches no table.
+ */
+atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, atlas_grid3 grid,
+                                        atlas_cube3 cube, int32_t heads,
+                                        int32_t head_dim, atlas_dtype dtype,
+                                        const atlas_rope *rope,
+                                        atlas_stream_t stream);
 
 /* Human-readable name of a status. Never NULL. */
 const char *atlas_status_string(atlas_status status);

@@ -21,7 +21,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("ATLAS_LIBRARY") or os.path.join(HERE, "libatlas.so")
 
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_ALIAS, ERR_CUDA, \
-    ERR_TIMEOUT, ERR_DEVICE = range(9)
+    ERR_TIMEOUT, ERR_DEVICE, ERR_CAPACITY = range(10)
 BF16, FP32 = 0, 1
 
 
@@ -63,6 +63,8 @@ def _declare(lib):
     lib.atlas_cube_reorder.restype = ctypes.c_int
     lib.atlas_cube_reorder.argtypes = [_vp, _vp, Grid3, Cube3, _i32, _i32, ctypes.c_int,
                                        ctypes.POINTER(Rope), _vp]
+    lib.atlas_cube_reorder_noalloc.restype = ctypes.c_int
+    lib.atlas_cube_reorder_noalloc.argtypes = lib.atlas_cube_reorder.argtypes
     lib.atlas_cube_unorder.restype = ctypes.c_int
     lib.atlas_cube_unorder.argtypes = [_vp, _vp, Grid3, Cube3, _i32, _i32, ctypes.c_int, _vp]
     lib.atlas_rope3d.restype = ctypes.c_int
@@ -143,6 +145,18 @@ def cube_reorder(src, dst, grid, cube, rope: Rope | None = None, stream=None):
         _ptr(src), _ptr(dst), Grid3(*grid), Cube3(*cube), heads, hd, _dtype_code(src),
         ctypes.byref(rope) if rope is not None else None, _stream(src, stream))
     _check(st, "atlas_cube_reorder")
+    return dst
+
+
+def cube_reorder_noalloc(src, dst, grid, cube, rope: Rope | None = None, stream=None):
+    """``cube_reorder`` through the entry point that allocates no device
+    memory (its RoPE table sits in a fixed 32768-pair array shared by all
+    calls on the device; overlapping calls race, see include/atlas.h)."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_reorder_noalloc(
+        _ptr(src), _ptr(dst), Grid3(*grid), Cube3(*cube), heads, hd, _dtype_code(src),
+        ctypes.byref(rope) if rope is not None else None, _stream(src, stream))
+    _check(st, "atlas_cube_reorder_noalloc")
     return dst
 
 

@@ -113,6 +113,25 @@ ATLAS_API atlas_status atlas_cube_reorder(const void *src, void *dst, atlas_grid
     return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+ATLAS_API atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, atlas_grid3 grid,
+                                                  atlas_cube3 cube, int32_t heads,
+                                                  int32_t head_dim, atlas_dtype dtype,
+                                                  const atlas_rope *rope,
+                                                  atlas_stream_t stream) {
+    if (!src || !dst) return ATLAS_ERR_NULL;
+    atlas_status st = check_grid(grid, heads, head_dim, dtype);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
+    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
+                         elem_bytes(dtype);
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), 0, rope};
+    return launch_permute_rope_noalloc(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 ATLAS_API atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, atlas_stream_t stream) {
@@ -195,6 +214,7 @@ ATLAS_API const char *atlas_status_string(atlas_status status) {
         case ATLAS_ERR_CUDA: return "ATLAS_ERR_CUDA: a CUDA call or launch failed";
         case ATLAS_ERR_TIMEOUT: return "ATLAS_ERR_TIMEOUT: a kernel's bounded wait expired";
         case ATLAS_ERR_DEVICE: return "ATLAS_ERR_DEVICE: no compute capability 10.0 device";
+        case ATLAS_ERR_CAPACITY: return "ATLAS_ERR_CAPACITY: fixed internal buffer too small";
     }
     return "ATLAS_ERR_UNKNOWN";
 }

@@ -72,6 +72,9 @@ struct PermuteArgs {
 };
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
 atlas_status release_rope_tables();
+// Reorder (+RoPE) with the cos/sin table in a fixed device array (no
+// allocation); ATLAS_ERR_CAPACITY if the table would not fit.
+atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stream);
 
 struct AttnArgs {
     const void *q_d, *k_d, *v_d;

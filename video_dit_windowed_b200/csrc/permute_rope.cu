@@ -315,6 +315,82 @@ atlas_status dispatch(const Params &p, bool rope, int mode, const DeviceInfo &de
     return launch<EB, false, 1>(p, dev, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Variant that allocates nothing (atlas_cube_reorder_noalloc): the cos/sin
+// table lives in a fixed file-scope device array instead of a cached
+// cudaMalloc'd buffer. Every call on a device shares the array, so calls that
+// overlap on the GPU (e.g. on two streams) race on its contents.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticRopeEntries = 32768;  // 256 KB of (cos, sin) per device
+static __device__ __align__(256) float2 g_static_rope_table[kStaticRopeEntries];
+
+std::mutex g_static_mutex;                      // guards the two arrays below
+float2 g_static_host_table[kStaticRopeEntries];  // host staging, reused per call
+float2 *g_static_table_dev[64] = {nullptr};      // device address, per device
+
+// Device address of the static table on `device` (the current device). The
+// array's name is only a host-side stand-in; its address is resolved once per
+// device with that device current. Caller holds g_static_mutex.
+atlas_status static_table_address(int device, float2 **out) {
+    if (device < 0 || device >= 64) return ATLAS_ERR_DEVICE;
+    if (g_static_table_dev[device] == nullptr) {
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_static_rope_table) != cudaSuccess)
+            return ATLAS_ERR_CUDA;
+        g_static_table_dev[device] = static_cast<float2 *>(addr);
+    }
+    *out = g_static_table_dev[device];
+    return ATLAS_OK;
+}
+
+size_t rope_table_entries(int64_t T, int64_t H, int64_t W, const atlas_rope &r) {
+    return static_cast<size_t>(T) * (r.d_t / 2) + static_cast<size_t>(H) * (r.d_h / 2) +
+           static_cast<size_t>(W) * (r.d_w / 2);
+}
+
+// Same layout and arithmetic as the cached table (fp64 angles, rounded once).
+void fill_rope_table(float2 *out, int64_t T, int64_t H, int64_t W, const atlas_rope &r) {
+    const int64_t ext[3] = {T, H, W};
+    const int32_t width[3] = {r.d_t, r.d_h, r.d_w};
+    const double scale[3] = {r.scale_t, r.scale_h, r.scale_w};
+    size_t n = 0;
+    for (int a = 0; a < 3; ++a)
+        for (int64_t c = 0; c < ext[a]; ++c)
+            for (int32_t k = 0; k < width[a] / 2; ++k) {
+                double omega = std::pow(r.theta, -2.0 * k / static_cast<double>(width[a]));
+                double phi = (static_cast<double>(c) * scale[a]) * omega;
+                out[n++] = make_float2(static_cast<float>(std::cos(phi)),
+                                       static_cast<float>(std::sin(phi)));
+            }
+}
+
+void fill_geometry(Params &p, const PermuteArgs &a) {
+    p.src = static_cast<const uint8_t *>(a.src);
+    p.dst = static_cast<uint8_t *>(a.dst);
+    p.rows = static_cast<uint32_t>(a.T * a.H * a.W);
+    p.heads = static_cast<uint32_t>(a.heads);
+    p.row_vecs = static_cast<uint32_t>(static_cast<int64_t>(a.heads) * a.head_dim *
+                                       a.elem_bytes / 16);
+    p.vph = static_cast<uint32_t>(a.head_dim * a.elem_bytes / 16);
+    Geom &g = p.g;
+    g.H = static_cast<uint32_t>(a.H);
+    g.W = static_cast<uint32_t>(a.W);
+    g.ct = static_cast<uint32_t>(a.ct);
+    g.ch = static_cast<uint32_t>(a.ch);
+    g.cw = static_cast<uint32_t>(a.cw);
+    g.cubes_h = g.H / g.ch;
+    g.cubes_w = g.W / g.cw;
+    g.L = g.ct * g.ch * g.cw;
+    g.by_W = FastDiv(g.W);
+    g.by_H = FastDiv(g.H);
+    g.by_ct = FastDiv(g.ct);
+    g.by_ch = FastDiv(g.ch);
+    g.by_cw = FastDiv(g.cw);
+    g.by_cubes_w = FastDiv(g.cubes_w);
+    g.by_cubes_h = FastDiv(g.cubes_h);
+    g.by_L = FastDiv(g.L);
+}
+
 }  // namespace
 
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream) {
@@ -375,6 +451,40 @@ atlas_status release_rope_tables() {
     g_tables.clear();
     cudaSetDevice(cur);
     return st;
+}
+
+atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stream) {
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    Params p{};
+    fill_geometry(p, a);
+    if (a.rope == nullptr) {
+        if (a.elem_bytes == 2) return dispatch<2>(p, false, 0, dev, stream);
+        return dispatch<4>(p, false, 0, dev, stream);
+    }
+    const atlas_rope &r = *a.rope;
+    const size_t n = rope_table_entries(a.T, a.H, a.W, r);
+    if (n > kStaticRopeEntries) return ATLAS_ERR_CAPACITY;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    float2 *tab = nullptr;
+    atlas_status st = static_table_address(dev.device, &tab);
+    if (st != ATLAS_OK) return st;
+    fill_rope_table(g_static_host_table, a.T, a.H, a.W, r);
+    // From pageable host memory: returns once the staging copy is taken, so
+    // the host buffer may be refilled by the next call; ordered on `stream`
+    // before the kernel.
+    if (n > 0 && cudaMemcpyAsync(tab, g_static_host_table, n * sizeof(float2),
+                                 cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return ATLAS_ERR_CUDA;
+    p.tab = tab;
+    p.half[0] = static_cast<uint32_t>(r.d_t / 2);
+    p.half[1] = static_cast<uint32_t>(r.d_h / 2);
+    p.half[2] = static_cast<uint32_t>(r.d_w / 2);
+    p.tab_base[0] = 0;
+    p.tab_base[1] = static_cast<uint32_t>(a.T) * p.half[0];
+    p.tab_base[2] = p.tab_base[1] + static_cast<uint32_t>(a.H) * p.half[1];
+    if (a.elem_bytes == 2) return dispatch<2>(p, true, 0, dev, stream);
+    return dispatch<4>(p, true, 0, dev, stream);
 }
 
 }  // namespace atlas
