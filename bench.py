@@ -53,7 +53,9 @@ def peaks():
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 100 ms from start() to stop(); only the samples
+    stamped inside the timed region (window()) are summarised."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -66,7 +68,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -77,7 +79,11 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def window(self, t0: float, t1: float):
+        self.t0, self.t1 = t0, t1
+
     def stop(self):
+        import datetime
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -90,14 +96,18 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, clk_max = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[4:8]):
+            if not (getattr(self, "t0", 0) <= ts <= getattr(self, "t1", 1e30)):
+                continue
+            sm.append(clk)
+            mx.append(clk_max)
+            for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
@@ -330,9 +340,11 @@ def run_atlas(args, world, rank, local):
         raise RuntimeError(f"device error word 0x{code:x} after warm-up")
 
     clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)            # let nvidia-smi start sampling before the timed region
     barrier(world)
     torch.cuda.synchronize(dev)
-    clocks.start()
+    t_wall0 = time.time()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -341,6 +353,7 @@ def run_atlas(args, world, rank, local):
         path.step(evs[i])
     stop.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.window(t_wall0, time.time())
     barrier(world)
     clk = clocks.stop()
     elapsed = start.elapsed_time(stop)
@@ -446,7 +459,7 @@ def run_e2e(path, w, dev, stream, args, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="atlas", choices=["atlas", "reference"])
     ap.add_argument("--workload", default="720p", choices=sorted(WORKLOADS))
