@@ -174,6 +174,12 @@ def bytes_reorder_rope(w):
     return 2 * 3 * w.n_detail * row, 2 * 2 * w.n_global * row
 
 
+def attn_bytes(w):
+    """Minimum DRAM bytes of one attention launch: Q, K, V read once, O written."""
+    row = w.heads * w.head_dim * w.elem_bytes
+    return (3 * (w.n_detail + w.n_global) + (w.n_detail + w.n_global)) * row
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "video_dit_windowed_b200", "csrc")
@@ -183,17 +189,24 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def measured_traffic():
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
+def measured_traffic(w):
+    """Per-launch DRAM bytes of the attention kernel for workload ``w``, from
+    the committed ncu summary if it was taken on the current kernel source and
+    the same workload geometry (scaled by the head count); else None."""
+    path = os.path.join(ROOT, "profiles", "attn_tc_traffic.txt")
     if not os.path.exists(path):
         return None
+    d = {}
     with open(path) as f:
-        d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#") and "=" in line:
+                k, v = line.split("=", 1)
+                d[k.strip()] = v.strip()
+    if d.get("source_hash") != kernel_source_hash() or d.get("workload") != w.name:
         return None
-    return d
+    per_head = (int(d["dram_read_bytes"]) + int(d["dram_write_bytes"])) / int(d["heads"])
+    return per_head * w.heads
 
 
 # ---------------------------------------------------------------------------
@@ -384,7 +397,7 @@ def run_atlas(args, world, rank, local):
     rr_gbs = (b_d + b_g) / (rr_ms * 1e-3) / 1e9 if rr_ms > 0 else None
     un_ms = statistics.median(phases["unorder"])
     un_bytes = 2 * w.n_detail * w.heads * w.head_dim * w.elem_bytes
-    traffic = measured_traffic()
+    traffic = measured_traffic(w)
     peak_tf = pk["bf16_tflops_sustained"]
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -400,7 +413,8 @@ def run_atlas(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": attn_tf,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
                      "peak_kind": f"{pk_kind} bf16 sustained",
-                     "traffic": traffic["bytes_per_launch"] if traffic else None},
+                     "traffic": traffic,
+                     "algorithmic_bytes": attn_bytes(w)},
         "roofline_reorder_rope": {"bound": "hbm", "achieved": rr_gbs, "peak": pk["hbm_gbs"],
                                   "unit": "GB/s",
                                   "frac": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
