@@ -309,7 +309,8 @@ def run_reference(args, world, rank):
         return
     w = workload(args)
     times = []
-    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    # each step a bounded sample: the whole --steps/--warmup run stays near a minute
+    budget = max(0.5, min(args.cpu_budget, 60.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
         tf, cores, sample, t = time_oracle(w, budget_s=budget, seed=i)
         if i >= args.warmup:
