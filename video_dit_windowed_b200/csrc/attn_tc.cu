@@ -22,11 +22,15 @@
 //                    shared-memory slots, in the order the MMAs use them),
 //   warp 9           tensor-memory owner and MMA issuer (one thread),
 //   warps 10-11      idle (complete the third warpgroup for the register split).
-// Tensor memory (512 columns): S0 | S1 | O0 | O1 (fp32). P (bf16) goes to
-// shared memory, so S of the next key tile can be computed as soon as the
-// softmax has loaded S of this one. The MMA issue order per key tile j is
-//   S0(j+1), S1(j+1), O0 += P0(j) V(j), O1 += P1(j) V(j),
-// which gives each softmax the time of about four MMAs to produce P(j).
+// Tensor memory (512 columns): S0 | S1 | O0 | O1 (fp32). The softmax writes
+// P (bf16) over the first half of its S columns and the P*V MMA reads it from
+// tensor memory, so P costs no shared-memory traffic. The MMA issue order per
+// key tile j is
+//   O0 += P0(j) V(j), S0(j+1), O1 += P1(j) V(j), S1(j+1).
+// MMAs issued by one thread execute in order: S_i(j+1) overwrites P_i(j) only
+// after O_i += P_i(j) V(j) has read it, and a commit after S_i(j+1) also
+// covers O_i += P_i(j) V(j). Each softmax therefore has the time of the other
+// tile's two MMAs to produce its P.
 // Every wait is bounded: on expiry a bit is set in the device error word,
 // the CTA drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -61,21 +65,17 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 
 template <int HD>
 struct Smem {
-    static constexpr int kTileBytes = kBM * HD * 2;     // one 128-row bf16 Q/K/V tile
-    static constexpr int kPBytes = kBM * kBN * 2;       // one 128 x 128 bf16 P tile
-    static constexpr int kSlots = (96 * 1024) / kTileBytes;  // K/V ring: 96 KB
+    static constexpr int kTileBytes = kBM * HD * 2;           // one 128-row bf16 tile
+    static constexpr int kSlots = (160 * 1024) / kTileBytes;  // K/V ring: 160 KB
     alignas(1024) uint8_t q[kQTiles][kTileBytes];
-    alignas(1024) uint8_t pmat[kQTiles][kPBytes];
     alignas(1024) uint8_t kv[kSlots][kTileBytes];
     uint64_t q_full[kQTiles];
     uint64_t q_empty;
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];
-    uint64_t s_full[kQTiles];    // S(j) is in TMEM               (MMA commit)
-    uint64_t s_free[kQTiles];    // softmax has loaded S(j)       (128 arrivals)
-    uint64_t p_full[kQTiles];    // P(j) in smem, O rescaled      (128 arrivals)
-    uint64_t pv_done[kQTiles];   // O += P(j) V(j) finished       (MMA commit)
-    uint64_t o_final[kQTiles];   // every MMA of the unit done    (MMA commit)
+    uint64_t s_full[kQTiles];    // S_i(j) is in TMEM (and O_i += P_i(j-1)V done)  (commit)
+    uint64_t p_full[kQTiles];    // P_i(j) in TMEM, O_i rescaled         (128 arrivals)
+    uint64_t o_final[kQTiles];   // every MMA of the unit done           (commit)
     uint64_t drain;
     uint32_t tmem_base;
     volatile int abort;
@@ -145,8 +145,8 @@ __device__ __forceinline__ int32_t key_row(const Unit &U, int32_t j) {
 }
 
 // ---------------------------------------------------------------------------
-// Producer: Q tiles once per unit, then K/V tiles in MMA order:
-// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1).
+// Producer: Q tiles once per unit, then K(0), V(0), K(1), V(1), ... in the
+// order the MMAs consume them.
 // ---------------------------------------------------------------------------
 template <int HD>
 __device__ void producer(const Params &p, Smem<HD> &sm) {
@@ -193,12 +193,11 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
                                  U.head, U.q0 + i * kBM);
         }
         q_armed = unit_iter + 1;
-        auto kmap = [&](int32_t j) { return j < U.n_wtiles ? &p.tm_kd : &p.tm_kg; };
-        auto vmap = [&](int32_t j) { return j < U.n_wtiles ? &p.tm_vd : &p.tm_vg; };
-        ok = load(kmap(0), U.head, key_row(U, 0));
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
-            if (j + 1 < U.n_tiles && !(ok = load(kmap(j + 1), U.head, key_row(U, j + 1)))) break;
-            ok = load(vmap(j), U.head, key_row(U, j));
+            const bool win = j < U.n_wtiles;
+            const int32_t row = key_row(U, j);
+            ok = load(win ? &p.tm_kd : &p.tm_kg, U.head, row) &&
+                 load(win ? &p.tm_vd : &p.tm_vg, U.head, row);
         }
     }
     if (!ok) {
@@ -213,7 +212,8 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (one thread).
+// MMA issuer (one thread). Per unit: S0(0), S1(0); then for each key tile j:
+// O0 += P0(j)V(j), S0(j+1), O1 += P1(j)V(j), S1(j+1).
 // ---------------------------------------------------------------------------
 template <int HD>
 __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
@@ -221,8 +221,7 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, HD, 1);
     uint32_t it = 0, unit_iter = 0;
-    uint32_t s_cnt = 0;   // S tiles issued per Q tile (same for both)
-    uint32_t p_cnt = 0;   // P tiles consumed per Q tile
+    uint32_t p_cnt = 0;   // P tiles consumed per Q tile (both tiles move together)
     bool ok = true;
 
     auto next_slot = [&](uint32_t &slot) -> bool {
@@ -232,47 +231,28 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         ptx::tc_fence_after();
         return r;
     };
-    // S_i = Q_i K^T for both Q tiles from the K tile in `slot`.
-    auto issue_s = [&](uint32_t slot) -> bool {
-        const uint32_t k_base = ptx::smem_addr(sm.kv[slot]);
+    // S_i = Q_i K^T from the K tile in `slot`.
+    auto issue_s = [&](int i, uint32_t k_slot) {
+        const uint32_t k_base = ptx::smem_addr(sm.kv[k_slot]);
+        const uint32_t q_base = ptx::smem_addr(sm.q[i]);
 #pragma unroll
-        for (int i = 0; i < kQTiles; ++i) {
-            if (s_cnt > 0 &&
-                !wait_phase(sm, sm.s_free[i], (s_cnt - 1) & 1, kErrTimeoutMma))
-                return false;
-            ptx::tc_fence_after();
-            const uint32_t q_base = ptx::smem_addr(sm.q[i]);
-#pragma unroll
-            for (int ks = 0; ks < HD / 16; ++ks) {
-                const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
-                ptx::mma_ss(tmem + i * kBN, ptx::smem_desc_sw128(q_base + off, 16, 1024),
-                            ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
-            }
-            ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
+        for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
+            ptx::mma_ss(tmem + i * kBN, ptx::smem_desc_sw128(q_base + off, 16, 1024),
+                        ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
         }
-        ++s_cnt;
-        ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
-        return true;
+        ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
     };
-    // O_i += P_i V for both Q tiles from the V tile in `slot`.
-    auto issue_pv = [&](uint32_t slot, bool first) -> bool {
-        const uint32_t v_base = ptx::smem_addr(sm.kv[slot]);
+    // O_i += P_i V, P_i from tensor memory, from the V tile in `slot`.
+    auto issue_pv = [&](int i, uint32_t v_slot, bool first) -> bool {
+        if (!wait_phase(sm, sm.p_full[i], p_cnt & 1, kErrTimeoutMma)) return false;
+        ptx::tc_fence_after();
+        const uint32_t v_base = ptx::smem_addr(sm.kv[v_slot]);
 #pragma unroll
-        for (int i = 0; i < kQTiles; ++i) {
-            if (!wait_phase(sm, sm.p_full[i], p_cnt & 1, kErrTimeoutMma)) return false;
-            ptx::tc_fence_after();
-            const uint32_t p_base = ptx::smem_addr(sm.pmat[i]);
-#pragma unroll
-            for (int ks = 0; ks < kBN / 16; ++ks) {
-                const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
-                ptx::mma_ss(tmem + 2 * kBN + i * HD, ptx::smem_desc_sw128(p_base + off, 16, 1024),
-                            ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
-                            kIdescPV, (!first || ks > 0) ? 1u : 0u);
-            }
-            ptx::mma_commit(ptx::smem_addr(&sm.pv_done[i]));
-        }
-        ++p_cnt;
-        ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[slot]));
+        for (int ks = 0; ks < kBN / 16; ++ks)
+            ptx::mma_ts(tmem + 2 * kBN + i * HD, tmem + i * kBN + ks * 8,
+                        ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
+                        kIdescPV, (!first || ks > 0) ? 1u : 0u);
         return true;
     };
 
@@ -281,11 +261,27 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         for (int i = 0; i < kQTiles && ok; ++i)
             ok = wait_phase(sm, sm.q_full[i], unit_iter & 1, kErrTimeoutMma);
         if (!ok) break;
-        uint32_t slot;
-        if (!(ok = next_slot(slot) && issue_s(slot))) break;
+        ptx::tc_fence_after();
+        uint32_t k_slot, v_slot;
+        if (!(ok = next_slot(k_slot))) break;
+        issue_s(0, k_slot);
+        issue_s(1, k_slot);
+        ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
-            if (j + 1 < U.n_tiles && !(ok = next_slot(slot) && issue_s(slot))) break;
-            ok = next_slot(slot) && issue_pv(slot, j == 0);
+            const bool more = j + 1 < U.n_tiles;
+            // ring order: V(j) was loaded before K(j+1)
+            if (!(ok = next_slot(v_slot)) || !(ok = issue_pv(0, v_slot, j == 0))) break;
+            if (more) {
+                if (!(ok = next_slot(k_slot))) break;
+                issue_s(0, k_slot);
+            }
+            if (!(ok = issue_pv(1, v_slot, j == 0))) break;
+            if (more) {
+                issue_s(1, k_slot);
+                ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
+            }
+            ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[v_slot]));
+            ++p_cnt;
         }
         if (!ok) break;
         for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
@@ -304,13 +300,99 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
     const uint32_t warp = (threadIdx.x / 32) & 3;
     const uint32_t r = threadIdx.x & 127;                 // row within the tile
     const uint32_t lane_sel = (warp * 32u) << 16;         // TMEM lane field
-    const uint32_t t_s = tmem + qt * kBN + lane_sel;
+    const uint32_t t_s = tmem + qt * kBN + lane_sel;      // S, then P over its first half
     const uint32_t t_o = tmem + 2 * kBN + qt * HD + lane_sel;
     const uint32_t err = kErrTimeoutSoftmax;
-    // This row of the P tile: two 64-key column blocks of 128-byte rows with
-    // the 128-byte swizzle (16-byte chunk c of row r stored at c ^ (r & 7)).
-    uint8_t *p_row = sm.pmat[qt] + r * 128;
-    const uint32_t swz = r & 7;
+    const float sc = p.scale_log2;
+    constexpr uint32_t kAll = 0xffffffffu;
+
+    // P = exp2(S*scale*log2e - m) as bf16 pairs into tensor memory (two
+    // stores of 32 columns); returns the row sum of the fp32 P.
+    auto exp_store = [&](const uint32_t (&sr)[kBN], float m) -> float {
+        float sum8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int c = half * 64 + 2 * e;
+                const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c]), sc, -m));
+                const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -m));
+                sum8[e & 7] += p0 + p1;
+                pk[e] = ptx::pack_bf16x2(p0, p1);
+            }
+            ptx::tmem_st32_nowait(t_s + half * 32, pk);
+        }
+        ptx::tmem_wait_st();
+#pragma unroll
+        for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+            for (int k = 0; k < w; ++k) sum8[k] += sum8[k + w];
+        return sum8[0];
+    };
+    // The same, with the row maximum of the raw S taken in the same pass.
+    auto exp_store_max = [&](const uint32_t (&sr)[kBN], float m, float &mx) -> float {
+        float sum8[8], m8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            sum8[k] = 0.f;
+            m8[k] = kNegInf;
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int c = half * 64 + 2 * e;
+                const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+                m8[e & 7] = ptx::max3(m8[e & 7], s0, s1);
+                const float p0 = ptx::ex2(fmaf(s0, sc, -m));
+                const float p1 = ptx::ex2(fmaf(s1, sc, -m));
+                sum8[e & 7] += p0 + p1;
+                pk[e] = ptx::pack_bf16x2(p0, p1);
+            }
+            ptx::tmem_st32_nowait(t_s + half * 32, pk);
+        }
+        ptx::tmem_wait_st();
+#pragma unroll
+        for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+            for (int k = 0; k < w; ++k) {
+                sum8[k] += sum8[k + w];
+                m8[k] = fmaxf(m8[k], m8[k + w]);
+            }
+        mx = m8[0];
+        return sum8[0];
+    };
+    auto row_max = [&](const uint32_t (&sr)[kBN]) -> float {
+        float m8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(sr[k]);
+#pragma unroll
+        for (int c = 8; c < kBN; c += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                m8[k] = ptx::max3(m8[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+        return ptx::max3(ptx::max3(m8[0], m8[1], m8[2]), ptx::max3(m8[3], m8[4], m8[5]),
+                         fmaxf(m8[6], m8[7]));
+    };
+    // O *= alpha (only warps where some row moved its reference). The P*V of
+    // the previous key tile has completed: the commit that signalled this S
+    // covers it.
+    auto rescale_o = [&](bool need, float alpha) {
+        if (!__any_sync(kAll, need)) return;
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            ptx::tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            ptx::tmem_st32(t_o + c * 32, o);
+        }
+    };
+
     uint32_t cnt = 0, unit_iter = 0;   // key tiles processed (all units)
     for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
         const Unit U = decode_unit(p, u);
@@ -323,89 +405,53 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         }
         float m_run = kNegInf, l_run = 0.f;
         for (int32_t j = 0; j < U.n_tiles; ++j, ++cnt) {
-            if (!__all_sync(0xffffffffu, wait_phase(sm, sm.s_full[qt], cnt & 1, err))) return;
+            if (!__all_sync(kAll, wait_phase(sm, sm.s_full[qt], cnt & 1, err))) return;
             ptx::tc_fence_after();
             uint32_t sr[kBN];
             ptx::tmem_ld128(t_s, sr);
-            // S is in registers: the MMA may overwrite it with the next tile.
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_addr(&sm.s_free[qt]));
             // Mask keys outside this row's allowed range.
             const int32_t k0 = key_row(U, j);
             const int32_t klo = j < U.n_wtiles ? lo : 0;
             const int32_t khi = j < U.n_wtiles ? hi : p.G;
-            if (k0 < klo || k0 + kBN > khi) {
+            const bool row_masked = k0 < klo || k0 + kBN > khi;
+            if (row_masked) {
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
                     if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
             }
-            // Row maximum: 8 independent chains of 3-input max, then a tree.
-            float m8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(sr[k]);
-#pragma unroll
-            for (int c = 8; c < kBN; c += 16)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    m8[k] = ptx::max3(m8[k], __uint_as_float(sr[c + k]),
-                                      __uint_as_float(sr[c + 8 + k]));
-            const float mx2 = ptx::max3(ptx::max3(m8[0], m8[1], m8[2]),
-                                        ptx::max3(m8[3], m8[4], m8[5]),
-                                        fmaxf(m8[6], m8[7])) * p.scale_log2;
-            // Lazy rescale: move the running max only when the tile's max
-            // exceeds it by more than the threshold (results are exact either
-            // way, because O and l share the same reference).
-            const bool need = (m_run == kNegInf) ? (mx2 != kNegInf)
-                                                 : (mx2 > m_run + kRescaleThreshold);
-            float alpha = 1.f;
-            if (need) {
-                alpha = (m_run == kNegInf) ? 0.f : ptx::ex2(m_run - mx2);
-                m_run = mx2;
-            }
-            l_run *= alpha;
-            const float m_use = (m_run == kNegInf) ? 0.f : m_run;
-            // P = exp2(S*scale*log2e - m) as bf16 pairs; the row sum comes
-            // from fp32 P, accumulated in 8 partial sums.
-            float sum8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
-            uint32_t pk[kBN / 2];
-#pragma unroll
-            for (int e = 0; e < kBN / 2; ++e) {
-                const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -m_use));
-                const float p1 =
-                    ptx::ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -m_use));
-                sum8[e & 7] += p0 + p1;
-                pk[e] = ptx::pack_bf16x2(p0, p1);
-            }
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                for (int k = 0; k < w; ++k) sum8[k] += sum8[k + w];
-            l_run += sum8[0];
-            // The previous P*V must be done before its P is overwritten and
-            // before O is rescaled.
-            if (cnt > 0 &&
-                !__all_sync(0xffffffffu, wait_phase(sm, sm.pv_done[qt], (cnt - 1) & 1, err)))
-                return;
-            ptx::tc_fence_after();
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    ptx::tmem_st32(t_o + c * 32, o);
+            float sum;
+            if (__any_sync(kAll, m_run == kNegInf || row_masked)) {
+                // No reference yet, or masked keys: row max first. The
+                // reference moves only when the tile's max exceeds it by more
+                // than the threshold (exact either way: O and l share it).
+                const float mx2 = row_max(sr) * sc;
+                const bool need = (m_run == kNegInf) ? (mx2 != kNegInf)
+                                                     : (mx2 > m_run + kRescaleThreshold);
+                float alpha = 1.f;
+                if (need) {
+                    alpha = (m_run == kNegInf) ? 0.f : ptx::ex2(m_run - mx2);
+                    m_run = mx2;
+                }
+                l_run *= alpha;
+                if (j > 0) rescale_o(need, alpha);
+                sum = exp_store(sr, m_run == kNegInf ? 0.f : m_run);
+            } else {
+                // Exponentials against the running reference right away, the
+                // tile max in the same pass; redo the (rare) rows whose max
+                // moved past the threshold.
+                float mx;
+                sum = exp_store_max(sr, m_run, mx);
+                const float mx2 = mx * sc;
+                const bool need = mx2 > m_run + kRescaleThreshold;
+                if (__any_sync(kAll, need)) {
+                    const float alpha = need ? ptx::ex2(m_run - mx2) : 1.f;
+                    if (need) m_run = mx2;
+                    l_run *= alpha;
+                    rescale_o(need, alpha);
+                    sum = exp_store(sr, m_run);
                 }
             }
-#pragma unroll
-            for (int c = 0; c < kBN / 8; ++c) {
-                uint8_t *dst = p_row + (c / 8) * (kBM * 128) + (((c & 7) ^ swz) << 4);
-                ptx::st_shared_v4(dst, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            }
-            ptx::fence_proxy_async_smem();
+            l_run += sum;
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
         }
@@ -457,9 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int i = 0; i < kQTiles; ++i) {
             ptx::mbar_init(ptx::smem_addr(&sm.q_full[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.s_full[i]), 1);
-            ptx::mbar_init(ptx::smem_addr(&sm.s_free[i]), kBM);
             ptx::mbar_init(ptx::smem_addr(&sm.p_full[i]), kBM);
-            ptx::mbar_init(ptx::smem_addr(&sm.pv_done[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.o_final[i]), 1);
         }
         ptx::mbar_init(ptx::smem_addr(&sm.q_empty), 1);
