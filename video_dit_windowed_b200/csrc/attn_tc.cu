@@ -231,15 +231,22 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         ptx::tc_fence_after();
         return r;
     };
+    // Descriptor words, computed once: the loops below only add constant
+    // offsets (bytes >> 4) to the low word.
+    constexpr uint32_t kHi = ptx::desc_sw128_hi(1024);
+    const uint32_t q_lo0 = ptx::desc_sw128_lo(ptx::smem_addr(sm.q[0]), 16);
+    const uint32_t k_lo0 = ptx::desc_sw128_lo(ptx::smem_addr(sm.kv[0]), 16);
+    const uint32_t v_lo0 = ptx::desc_sw128_lo(ptx::smem_addr(sm.kv[0]), kBN * 128);
+    constexpr uint32_t kTile16 = Smem<HD>::kTileBytes >> 4;
     // S_i = Q_i K^T from the K tile in `slot`.
     auto issue_s = [&](int i, uint32_t k_slot) {
-        const uint32_t k_base = ptx::smem_addr(sm.kv[k_slot]);
-        const uint32_t q_base = ptx::smem_addr(sm.q[i]);
+        const uint32_t q_lo = q_lo0 + i * kTile16, k_lo = k_lo0 + k_slot * kTile16;
+        const uint32_t d_s = tmem + i * kBN;
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint32_t off = (ks / 4) * (kBM * 128) + (ks % 4) * 32;
-            ptx::mma_ss(tmem + i * kBN, ptx::smem_desc_sw128(q_base + off, 16, 1024),
-                        ptx::smem_desc_sw128(k_base + off, 16, 1024), kIdescQK, ks > 0);
+            const uint32_t off = ((ks / 4) * (kBM * 128) + (ks % 4) * 32) >> 4;
+            ptx::mma_ss(d_s, ptx::desc_join(q_lo + off, kHi), ptx::desc_join(k_lo + off, kHi),
+                        kIdescQK, ks > 0);
         }
         ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
     };
@@ -247,12 +254,13 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     auto issue_pv = [&](int i, uint32_t v_slot, bool first) -> bool {
         if (!wait_phase(sm, sm.p_full[i], p_cnt & 1, kErrTimeoutMma)) return false;
         ptx::tc_fence_after();
-        const uint32_t v_base = ptx::smem_addr(sm.kv[v_slot]);
+        const uint32_t v_lo = v_lo0 + v_slot * kTile16;
+        const uint32_t d_o = tmem + 2 * kBN + i * HD, a_p = tmem + i * kBN;
+        ptx::mma_ts(d_o, a_p, ptx::desc_join(v_lo, kHi), kIdescPV, first ? 0u : 1u);
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks)
-            ptx::mma_ts(tmem + 2 * kBN + i * HD, tmem + i * kBN + ks * 8,
-                        ptx::smem_desc_sw128(v_base + ks * 16 * 128, kBN * 128, 1024),
-                        kIdescPV, (!first || ks > 0) ? 1u : 0u);
+        for (int ks = 1; ks < kBN / 16; ++ks)
+            ptx::mma_ts(d_o, a_p + ks * 8, ptx::desc_join(v_lo + ((ks * 16 * 128) >> 4), kHi),
+                        kIdescPV, 1u);
         return true;
     };
 
