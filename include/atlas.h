@@ -212,6 +212,18 @@ const char *atlas_status_string(atlas_status status);
  */
 atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *code);
 
+/*
+ * Failure-path test hook. The next bf16 atlas_local_global_attn launch (any
+ * thread, any device) leaves the first K tile of its first work unit
+ * unloaded. The waits that depend on it expire after their bounded limit
+ * (about 2 s): that CTA records ATLAS_ERR_TIMEOUT bits in the device error
+ * word, drains its in-flight copies and MMAs, frees tensor memory and exits,
+ * and its output rows are left incomplete. No fault, trap or hang is
+ * involved, and the context stays usable. atlas_last_device_error then
+ * returns ATLAS_ERR_TIMEOUT. One-shot; always ATLAS_OK.
+ */
+atlas_status atlas_debug_stall_next_attention(void);
+
 /* Free the cached RoPE tables of every device (synchronises the device). */
 atlas_status atlas_release_caches(void);
 

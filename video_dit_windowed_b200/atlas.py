@@ -78,6 +78,8 @@ def _declare(lib):
     lib.atlas_status_string.argtypes = [ctypes.c_int]
     lib.atlas_last_device_error.restype = ctypes.c_int
     lib.atlas_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.atlas_debug_stall_next_attention.restype = ctypes.c_int
+    lib.atlas_debug_stall_next_attention.argtypes = []
     lib.atlas_release_caches.restype = ctypes.c_int
     lib.atlas_release_caches.argtypes = []
     lib.atlas_version.restype = ctypes.c_int32
@@ -205,6 +207,12 @@ def last_device_error(stream=None) -> int:
     if st not in (OK, ERR_TIMEOUT):
         raise AtlasError(st, "atlas_last_device_error")
     return int(code.value)
+
+
+def debug_stall_next_attention():
+    """Test hook: the next bf16 attention launch leaves one K tile unloaded,
+    so its bounded waits expire and it reports ATLAS_ERR_TIMEOUT."""
+    _check(lib().atlas_debug_stall_next_attention(), "atlas_debug_stall_next_attention")
 
 
 def release_caches():

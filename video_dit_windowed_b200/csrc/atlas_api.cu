@@ -3,6 +3,7 @@
 // Every entry point checks its arguments on the host and returns a status
 // without launching anything when they are bad. See include/atlas.h for the
 // contract of each call and the passages it implements.
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -25,6 +26,12 @@ uint32_t *device_error_word() {
     }
     return addr[dev];
 }
+
+namespace {
+std::atomic<int> g_stall_request{0};
+}  // namespace
+
+bool take_stall_request() { return g_stall_request.exchange(0) != 0; }
 
 bool current_device(DeviceInfo *out) {
     static std::mutex mu;
@@ -233,5 +240,10 @@ ATLAS_API atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *
 }
 
 ATLAS_API atlas_status atlas_release_caches(void) { return release_rope_tables(); }
+
+ATLAS_API atlas_status atlas_debug_stall_next_attention(void) {
+    g_stall_request.store(1);
+    return ATLAS_OK;
+}
 
 ATLAS_API int32_t atlas_version(void) { return 100; }

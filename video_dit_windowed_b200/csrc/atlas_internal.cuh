@@ -87,6 +87,9 @@ struct AttnArgs {
     float *lse;
 };
 atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
+// One-shot request (atlas_debug_stall_next_attention): true once, for the
+// next bf16 attention launch, which then leaves one K tile unloaded.
+bool take_stall_request();
 atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream);
 
 }  // namespace atlas

@@ -90,6 +90,7 @@ struct Params {
     int32_t N, L, G, heads;
     float scale_log2;
     int32_t n_dunits, n_gunits, units_per_head, n_units, n_gtiles;
+    int32_t stall_unit;   // test hook: this unit's first K tile is never loaded (-1: off)
 };
 
 struct Unit {
@@ -196,6 +197,13 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
             const bool win = j < U.n_wtiles;
             const int32_t row = key_row(U, j);
+            if (j == 0 && u == p.stall_unit) {
+                // Failure-path test: leave this slot unarmed so the MMA
+                // issuer's bounded wait on it expires.
+                ++it;
+                ok = load(win ? &p.tm_vd : &p.tm_vg, U.head, row);
+                continue;
+            }
             ok = load(win ? &p.tm_kd : &p.tm_kg, U.head, row) &&
                  load(win ? &p.tm_vd : &p.tm_vg, U.head, row);
         }
@@ -627,6 +635,7 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.units_per_head = p.n_dunits + p.n_gunits;
     p.n_units = p.units_per_head * a.heads;
     p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
+    p.stall_unit = take_stall_request() ? 0 : -1;
     if (p.n_units == 0) return ATLAS_OK;
     const size_t smem = sizeof(Smem<HD>) + 1024;
     static std::once_flag attr_once;
