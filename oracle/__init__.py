@@ -51,6 +51,8 @@ def build(source: str = SOURCE, out: str = LIB_PATH, extra_flags=()) -> str:
 def _declare(lib):
     lib.atlas_oracle_cube_position.restype = _i64
     lib.atlas_oracle_cube_position.argtypes = [_i64] * 7
+    lib.atlas_oracle_cube_windows.restype = _i64
+    lib.atlas_oracle_cube_windows.argtypes = [_i64] * 6 + [_ptr]
     lib.atlas_oracle_cube_positions.restype = None
     lib.atlas_oracle_cube_positions.argtypes = [_i64] * 6 + [_ptr]
     for name in ("atlas_oracle_cube_reorder", "atlas_oracle_cube_unorder"):
@@ -60,6 +62,10 @@ def _declare(lib):
     lib.atlas_oracle_rope3d_rows.restype = None
     lib.atlas_oracle_rope3d_rows.argtypes = (
         [_ptr, _ptr, _i64, _ptr] + [_i64] * 5 + [_f64] + [_i64] * 3 + [_f64] * 3)
+    lib.atlas_oracle_attention_head_windows.restype = ctypes.c_int
+    lib.atlas_oracle_attention_head_windows.argtypes = (
+        [_i64, _i64, _ptr, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
+         _i64, _ptr, _ptr, _ptr, _ptr, ctypes.c_int])
     lib.atlas_oracle_attention_head.restype = ctypes.c_int
     lib.atlas_oracle_attention_head.argtypes = (
         [_i64, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
@@ -98,6 +104,17 @@ class Oracle:
         pos = np.empty(n, dtype=np.int64)
         self.lib.atlas_oracle_cube_positions(T, H, W, *cube, pos.ctypes.data)
         return pos
+
+    def cube_windows(self, grid, cube) -> np.ndarray:
+        """offsets[c] = first cube-order position of cube c; the last entry
+        is T*H*W (partial cubes at the far edges included)."""
+        T, H, W = grid
+        ct, ch, cw = cube
+        n = -(-T // ct) * -(-H // ch) * -(-W // cw)
+        off = np.empty(n + 1, dtype=np.int64)
+        got = self.lib.atlas_oracle_cube_windows(T, H, W, ct, ch, cw, off.ctypes.data)
+        assert got == n
+        return off
 
     def cube_position(self, grid, cube, r: int) -> int:
         return int(self.lib.atlas_oracle_cube_position(*grid, *cube, int(r)))
@@ -147,12 +164,14 @@ class Oracle:
     # -- attention ------------------------------------------------------
     def attention_head(self, n_detail: int, window_len: int, n_global: int,
                        scale: float, k_d, v_d, kd_lo: int, k_g, v_g, q_ids,
-                       q, n_threads: int = 1):
+                       q, n_threads: int = 1, win_off=None):
         """Asymmetric global-local attention for one head.
 
         ``k_d``/``v_d``: detail rows ``kd_lo .. kd_lo+len-1`` [rows, D];
         ``k_g``/``v_g``: all global rows [G, D]; ``q_ids``: query ids in
-        [0, N+G) (>= N means global row id-N); ``q``: [n_q, D].
+        [0, N+G) (>= N means global row id-N); ``q``: [n_q, D]. Windows are
+        ``window_len`` consecutive detail positions, or the ranges of
+        ``win_off`` (n_win+1 offsets) when given.
         Returns (o [n_q, D] float64, lse [n_q] float64, natural log).
         """
         f = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float64))
@@ -168,8 +187,13 @@ class Oracle:
         assert ids.shape == (n_q,)
         o = np.empty((n_q, D), dtype=np.float64)
         lse = np.empty(n_q, dtype=np.float64)
-        st = self.lib.atlas_oracle_attention_head(
-            n_detail, window_len, n_global, D, float(scale),
+        if win_off is not None:
+            off = np.ascontiguousarray(np.asarray(win_off, dtype=np.int64))
+            off_ptr, n_win = off.ctypes.data, off.size - 1
+        else:
+            off, off_ptr, n_win = None, None, 0
+        st = self.lib.atlas_oracle_attention_head_windows(
+            n_detail, window_len, off_ptr, n_win, n_global, D, float(scale),
             k_d.ctypes.data, v_d.ctypes.data, kd_lo, kd_lo + k_d.shape[0],
             k_g.ctypes.data, v_g.ctypes.data, n_q, ids.ctypes.data,
             q.ctypes.data, o.ctypes.data, lse.ctypes.data, int(n_threads))
@@ -180,7 +204,7 @@ class Oracle:
         return o, lse
 
     def attention_full(self, q_d, k_d, v_d, window_len, q_g, k_g, v_g,
-                       scale, n_threads: int = 1):
+                       scale, n_threads: int = 1, win_off=None):
         """All rows, all heads. Detail tensors [N, heads, D] in cube order,
         global [G, heads, D]. Returns (o_d, o_g, lse [heads, N+G])."""
         q_d = np.asarray(q_d, dtype=np.float64)
@@ -196,7 +220,7 @@ class Oracle:
             o, l = self.attention_head(
                 N, window_len, G, scale, np.asarray(k_d)[:, h, :],
                 np.asarray(v_d)[:, h, :], 0, np.asarray(k_g)[:, h, :],
-                np.asarray(v_g)[:, h, :], ids, q_all, n_threads)
+                np.asarray(v_g)[:, h, :], ids, q_all, n_threads, win_off)
             o_d[:, h, :] = o[:N]
             o_g[:, h, :] = o[N:]
             lse[h] = l

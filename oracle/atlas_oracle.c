@@ -29,7 +29,9 @@
  *   - tokens are stored in raster order r = (t*H + h)*W + w, one row of
  *     heads*head_dim values per token;
  *   - cubes are numbered in raster order over the cube grid, and the tokens
- *     of one cube in raster order over the cube's own extent;
+ *     of one cube in raster order over the cube's own extent; where the cube
+ *     size does not divide an axis, the last cube along it is partial (keeps
+ *     only the tokens that exist), so windows have variable length;
  *   - RoPE splits head_dim into contiguous [t | h | w] segments and rotates
  *     interleaved channel pairs (2k, 2k+1) of a segment of width d by the
  *     angle p * theta^(-2k/d), p = index * scale for that axis;
@@ -51,21 +53,56 @@
 /* Cube reorder ([TS] Methodologie 1, Fase 2; [AB] "reordered windows")     */
 /* ------------------------------------------------------------------------ */
 
+/* Cubes along an axis of extent E cut into cubes of c tokens: ceil(E/c)
+ * cubes, all of c tokens except the last, which keeps what is left. */
+static int64_t cube_extent(int64_t E, int64_t c, int64_t b)
+{
+    return (b + 1) * c <= E ? c : E - b * c;
+}
+
 /* Position j, in the cube-contiguous sequence, of the token at raster index
- * r of a T x H x W grid cut into ct x ch x cw cubes. Each cube's
- * L = ct*ch*cw tokens occupy positions cube*L .. cube*L + L - 1. */
+ * r of a T x H x W grid cut into ct x ch x cw cubes. Cubes are taken in
+ * raster order over the cube grid; a cube at the far edge of an axis the
+ * cube size does not divide keeps only the tokens that exist (a partial
+ * cube). Each cube's tokens are contiguous, in raster order over the cube's
+ * own extent. The tokens before cube (bt, bh, bw) are: every whole slab of
+ * bt*ct frames, then bh rows of cubes of that slab (bh*ch rows of the grid,
+ * et frames deep), then bw cubes of that row (bw*cw columns, et x eh deep).
+ * When the cube divides the grid this is cube*L + local with L = ct*ch*cw. */
 int64_t atlas_oracle_cube_position(int64_t T, int64_t H, int64_t W,
                                    int64_t ct, int64_t ch, int64_t cw,
                                    int64_t r)
 {
-    (void)T;
     int64_t t = r / (H * W);
     int64_t h = (r / W) % H;
     int64_t w = r % W;
-    int64_t cubes_h = H / ch, cubes_w = W / cw;
-    int64_t cube = ((t / ct) * cubes_h + (h / ch)) * cubes_w + (w / cw);
-    int64_t local = ((t % ct) * ch + (h % ch)) * cw + (w % cw);
-    return cube * (ct * ch * cw) + local;
+    int64_t bt = t / ct, bh = h / ch, bw = w / cw;
+    int64_t et = cube_extent(T, ct, bt);
+    int64_t eh = cube_extent(H, ch, bh);
+    int64_t ew = cube_extent(W, cw, bw);
+    int64_t before = bt * ct * H * W + et * (bh * ch) * W + et * eh * (bw * cw);
+    int64_t local = ((t - bt * ct) * eh + (h - bh * ch)) * ew + (w - bw * cw);
+    return before + local;
+}
+
+/* Window (cube) boundaries of the cube-contiguous sequence: offsets[c] is
+ * the first position of cube c (raster order over the cube grid) and
+ * offsets[n_cubes] = T*H*W. Returns n_cubes; offsets must hold n_cubes+1. */
+int64_t atlas_oracle_cube_windows(int64_t T, int64_t H, int64_t W,
+                                  int64_t ct, int64_t ch, int64_t cw,
+                                  int64_t *offsets)
+{
+    int64_t nt = (T + ct - 1) / ct, nh = (H + ch - 1) / ch, nw = (W + cw - 1) / cw;
+    int64_t n = 0, pos = 0;
+    for (int64_t bt = 0; bt < nt; ++bt)
+        for (int64_t bh = 0; bh < nh; ++bh)
+            for (int64_t bw = 0; bw < nw; ++bw) {
+                offsets[n++] = pos;
+                pos += cube_extent(T, ct, bt) * cube_extent(H, ch, bh) *
+                       cube_extent(W, cw, bw);
+            }
+    offsets[n] = pos;
+    return n;
 }
 
 /* Fill pos[r] = cube position of raster token r, for every r < T*H*W. */
@@ -162,16 +199,34 @@ void atlas_oracle_rope3d_rows(const double *x, double *y, int64_t n_rows,
  * A detail query sees the keys of its own cube (window of L consecutive
  * positions) and every global key; a global query sees every global key and
  * no detail key (mask value -inf). */
-static int allowed(int64_t q, int64_t k, int64_t N, int64_t L)
+/* The window holding detail position x: x / L for windows of L positions,
+ * else the last c with win_off[c] <= x (win_off: n_win+1 increasing
+ * offsets, win_off[0] = 0, win_off[n_win] = N). */
+static int64_t window_of(int64_t x, int64_t L, const int64_t *win_off, int64_t n_win)
+{
+    if (win_off == NULL) return x / L;
+    int64_t lo = 0, hi = n_win - 1;
+    while (lo < hi) {
+        int64_t mid = (lo + hi + 1) / 2;
+        if (win_off[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+static int allowed(int64_t q, int64_t k, int64_t N, int64_t L,
+                   const int64_t *win_off, int64_t n_win)
 {
     int q_detail = q < N, k_detail = k < N;
-    if (q_detail && k_detail) return (q / L) == (k / L);
+    if (q_detail && k_detail)
+        return window_of(q, L, win_off, n_win) == window_of(k, L, win_off, n_win);
     if (q_detail && !k_detail) return 1;
     if (!q_detail && k_detail) return 0;
     return 1;
 }
 
-/* One head. For each of the n_q queries (ids q_ids[i], vectors q[i]),
+/* One head. Windows: window_len consecutive detail positions, or, when
+ * win_off is not NULL, the n_win ranges [win_off[c], win_off[c+1]).
+ * For each of the n_q queries (ids q_ids[i], vectors q[i]),
  * evaluate allowed() against all N+G keys, take logits scale*<q,k> on the
  * allowed ones, then a two-pass softmax (max, then sum of exp) and the
  * weighted sum of V. Outputs o[i] (head_dim values) and lse[i] (natural
@@ -181,15 +236,16 @@ static int allowed(int64_t q, int64_t k, int64_t N, int64_t L)
  * k_g/v_g hold all G global rows. If an allowed detail key falls outside
  * the rows supplied the function returns 1 (caller error); 2 on allocation
  * failure; 0 on success. */
-int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
-                                int64_t n_global, int64_t head_dim,
-                                double scale,
-                                const double *k_d, const double *v_d,
-                                int64_t kd_lo, int64_t kd_hi,
-                                const double *k_g, const double *v_g,
-                                int64_t n_q, const int64_t *q_ids,
-                                const double *q, double *o, double *lse,
-                                int n_threads)
+int atlas_oracle_attention_head_windows(int64_t n_detail, int64_t window_len,
+                                        const int64_t *win_off, int64_t n_win,
+                                        int64_t n_global, int64_t head_dim,
+                                        double scale,
+                                        const double *k_d, const double *v_d,
+                                        int64_t kd_lo, int64_t kd_hi,
+                                        const double *k_g, const double *v_g,
+                                        int64_t n_q, const int64_t *q_ids,
+                                        const double *q, double *o, double *lse,
+                                        int n_threads)
 {
     int64_t N = n_detail, G = n_global, D = head_dim;
     int status = 0;
@@ -210,7 +266,7 @@ int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
         int64_t n_allowed = 0;
         int bad = 0;
         for (int64_t kid = 0; kid < N + G; ++kid) {
-            if (!allowed(qid, kid, N, window_len)) continue;
+            if (!allowed(qid, kid, N, window_len, win_off, n_win)) continue;
             const double *kr, *vr;
             if (kid < N) {
                 if (kid < kd_lo || kid >= kd_hi) { bad = 1; break; }
@@ -250,6 +306,23 @@ int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
         free(vrow);
     }
     return status;
+}
+
+/* Windows of window_len consecutive detail positions (the cube divides the
+ * grid). */
+int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
+                                int64_t n_global, int64_t head_dim,
+                                double scale,
+                                const double *k_d, const double *v_d,
+                                int64_t kd_lo, int64_t kd_hi,
+                                const double *k_g, const double *v_g,
+                                int64_t n_q, const int64_t *q_ids,
+                                const double *q, double *o, double *lse,
+                                int n_threads)
+{
+    return atlas_oracle_attention_head_windows(n_detail, window_len, NULL, 0, n_global,
+                                               head_dim, scale, k_d, v_d, kd_lo, kd_hi,
+                                               k_g, v_g, n_q, q_ids, q, o, lse, n_threads);
 }
 
 /* Number of threads an OpenMP parallel region of this library would use by

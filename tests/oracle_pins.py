@@ -118,7 +118,50 @@ def pin_cube_special_cases(o):
         assert np.array_equal(o.cube_positions(grid, grid), np.arange(n))
 
 
-CUBE_PINS = [pin_cube_matches_rearrange, pin_cube_bijection,
+# Grids the cube does not divide: the last cube along such an axis is partial.
+PARTIAL_CASES = [
+    ((5, 7, 9), (2, 3, 4)),
+    ((3, 5, 6), (2, 2, 4)),
+    ((4, 8, 10), (2, 4, 4)),
+    ((1, 3, 2), (3, 4, 5)),
+    ((4, 8, 8), (2, 4, 4)),
+]
+
+
+def lexsort_order(grid, cube):
+    """order[j] = raster index at cube position j, by sorting every token on
+    (cube t, cube h, cube w, t in cube, h in cube, w in cube)."""
+    T, H, W = grid
+    ct, ch, cw = cube
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    t, h, w = t.ravel(), h.ravel(), w.ravel()
+    return np.lexsort((w % cw, h % ch, t % ct, w // cw, h // ch, t // ct))
+
+
+def pin_cube_partial_matches_lexsort(o):
+    for grid, cube in PARTIAL_CASES + CUBE_CASES:
+        pos = o.cube_positions(grid, cube)
+        order = lexsort_order(grid, cube)
+        assert np.array_equal(pos[order], np.arange(pos.size)), (grid, cube)
+
+
+def pin_cube_windows_are_cubes(o):
+    """Window offsets bound exactly the tokens of one (possibly partial) cube."""
+    for grid, cube in PARTIAL_CASES + CUBE_CASES:
+        T, H, W = grid
+        ct, ch, cw = cube
+        off = o.cube_windows(grid, cube)
+        order = lexsort_order(grid, cube)
+        t, h, w = order // (H * W), (order // W) % H, order % W
+        key = ((t // ct) * -(-H // ch) + h // ch) * -(-W // cw) + w // cw
+        counts = np.bincount(key, minlength=off.size - 1)
+        assert np.array_equal(off, np.concatenate([[0], np.cumsum(counts)])), (grid, cube)
+        for c in range(off.size - 1):
+            assert np.all(key[off[c]:off[c + 1]] == c)
+
+
+CUBE_PINS = [pin_cube_matches_rearrange, pin_cube_bijection, pin_cube_partial_matches_lexsort,
+             pin_cube_windows_are_cubes,
              pin_cube_worked_example, pin_cube_locality,
              pin_cube_roundtrip_bytes, pin_cube_special_cases]
 
@@ -410,7 +453,45 @@ def pin_attention_rejects_missing_rows(o):
     assert np.array_equal(out, np.ones((1, D)))
 
 
-ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_full_when_one_cube,
+def pin_attention_partial_cubes_dense_sdpa(o):
+    """Variable windows (partial cubes): equal to dense masked attention
+    whose mask comes from token coordinates (same cube <=> same floor
+    division), with detail tokens in the lexsort cube order."""
+    for ci, (grid, cube) in enumerate(PARTIAL_CASES[:3]):
+        T, H, W = grid
+        ct, ch, cw = cube
+        G, heads, D = 6, 2, 16
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 300 + ci)
+        order = lexsort_order(grid, cube)
+        t, h, w = order // (H * W), (order // W) % H, order % W
+        key = np.stack([t // ct, h // ch, w // cw], -1)
+        same = np.all(key[:, None, :] == key[None, :, :], -1)
+        mask = np.zeros((N + G, N + G), dtype=bool)
+        mask[:N, :N] = same
+        mask[:N, N:] = True
+        mask[N:, N:] = True
+        off = o.cube_windows(grid, cube)
+        od, og, lse = o.attention_full(qd, kd, vd, 1, qg, kg, vg, 0.25, win_off=off)
+        q = torch.from_numpy(np.concatenate([qd, qg])).permute(1, 0, 2)
+        k = torch.from_numpy(np.concatenate([kd, kg])).permute(1, 0, 2)
+        v = torch.from_numpy(np.concatenate([vd, vg])).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k, v, attn_mask=torch.from_numpy(mask), scale=0.25).permute(1, 0, 2).numpy()
+        assert np.max(np.abs(ref - np.concatenate([od, og]))) < 1e-12, (grid, cube)
+
+
+def pin_attention_offsets_equal_fixed_windows(o):
+    """Offsets k*L give exactly the fixed-length-window result."""
+    grid, cube, G, heads, D = (4, 8, 8), (2, 4, 4), 9, 2, 16
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 17)
+    a = o.attention_full(qd, kd, vd, 32, qg, kg, vg, 0.3)
+    b = o.attention_full(qd, kd, vd, 1, qg, kg, vg, 0.3, win_off=np.arange(0, N + 1, 32))
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
+             pin_attention_offsets_equal_fixed_windows, pin_attention_full_when_one_cube,
              pin_attention_single_token_windows, pin_attention_zero_keys_mean,
              pin_attention_rows_sum_to_one, pin_attention_global_ignores_detail,
              pin_attention_probe_mass, pin_attention_rejects_missing_rows]

@@ -10,7 +10,10 @@ import oracle_pins
 
 # (name, text in atlas_oracle.c, replacement)
 MUTANTS = [
-    ("window_off_by_one", "return (q / L) == (k / L);", "return (q / L) == ((k + 1) / L);"),
+    ("window_off_by_one", "if (win_off == NULL) return x / L;", "if (win_off == NULL) return (x + 1) / L;"),
+    ("varlen_window_search", "if (win_off[mid] <= x) lo = mid; else hi = mid - 1;",
+     "if (win_off[mid] < x) lo = mid; else hi = mid - 1;"),
+    ("partial_cube_extent", "return (b + 1) * c <= E ? c : E - b * c;", "return c;"),
     ("global_sees_detail", "if (!q_detail && k_detail) return 0;", "if (!q_detail && k_detail) return 1;"),
     ("detail_misses_global", "if (q_detail && !k_detail) return 1;", "if (q_detail && !k_detail) return 0;"),
     ("rope_sign", "y[off + 2 * k] = x0 * c - x1 * s;", "y[off + 2 * k] = x0 * c + x1 * s;"),
@@ -18,10 +21,10 @@ MUTANTS = [
     ("rope_wrong_axis", "rope_segment(xr, yr, d_t + d_h, d_w, p_w, theta);", "rope_segment(xr, yr, d_t + d_h, d_w, p_h, theta);"),
     ("rope_scale_mixup", "double p_h = (double)((r / W) % H) * s_h;", "double p_h = (double)((r / W) % H) * s_w;"),
     ("rope_pair_layout", "double x0 = x[off + 2 * k], x1 = x[off + 2 * k + 1];", "double x0 = x[off + k], x1 = x[off + k + d / 2];"),
-    ("cube_local_transposed", "int64_t local = ((t % ct) * ch + (h % ch)) * cw + (w % cw);",
-     "int64_t local = ((h % ch) * ct + (t % ct)) * cw + (w % cw);"),
-    ("cube_order_transposed", "int64_t cube = ((t / ct) * cubes_h + (h / ch)) * cubes_w + (w / cw);",
-     "int64_t cube = ((w / cw) * cubes_h + (h / ch)) * (T / ct) + (t / ct);"),
+    ("cube_local_transposed", "int64_t local = ((t - bt * ct) * eh + (h - bh * ch)) * ew + (w - bw * cw);",
+     "int64_t local = ((h - bh * ch) * et + (t - bt * ct)) * ew + (w - bw * cw);"),
+    ("cube_order_transposed", "int64_t before = bt * ct * H * W + et * (bh * ch) * W + et * eh * (bw * cw);",
+     "int64_t before = bw * cw * H * T + ew * (bh * ch) * T + ew * eh * (bt * ct);"),
     ("dropped_scale", "logit[n_allowed] = scale * dot;", "logit[n_allowed] = dot;"),
     ("lse_missing_max", "lse[i] = m + log(sum);", "lse[i] = log(sum);"),
     ("unorder_not_inverse", "memcpy(dst + r * row_bytes, src + j * row_bytes, (size_t)row_bytes);",
