@@ -84,13 +84,15 @@ typedef struct {
  * ratios), at the token's grid position.
  *
  * src: [T*H*W, heads, head_dim] in raster order. dst: same size, cube order:
- * cubes in raster order over the (T/ct) x (H/ch) x (W/cw) cube grid, the
- * L = ct*ch*cw tokens of a cube in raster order over the cube, position
- * j = cube*L + local. Without rope the copy is bit-exact. With rope the
+ * cubes in raster order over the ceil(T/ct) x ceil(H/ch) x ceil(W/cw) cube
+ * grid, the tokens of a cube in raster order over the cube, contiguous. When
+ * the cube divides the grid, position j = cube*L + local with L = ct*ch*cw.
+ * Otherwise the last cube along such an axis is partial (it keeps only the
+ * tokens that exist) and windows have variable length: see
+ * atlas_cube_window_offsets. Without rope the copy is bit-exact. With rope the
  * rotation runs in fp32 on fp64-built, fp32-rounded cos/sin and rounds once
  * to dtype (round to nearest even).
- * Errors: NULL pointers; a cube extent that does not divide the grid or is
- * < 1 (SHAPE); head_dim not even or the RoPE split not summing to head_dim
+ * Errors: NULL pointers; a cube extent < 1 (SHAPE); head_dim not even or the RoPE split not summing to head_dim
  * or odd (UNSUPPORTED); rows not a multiple of 16 bytes, or misaligned
  * pointers (ALIGN); src and dst overlapping (ALIAS).
  */
@@ -200,6 +202,43 @@ atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, atlas_grid3 
                                         int32_t head_dim, atlas_dtype dtype,
                                         const atlas_rope *rope,
                                         atlas_stream_t stream);
+
+/*
+ * atlas_cube_window_offsets -- window boundaries of the cube order (host).
+ *
+ * Passage: as atlas_cube_reorder. Cube c (raster order over the cube grid)
+ * occupies cube-order positions [offsets[c], offsets[c+1]); offsets[n] =
+ * T*H*W. Partial cubes at the far edges are shorter windows.
+ * offsets: host array of `capacity` int32, or NULL to only query the count.
+ * *n_windows receives the number of cubes. Errors: NULL n_windows (NULL),
+ * a non-positive extent or more than 2^31-1 tokens (SHAPE), capacity <
+ * n_windows+1 (CAPACITY). Host only: no device work, no allocation.
+ */
+atlas_status atlas_cube_window_offsets(atlas_grid3 grid, atlas_cube3 cube,
+                                       int32_t *offsets, int64_t capacity,
+                                       int64_t *n_windows);
+
+/*
+ * atlas_local_global_attn_windows -- steps (3) and (4) with windows of
+ * variable length (for example the partial cubes of a grid the cube does
+ * not divide).
+ *
+ * Passages: as atlas_local_global_attn. Detail row q sees the detail keys of
+ * the window w with window_offsets[w] <= q < window_offsets[w+1], and every
+ * global key. window_offsets: DEVICE array of n_windows+1 int32, increasing,
+ * window_offsets[0] = 0 and window_offsets[n_windows] = n_detail (the
+ * library does not read it on the host; other contents give undefined rows
+ * but no out-of-bounds access). Everything else as atlas_local_global_attn.
+ * Errors: NULL window_offsets with n_detail > 0 (NULL), n_windows < 1 or >
+ * n_detail (SHAPE), offsets not 4-byte aligned (ALIGN), as
+ * atlas_local_global_attn otherwise.
+ */
+atlas_status atlas_local_global_attn_windows(
+    const void *q_d, const void *k_d, const void *v_d, int64_t n_detail,
+    const int32_t *window_offsets, int64_t n_windows, const void *q_g,
+    const void *k_g, const void *v_g, int64_t n_global, int32_t heads,
+    int32_t head_dim, float softmax_scale, atlas_dtype dtype, void *o_d,
+    void *o_g, float *lse, atlas_stream_t stream);
 
 /* Human-readable name of a status. Never NULL. */
 const char *atlas_status_string(atlas_status status);

@@ -69,7 +69,6 @@ def test_reorder_validation(lib):
     big = FAKE + (1 << 30)
     assert reorder(lib, None, big) == atlas.ERR_NULL
     assert reorder(lib, FAKE, None) == atlas.ERR_NULL
-    assert reorder(lib, FAKE, big, cube=atlas.Cube3(3, 4, 4)) == atlas.ERR_SHAPE
     assert reorder(lib, FAKE, big, cube=atlas.Cube3(0, 4, 4)) == atlas.ERR_SHAPE
     assert reorder(lib, FAKE, big, grid=atlas.Grid3(0, 8, 8)) == atlas.ERR_SHAPE
     assert reorder(lib, FAKE + 8, big) == atlas.ERR_ALIGN
@@ -90,7 +89,7 @@ def test_reorder_validation(lib):
 def test_unorder_and_rope_validation(lib):
     big = FAKE + (1 << 30)
     assert lib.atlas_cube_unorder(None, big, G, C, 2, 64, atlas.FP32, None) == atlas.ERR_NULL
-    assert lib.atlas_cube_unorder(FAKE, big, G, atlas.Cube3(2, 3, 4), 2, 64, atlas.FP32,
+    assert lib.atlas_cube_unorder(FAKE, big, G, atlas.Cube3(2, 0, 4), 2, 64, atlas.FP32,
                                   None) == atlas.ERR_SHAPE
     assert lib.atlas_cube_unorder(FAKE, FAKE + 16, G, C, 2, 64, atlas.FP32,
                                   None) == atlas.ERR_ALIAS
@@ -134,3 +133,35 @@ def test_valid_call_without_gpu_reports_device(lib):
     assert attn(lib) == atlas.ERR_DEVICE
     big = FAKE + (1 << 30)
     assert reorder(lib, FAKE, big) == atlas.ERR_DEVICE
+
+
+def test_cube_window_offsets_host(lib):
+    import numpy as np
+    import oracle
+    orc = oracle.Oracle()
+    for grid, cube in (((5, 7, 9), (2, 3, 4)), ((4, 8, 8), (2, 4, 4)), ((21, 48, 80), (3, 16, 16))):
+        got = atlas.cube_window_offsets(grid, cube).numpy()
+        assert np.array_equal(got, orc.cube_windows(grid, cube))
+    n = ctypes.c_int64(0)
+    small = (ctypes.c_int32 * 3)()
+    assert lib.atlas_cube_window_offsets(atlas.Grid3(5, 7, 9), atlas.Cube3(2, 3, 4), small, 3,
+                                         ctypes.byref(n)) == atlas.ERR_CAPACITY
+    assert lib.atlas_cube_window_offsets(atlas.Grid3(5, 7, 9), atlas.Cube3(0, 3, 4), None, 0,
+                                         ctypes.byref(n)) == atlas.ERR_SHAPE
+    assert lib.atlas_cube_window_offsets(atlas.Grid3(5, 7, 9), atlas.Cube3(2, 3, 4), None, 0,
+                                         None) == atlas.ERR_NULL
+
+
+def test_windows_attention_validation(lib):
+    base = dict(q_d=FAKE, k_d=FAKE + (1 << 28), v_d=FAKE + (2 << 28), q_g=FAKE + (3 << 28),
+                k_g=FAKE + (4 << 28), v_g=FAKE + (5 << 28), o_d=FAKE + (6 << 28),
+                o_g=FAKE + (7 << 28))
+    def call(off=FAKE + (8 << 28), n_win=8, n_d=256, **kw):
+        a = dict(base, **kw)
+        return lib.atlas_local_global_attn_windows(a["q_d"], a["k_d"], a["v_d"], n_d, off, n_win,
+                                                   a["q_g"], a["k_g"], a["v_g"], 32, 2, 64, 0.0,
+                                                   atlas.BF16, a["o_d"], a["o_g"], None, None)
+    assert call(off=None) == atlas.ERR_NULL
+    assert call(n_win=0) == atlas.ERR_SHAPE
+    assert call(n_win=300) == atlas.ERR_SHAPE
+    assert call(off=FAKE + (8 << 28) + 2) == atlas.ERR_ALIGN

@@ -1,0 +1,146 @@
+"""GPU parity for grids the cube does not divide (partial cubes, variable
+windows) against the fp64 oracle, through the C-ABI.
+
+Reading of "Technische Samenvatting: AtlasVid", Methodologie 1 Fase 2 (the
+tokens of one cube are made contiguous) where the pages are silent: the last
+cube along an axis the cube size does not divide is partial, stays
+contiguous, and is its own, shorter window.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import (assert_attn_close, assert_rope_close, check_no_device_error, f64, n_threads,
+                     orc)
+from video_dit_windowed_b200 import atlas
+from video_dit_windowed_b200.workloads import normal
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+# grid, cube, heads, head_dim, dtype
+CASES = [
+    ((5, 7, 9), (2, 3, 4), 2, 64, "fp32"),
+    ((5, 7, 9), (2, 3, 4), 3, 128, "bf16"),
+    ((4, 8, 10), (2, 4, 4), 2, 64, "bf16"),
+    ((3, 17, 23), (3, 16, 16), 2, 128, "bf16"),
+    ((1, 3, 2), (3, 4, 5), 1, 64, "bf16"),
+]
+
+
+def tdt(name):
+    return torch.bfloat16 if name == "bf16" else torch.float32
+
+
+def split_for(hd):
+    return (16, 24, 24) if hd == 64 else (44, 42, 42)
+
+
+@pytest.mark.parametrize("grid,cube,heads,hd,dtype", CASES)
+def test_partial_reorder_unorder_bit_exact(grid, cube, heads, hd, dtype):
+    n = grid[0] * grid[1] * grid[2]
+    x = normal((n, heads, hd), "v_d", tdt(dtype), device=DEV)
+    y, z, y2 = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    atlas.cube_reorder(x, y, grid, cube)
+    atlas.cube_unorder(y, z, grid, cube)
+    atlas.cube_reorder_noalloc(x, y2, grid, cube)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    expect = orc().cube_reorder(x.cpu().view(torch.uint8).numpy().reshape(n, -1), grid, cube)
+    assert y.cpu().view(torch.uint8).numpy().reshape(n, -1).tobytes() == expect.tobytes()
+    assert torch.equal(z.view(torch.uint8), x.view(torch.uint8))
+    assert torch.equal(y2.view(torch.uint8), y.view(torch.uint8))
+
+
+@pytest.mark.parametrize("grid,cube,heads,hd,dtype", CASES)
+def test_partial_reorder_rope(grid, cube, heads, hd, dtype):
+    n = grid[0] * grid[1] * grid[2]
+    split, scales = split_for(hd), (2.0, 1.0, 1.0)
+    x = normal((n, heads, hd), "q_d", tdt(dtype), device=DEV)
+    y = torch.empty_like(x)
+    atlas.cube_reorder(x, y, grid, cube, atlas.make_rope(10000.0, split, scales))
+    torch.cuda.synchronize()
+    xd = f64(x)
+    exact = orc().cube_reorder(orc().rope3d_grid(xd, grid, 10000.0, split, scales), grid, cube)
+    assert_rope_close(f64(y), exact, orc().cube_reorder(xd, grid, cube), dtype)
+
+
+@pytest.mark.parametrize("grid,cube,heads,hd,dtype", CASES)
+def test_partial_cube_chain(grid, cube, heads, hd, dtype):
+    """raster -> reorder(+RoPE) -> variable-window attention -> unorder,
+    against the oracle's chain in raster order."""
+    n = grid[0] * grid[1] * grid[2]
+    G, split = 37, split_for(hd)
+    rd = atlas.make_rope(10000.0, split, (1.0, 1.0, 1.0))
+    mk = lambda rows, s: normal((rows, heads, hd), s, tdt(dtype), seed=1, device=DEV)
+    x_q, x_k, x_v = mk(n, "q_d"), mk(n, "k_d"), mk(n, "v_d")
+    q_g, k_g, v_g = mk(G, "q_g"), mk(G, "k_g"), mk(G, "v_g")
+    q_d, k_d, v_d = torch.empty_like(x_q), torch.empty_like(x_k), torch.empty_like(x_v)
+    atlas.cube_reorder(x_q, q_d, grid, cube, rd)
+    atlas.cube_reorder(x_k, k_d, grid, cube, rd)
+    atlas.cube_reorder(x_v, v_d, grid, cube)
+    off = atlas.cube_window_offsets(grid, cube).to(DEV)
+    o_d, o_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    lse = torch.empty(heads, n + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_windows(q_d, k_d, v_d, off, q_g, k_g, v_g, o_d, o_g, lse)
+    o_r = torch.empty_like(o_d)
+    atlas.cube_unorder(o_d, o_r, grid, cube)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    o = orc()
+    rq = o.cube_reorder(o.rope3d_grid(f64(x_q), grid, 10000.0, split, (1, 1, 1)), grid, cube)
+    rk = o.cube_reorder(o.rope3d_grid(f64(x_k), grid, 10000.0, split, (1, 1, 1)), grid, cube)
+    rv = o.cube_reorder(f64(x_v), grid, cube)
+    win = o.cube_windows(grid, cube)
+    ref_d, ref_g, ref_lse = o.attention_full(rq, rk, rv, 1, f64(q_g), f64(k_g), f64(v_g),
+                                             hd ** -0.5, n_threads(), win_off=win)
+    got = np.concatenate([f64(o_r), f64(o_g)])
+    ref = np.concatenate([o.cube_unorder(ref_d, grid, cube), ref_g])
+    assert_attn_close(got, ref, dtype, f"{grid} {cube}")
+    assert np.max(np.abs(f64(lse) - ref_lse)) <= (5e-3 if dtype == "bf16" else 1e-4)
+
+
+def test_offsets_of_fixed_windows_match_fixed_path():
+    """Offsets k*L select exactly the fixed-length path's result."""
+    N, L, G, heads, hd = 3072, 768, 300, 2, 128
+    mk = lambda rows, s: normal((rows, heads, hd), s, torch.bfloat16, seed=2, device=DEV)
+    q_d, k_d, v_d, q_g, k_g, v_g = (mk(N, "q_d"), mk(N, "k_d"), mk(N, "v_d"), mk(G, "q_g"),
+                                    mk(G, "k_g"), mk(G, "v_g"))
+    a_d, a_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    b_d, b_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    atlas.local_global_attn(q_d, k_d, v_d, L, q_g, k_g, v_g, a_d, a_g)
+    off = torch.arange(0, N + 1, L, dtype=torch.int32, device=DEV)
+    atlas.local_global_attn_windows(q_d, k_d, v_d, off, q_g, k_g, v_g, b_d, b_g)
+    torch.cuda.synchronize()
+    assert torch.equal(a_d.view(torch.int16), b_d.view(torch.int16))
+    assert torch.equal(a_g.view(torch.int16), b_g.view(torch.int16))
+
+
+def test_partial_cubes_at_scale_sampled():
+    """720p-like grid whose H the cube does not divide (partial cubes of 13
+    rows), 8 heads; sampled windows (a full one, a partial one, the last) on
+    the first and last head against the oracle."""
+    grid, cube, G, heads, hd = (21, 45, 80), (3, 16, 16), 5040, 8, 128
+    n = grid[0] * grid[1] * grid[2]
+    mk = lambda rows, s: normal((rows, heads, hd), s, torch.bfloat16, seed=3, device=DEV)
+    q_d, k_d, v_d = mk(n, "q_d"), mk(n, "k_d"), mk(n, "v_d")
+    q_g, k_g, v_g = mk(G, "q_g"), mk(G, "k_g"), mk(G, "v_g")
+    off_h = atlas.cube_window_offsets(grid, cube)
+    off = off_h.to(DEV)
+    o_d, o_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    atlas.local_global_attn_windows(q_d, k_d, v_d, off, q_g, k_g, v_g, o_d, o_g)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    offs = off_h.numpy().astype(np.int64)
+    sizes = np.diff(offs)
+    wins = [0, int(np.argmin(sizes)), len(sizes) - 1]
+    assert sizes[wins[1]] < 768
+    for head in (0, heads - 1):
+        kg, vg = f64(k_g[:, head]), f64(v_g[:, head])
+        for w in wins:
+            lo, hi = int(offs[w]), int(offs[w + 1])
+            rows = np.arange(lo, hi)
+            ref, _ = orc().attention_head(n, 1, G, hd ** -0.5, f64(k_d[lo:hi, head]),
+                                          f64(v_d[lo:hi, head]), lo, kg, vg, rows,
+                                          f64(q_d[lo:hi, head]), n_threads(), win_off=offs)
+            assert_attn_close(f64(o_d[lo:hi, head]), ref, "bf16", f"window {w} head {head}")

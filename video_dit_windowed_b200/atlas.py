@@ -74,6 +74,12 @@ def _declare(lib):
     lib.atlas_local_global_attn.argtypes = [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64,
                                             _i32, _i32, ctypes.c_float, ctypes.c_int, _vp, _vp,
                                             _vp, _vp]
+    lib.atlas_local_global_attn_windows.restype = ctypes.c_int
+    lib.atlas_local_global_attn_windows.argtypes = [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp,
+                                                    _i64, _i32, _i32, ctypes.c_float, ctypes.c_int,
+                                                    _vp, _vp, _vp, _vp]
+    lib.atlas_cube_window_offsets.restype = ctypes.c_int
+    lib.atlas_cube_window_offsets.argtypes = [Grid3, Cube3, _vp, _i64, ctypes.POINTER(_i64)]
     lib.atlas_status_string.restype = ctypes.c_char_p
     lib.atlas_status_string.argtypes = [ctypes.c_int]
     lib.atlas_last_device_error.restype = ctypes.c_int
@@ -194,6 +200,38 @@ def local_global_attn(q_d, k_d, v_d, window_len, q_g, k_g, v_g, o_d, o_g, lse=No
         nz(q_g, n_g), nz(k_g, n_g), nz(v_g, n_g), n_g, heads, hd, float(softmax_scale),
         _dtype_code(ref), nz(o_d, n_d), nz(o_g, n_g), _ptr(lse), _stream(ref, stream))
     _check(st, "atlas_local_global_attn")
+    return o_d, o_g, lse
+
+
+def cube_window_offsets(grid, cube):
+    """Window boundaries of the cube order as a host int32 tensor [n+1]
+    (partial cubes at the far edges included)."""
+    import torch
+    n = _i64(0)
+    _check(lib().atlas_cube_window_offsets(Grid3(*grid), Cube3(*cube), None, 0, ctypes.byref(n)),
+           "atlas_cube_window_offsets")
+    out = torch.empty(n.value + 1, dtype=torch.int32)
+    _check(lib().atlas_cube_window_offsets(Grid3(*grid), Cube3(*cube),
+                                           ctypes.c_void_p(out.data_ptr()), out.numel(),
+                                           ctypes.byref(n)), "atlas_cube_window_offsets")
+    return out
+
+
+def local_global_attn_windows(q_d, k_d, v_d, window_offsets, q_g, k_g, v_g, o_d, o_g,
+                              lse=None, softmax_scale: float = 0.0, stream=None):
+    """Like ``local_global_attn`` with variable-length windows given by the
+    device int32 tensor ``window_offsets`` [n_windows + 1]."""
+    ref = q_d if q_d is not None and q_d.shape[0] > 0 else q_g
+    heads, hd = ref.shape[1], ref.shape[2]
+    n_d = q_d.shape[0] if q_d is not None else 0
+    n_g = q_g.shape[0] if q_g is not None else 0
+    nz = lambda t, n: _ptr(t) if (t is not None and n > 0) else None
+    st = lib().atlas_local_global_attn_windows(
+        nz(q_d, n_d), nz(k_d, n_d), nz(v_d, n_d), n_d, nz(window_offsets, n_d),
+        window_offsets.numel() - 1 if window_offsets is not None else 0,
+        nz(q_g, n_g), nz(k_g, n_g), nz(v_g, n_g), n_g, heads, hd, float(softmax_scale),
+        _dtype_code(ref), nz(o_d, n_d), nz(o_g, n_g), _ptr(lse), _stream(ref, stream))
+    _check(st, "atlas_local_global_attn_windows")
     return o_d, o_g, lse
 
 

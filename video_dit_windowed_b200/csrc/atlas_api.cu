@@ -77,9 +77,10 @@ atlas_status check_grid(atlas_grid3 g, int32_t heads, int32_t head_dim, atlas_dt
     return ATLAS_OK;
 }
 
+// A cube that does not divide the grid leaves partial cubes at the far edges.
 atlas_status check_cube(atlas_grid3 g, atlas_cube3 c) {
+    (void)g;
     if (c.ct < 1 || c.ch < 1 || c.cw < 1) return ATLAS_ERR_SHAPE;
-    if (g.T % c.ct || g.H % c.ch || g.W % c.cw) return ATLAS_ERR_SHAPE;
     return ATLAS_OK;
 }
 
@@ -171,14 +172,26 @@ ATLAS_API atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid
     return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
-ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d, const void *v_d,
-                                               int64_t n_detail, int64_t window_len,
-                                               const void *q_g, const void *k_g, const void *v_g,
-                                               int64_t n_global, int32_t heads, int32_t head_dim,
-                                               float softmax_scale, atlas_dtype dtype, void *o_d,
-                                               void *o_g, float *lse, atlas_stream_t stream) {
+namespace atlas {
+namespace {
+
+// Shared validation and dispatch of the two attention entry points. With
+// win_off (device, n_win+1 int32) the windows are its ranges; otherwise
+// windows of window_len rows.
+atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d,
+                               int64_t n_detail, int64_t window_len, const int32_t *win_off,
+                               int64_t n_win, const void *q_g, const void *k_g, const void *v_g,
+                               int64_t n_global, int32_t heads, int32_t head_dim,
+                               float softmax_scale, atlas_dtype dtype, void *o_d, void *o_g,
+                               float *lse, atlas_stream_t stream) {
     if (n_detail < 0 || n_global < 0 || heads < 1) return ATLAS_ERR_SHAPE;
-    if (n_detail > 0 && (window_len < 1 || n_detail % window_len != 0)) return ATLAS_ERR_SHAPE;
+    if (win_off == nullptr) {
+        if (n_detail > 0 && (window_len < 1 || n_detail % window_len != 0)) return ATLAS_ERR_SHAPE;
+    } else {
+        if (n_win < 1 || n_win > n_detail) return ATLAS_ERR_SHAPE;
+        if (reinterpret_cast<uintptr_t>(win_off) & 3u) return ATLAS_ERR_ALIGN;
+        window_len = 1;
+    }
     if (n_detail + n_global > kMaxRows || static_cast<int64_t>(heads) > 65535)
         return ATLAS_ERR_SHAPE;
     if (n_detail > 0 && (!q_d || !k_d || !v_d || !o_d)) return ATLAS_ERR_NULL;
@@ -205,9 +218,62 @@ ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d,
     if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
     float scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(head_dim));
     AttnArgs a{q_d, k_d, v_d, n_detail, window_len, q_g, k_g, v_g, n_global,
-               heads, head_dim, scale, o_d, o_g, lse};
+               heads, head_dim, scale, o_d, o_g, lse, n_detail > 0 ? win_off : nullptr,
+               n_detail > 0 ? n_win : 0};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dtype == ATLAS_BF16 ? launch_attn_tc_bf16(a, s) : launch_attn_simt_f32(a, s);
+}
+
+}  // namespace
+}  // namespace atlas
+
+ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d, const void *v_d,
+                                               int64_t n_detail, int64_t window_len,
+                                               const void *q_g, const void *k_g, const void *v_g,
+                                               int64_t n_global, int32_t heads, int32_t head_dim,
+                                               float softmax_scale, atlas_dtype dtype, void *o_d,
+                                               void *o_g, float *lse, atlas_stream_t stream) {
+    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, window_len, nullptr, 0, q_g, k_g,
+                                    v_g, n_global, heads, head_dim, softmax_scale, dtype, o_d,
+                                    o_g, lse, stream);
+}
+
+ATLAS_API atlas_status atlas_local_global_attn_windows(
+    const void *q_d, const void *k_d, const void *v_d, int64_t n_detail,
+    const int32_t *window_offsets, int64_t n_windows, const void *q_g, const void *k_g,
+    const void *v_g, int64_t n_global, int32_t heads, int32_t head_dim, float softmax_scale,
+    atlas_dtype dtype, void *o_d, void *o_g, float *lse, atlas_stream_t stream) {
+    if (n_detail > 0 && window_offsets == nullptr) return ATLAS_ERR_NULL;
+    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, 1, n_detail > 0 ? window_offsets
+                                                                            : nullptr,
+                                    n_windows, q_g, k_g, v_g, n_global, heads, head_dim,
+                                    softmax_scale, dtype, o_d, o_g, lse, stream);
+}
+
+ATLAS_API atlas_status atlas_cube_window_offsets(atlas_grid3 grid, atlas_cube3 cube,
+                                                 int32_t *offsets, int64_t capacity,
+                                                 int64_t *n_windows) {
+    if (!n_windows) return ATLAS_ERR_NULL;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1)
+        return ATLAS_ERR_SHAPE;
+    if (grid.T * grid.H * grid.W > kMaxRows) return ATLAS_ERR_SHAPE;
+    auto n_along = [](int64_t e, int64_t c) { return (e + c - 1) / c; };
+    auto ext = [](int64_t e, int64_t c, int64_t b) { return (b + 1) * c <= e ? c : e - b * c; };
+    const int64_t nt = n_along(grid.T, cube.ct), nh = n_along(grid.H, cube.ch),
+                  nw = n_along(grid.W, cube.cw);
+    *n_windows = nt * nh * nw;
+    if (!offsets) return ATLAS_OK;  // size query
+    if (capacity < *n_windows + 1) return ATLAS_ERR_CAPACITY;
+    int64_t n = 0, pos = 0;
+    for (int64_t bt = 0; bt < nt; ++bt)
+        for (int64_t bh = 0; bh < nh; ++bh)
+            for (int64_t bw = 0; bw < nw; ++bw) {
+                offsets[n++] = static_cast<int32_t>(pos);
+                pos += ext(grid.T, cube.ct, bt) * ext(grid.H, cube.ch, bh) *
+                       ext(grid.W, cube.cw, bw);
+            }
+    offsets[n] = static_cast<int32_t>(pos);
+    return ATLAS_OK;
 }
 
 ATLAS_API const char *atlas_status_string(atlas_status status) {

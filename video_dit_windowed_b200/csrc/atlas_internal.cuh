@@ -85,6 +85,8 @@ struct AttnArgs {
     float scale;
     void *o_d, *o_g;
     float *lse;
+    const int32_t *win_off = nullptr;  // window offsets (device), NULL: windows of window_len
+    int64_t n_win = 0;
 };
 atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
 // One-shot request (atlas_debug_stall_next_attention): true once, for the

@@ -18,6 +18,8 @@ struct Params {
     int64_t N, L, G;
     int32_t heads;
     float scale;
+    const int32_t *win_off;  // window offsets (NULL: windows of L rows)
+    int64_t n_win;
 };
 
 template <int HD>
@@ -62,9 +64,21 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const Params p) 
     }
     float m = -__builtin_huge_valf(), l = 0.f;
     if (detail) {
-        const int64_t lo = (row / p.L) * p.L;
-        accumulate_keys<HD>(p.k_d + head * HD, p.v_d + head * HD, lo, lo + p.L, stride, q,
-                            p.scale, m, l, o);
+        int64_t lo, hi;
+        if (p.win_off == nullptr) {
+            lo = (row / p.L) * p.L;
+            hi = lo + p.L;
+        } else {  // last window whose start is <= row
+            int64_t a = 0, b = p.n_win - 1;
+            while (a < b) {
+                const int64_t mid = (a + b + 1) / 2;
+                if (p.win_off[mid] <= row) a = mid; else b = mid - 1;
+            }
+            lo = p.win_off[a];
+            hi = p.win_off[a + 1];
+        }
+        accumulate_keys<HD>(p.k_d + head * HD, p.v_d + head * HD, lo, hi, stride, q, p.scale,
+                            m, l, o);
     }
     if (p.G > 0)
         accumulate_keys<HD>(p.k_g + head * HD, p.v_g + head * HD, 0, p.G, stride, q, p.scale, m,
@@ -103,6 +117,8 @@ atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream) {
     p.G = a.n_global;
     p.heads = a.heads;
     p.scale = a.scale;
+    p.win_off = a.win_off;
+    p.n_win = a.n_win;
     if (a.head_dim == 64) return launch_hd<64>(p, stream);
     if (a.head_dim == 128) return launch_hd<128>(p, stream);
     return ATLAS_ERR_UNSUPPORTED;

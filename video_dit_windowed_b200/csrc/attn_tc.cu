@@ -91,7 +91,26 @@ struct Params {
     float scale_log2;
     int32_t n_dunits, n_gunits, units_per_head, n_units, n_gtiles;
     int32_t stall_unit;   // test hook: this unit's first K tile is never loaded (-1: off)
+    const int32_t *win_off;  // window offsets [n_win + 1] (NULL: windows of L rows)
+    int32_t n_win;
 };
+
+// The window holding detail row x, and its row range [start, end).
+__device__ __forceinline__ int32_t window_of(const Params &p, int32_t x) {
+    if (p.win_off == nullptr) return x / p.L;
+    int32_t lo = 0, hi = p.n_win - 1;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.win_off + mid) <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+__device__ __forceinline__ int32_t window_start(const Params &p, int32_t w) {
+    return p.win_off == nullptr ? w * p.L : __ldg(p.win_off + w);
+}
+__device__ __forceinline__ int32_t window_end(const Params &p, int32_t w) {
+    return p.win_off == nullptr ? min(p.N, (w + 1) * p.L) : __ldg(p.win_off + w + 1);
+}
 
 struct Unit {
     int32_t head, detail, q0, rows, kw0, n_wtiles, n_tiles;
@@ -105,9 +124,9 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
     if (U.detail) {
         U.q0 = lu * kUnitRows;
         U.rows = p.N;
-        int32_t q_last = min(U.q0 + kUnitRows, p.N) - 1;
-        U.kw0 = (U.q0 / p.L) * p.L;
-        int32_t kw1 = min(p.N, (q_last / p.L + 1) * p.L);
+        const int32_t q_last = min(U.q0 + kUnitRows, p.N) - 1;
+        U.kw0 = window_start(p, window_of(p, U.q0));
+        const int32_t kw1 = window_end(p, window_of(p, q_last));
         U.n_wtiles = (kw1 - U.kw0 + kBN - 1) / kBN;
     } else {
         U.q0 = (lu - p.n_dunits) * kUnitRows;
@@ -416,8 +435,9 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         const bool row_valid = q < U.rows;
         int32_t lo = 0, hi = p.N;
         if (U.detail) {
-            lo = (min(q, p.N - 1) / p.L) * p.L;
-            hi = min(lo + p.L, p.N);
+            const int32_t w = window_of(p, min(q, p.N - 1));
+            lo = window_start(p, w);
+            hi = window_end(p, w);
         }
         float m_run = kNegInf, l_run = 0.f;
         for (int32_t j = 0; j < U.n_tiles; ++j, ++cnt) {
@@ -636,6 +656,8 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.n_units = p.units_per_head * a.heads;
     p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
     p.stall_unit = take_stall_request() ? 0 : -1;
+    p.win_off = a.win_off;
+    p.n_win = static_cast<int32_t>(a.n_win);
     if (p.n_units == 0) return ATLAS_OK;
     const size_t smem = sizeof(Smem<HD>) + 1024;
     static std::once_flag attr_once;

@@ -15,6 +15,7 @@
 // done once per row per thread with multiply-shift division.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -37,6 +38,7 @@ struct FastDiv {
     uint32_t d = 1;
     FastDiv() = default;
     explicit FastDiv(uint32_t div) : d(div) {
+        if (div == 0) div = d = 1;  // never used for division by zero
         uint32_t l = 0;
         while ((1ull << l) < div) ++l;
         s = 31 + l;
@@ -48,7 +50,7 @@ struct FastDiv {
 };
 
 struct Geom {
-    uint32_t H, W, ct, ch, cw, cubes_h, cubes_w, L;
+    uint32_t T, H, W, ct, ch, cw, cubes_h, cubes_w, L;
     FastDiv by_W, by_H, by_ct, by_ch, by_cw, by_cubes_w, by_cubes_h, by_L;
 };
 
@@ -125,6 +127,47 @@ __device__ __forceinline__ void cube_coords(const Geom &g, uint32_t j, uint32_t 
     w = bw * g.cw + lw;
 }
 
+// Grids the cube does not divide: the last cube along such an axis is
+// partial (keeps the tokens that exist) and stays contiguous. Tokens before
+// cube (bt, bh, bw): the whole slabs of bt*ct frames, then bh cube rows of
+// its slab, then bw cubes of its row; inside a cube, raster order over the
+// cube's own extent. Plain 32-bit division: only this path needs it.
+__device__ __forceinline__ uint32_t extent(uint32_t E, uint32_t c, uint32_t b) {
+    return min(c, E - b * c);
+}
+
+__device__ __forceinline__ uint32_t cube_position_general(const Geom &g, uint32_t t,
+                                                          uint32_t h, uint32_t w) {
+    const uint32_t bt = t / g.ct, bh = h / g.ch, bw = w / g.cw;
+    const uint32_t et = extent(g.T, g.ct, bt), eh = extent(g.H, g.ch, bh),
+                   ew = extent(g.W, g.cw, bw);
+    const uint32_t before = bt * g.ct * g.H * g.W + et * (bh * g.ch) * g.W + et * eh * (bw * g.cw);
+    return before + ((t - bt * g.ct) * eh + (h - bh * g.ch)) * ew + (w - bw * g.cw);
+}
+
+__device__ __forceinline__ void cube_coords_general(const Geom &g, uint32_t j, uint32_t &t,
+                                                    uint32_t &h, uint32_t &w) {
+    const uint32_t slab = g.ct * g.H * g.W;
+    const uint32_t bt = j / slab;
+    uint32_t rem = j - bt * slab;
+    const uint32_t et = extent(g.T, g.ct, bt);
+    const uint32_t row = et * g.ch * g.W;
+    const uint32_t bh = rem / row;
+    rem -= bh * row;
+    const uint32_t eh = extent(g.H, g.ch, bh);
+    const uint32_t cube = et * eh * g.cw;
+    const uint32_t bw = rem / cube;
+    rem -= bw * cube;
+    const uint32_t ew = extent(g.W, g.cw, bw);
+    const uint32_t plane = eh * ew;
+    const uint32_t lt = rem / plane;
+    rem -= lt * plane;
+    const uint32_t lh = rem / ew;
+    t = bt * g.ct + lt;
+    h = bh * g.ch + lh;
+    w = bw * g.cw + (rem - lh * ew);
+}
+
 // Rotate the pairs of one 16-byte vector. bf16: 4 pairs, fp32: 2 pairs.
 template <int EB>
 __device__ __forceinline__ uint4 rotate(uint4 v, const float2 *cs);
@@ -161,7 +204,8 @@ __device__ __forceinline__ uint4 rotate<4>(uint4 v, const float2 *cs) {
 }
 
 // MODE 0: dst in cube order, src raster (reorder). MODE 1: dst raster, src
-// cube order (unorder). MODE 2: dst and src raster (RoPE only).
+// cube order (unorder). MODE 2: dst and src raster (RoPE only). MODE 3 / 4:
+// as 0 / 1 for grids the cube does not divide (partial cubes).
 template <int EB, bool ROPE, int MODE>
 __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) {
     constexpr int kPairs = 16 / EB / 2;  // RoPE pairs in one 16-byte vector
@@ -194,6 +238,12 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) 
         } else if (MODE == 1) {
             raster_coords(p.g, row, t, h, w);
             src_row = cube_position(p.g, t, h, w);
+        } else if (MODE == 3) {
+            cube_coords_general(p.g, row, t, h, w);
+            src_row = (t * p.g.H + h) * p.g.W + w;
+        } else if (MODE == 4) {
+            raster_coords(p.g, row, t, h, w);
+            src_row = cube_position_general(p.g, t, h, w);
         } else {
             raster_coords(p.g, row, t, h, w);
             src_row = row;
@@ -304,15 +354,18 @@ atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
 
+// mode: 0 reorder, 1 unorder, 2 raster RoPE; `general` selects the
+// partial-cube index arithmetic for reorder and unorder.
 template <int EB>
-atlas_status dispatch(const Params &p, bool rope, int mode, const DeviceInfo &dev,
+atlas_status dispatch(const Params &p, bool rope, int mode, bool general, const DeviceInfo &dev,
                       cudaStream_t stream) {
     if (rope) {
-        if (mode == 0) return launch<EB, true, 0>(p, dev, stream);
-        return launch<EB, true, 2>(p, dev, stream);
+        if (mode == 2) return launch<EB, true, 2>(p, dev, stream);
+        return general ? launch<EB, true, 3>(p, dev, stream) : launch<EB, true, 0>(p, dev, stream);
     }
-    if (mode == 0) return launch<EB, false, 0>(p, dev, stream);
-    return launch<EB, false, 1>(p, dev, stream);
+    if (mode == 0)
+        return general ? launch<EB, false, 3>(p, dev, stream) : launch<EB, false, 0>(p, dev, stream);
+    return general ? launch<EB, false, 4>(p, dev, stream) : launch<EB, false, 1>(p, dev, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -373,13 +426,16 @@ void fill_geometry(Params &p, const PermuteArgs &a) {
                                        a.elem_bytes / 16);
     p.vph = static_cast<uint32_t>(a.head_dim * a.elem_bytes / 16);
     Geom &g = p.g;
+    g.T = static_cast<uint32_t>(a.T);
     g.H = static_cast<uint32_t>(a.H);
     g.W = static_cast<uint32_t>(a.W);
     g.ct = static_cast<uint32_t>(a.ct);
     g.ch = static_cast<uint32_t>(a.ch);
     g.cw = static_cast<uint32_t>(a.cw);
-    g.cubes_h = g.H / g.ch;
-    g.cubes_w = g.W / g.cw;
+    // (cube counts of the divisible path; at least 1 so the dividers stay
+    // defined when a partial cube covers a whole axis)
+    g.cubes_h = std::max(1u, g.H / g.ch);
+    g.cubes_w = std::max(1u, g.W / g.cw);
     g.L = g.ct * g.ch * g.cw;
     g.by_W = FastDiv(g.W);
     g.by_H = FastDiv(g.H);
@@ -405,13 +461,16 @@ atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream) {
                                        a.elem_bytes / 16);
     p.vph = static_cast<uint32_t>(a.head_dim * a.elem_bytes / 16);
     Geom &g = p.g;
+    g.T = static_cast<uint32_t>(a.T);
     g.H = static_cast<uint32_t>(a.H);
     g.W = static_cast<uint32_t>(a.W);
     g.ct = static_cast<uint32_t>(a.ct);
     g.ch = static_cast<uint32_t>(a.ch);
     g.cw = static_cast<uint32_t>(a.cw);
-    g.cubes_h = g.H / g.ch;
-    g.cubes_w = g.W / g.cw;
+    // (cube counts of the divisible path; at least 1 so the dividers stay
+    // defined when a partial cube covers a whole axis)
+    g.cubes_h = std::max(1u, g.H / g.ch);
+    g.cubes_w = std::max(1u, g.W / g.cw);
     g.L = g.ct * g.ch * g.cw;
     g.by_W = FastDiv(g.W);
     g.by_H = FastDiv(g.H);
@@ -434,8 +493,9 @@ atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream) {
         p.tab_base[1] = static_cast<uint32_t>(a.T) * p.half[0];
         p.tab_base[2] = p.tab_base[1] + static_cast<uint32_t>(a.H) * p.half[1];
     }
-    if (a.elem_bytes == 2) return dispatch<2>(p, rope, a.mode, dev, stream);
-    return dispatch<4>(p, rope, a.mode, dev, stream);
+    const bool general = (a.T % a.ct) || (a.H % a.ch) || (a.W % a.cw);
+    if (a.elem_bytes == 2) return dispatch<2>(p, rope, a.mode, general, dev, stream);
+    return dispatch<4>(p, rope, a.mode, general, dev, stream);
 }
 
 atlas_status release_rope_tables() {
@@ -458,9 +518,10 @@ atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stre
     if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
     Params p{};
     fill_geometry(p, a);
+    const bool general = (a.T % a.ct) || (a.H % a.ch) || (a.W % a.cw);
     if (a.rope == nullptr) {
-        if (a.elem_bytes == 2) return dispatch<2>(p, false, 0, dev, stream);
-        return dispatch<4>(p, false, 0, dev, stream);
+        if (a.elem_bytes == 2) return dispatch<2>(p, false, 0, general, dev, stream);
+        return dispatch<4>(p, false, 0, general, dev, stream);
     }
     const atlas_rope &r = *a.rope;
     const size_t n = rope_table_entries(a.T, a.H, a.W, r);
@@ -483,8 +544,8 @@ atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stre
     p.tab_base[0] = 0;
     p.tab_base[1] = static_cast<uint32_t>(a.T) * p.half[0];
     p.tab_base[2] = p.tab_base[1] + static_cast<uint32_t>(a.H) * p.half[1];
-    if (a.elem_bytes == 2) return dispatch<2>(p, true, 0, dev, stream);
-    return dispatch<4>(p, true, 0, dev, stream);
+    if (a.elem_bytes == 2) return dispatch<2>(p, true, 0, general, dev, stream);
+    return dispatch<4>(p, true, 0, general, dev, stream);
 }
 
 }  // namespace atlas
