@@ -66,6 +66,10 @@ def _declare(lib):
     lib.atlas_oracle_attention_head_windows.argtypes = (
         [_i64, _i64, _ptr, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
          _i64, _ptr, _ptr, _ptr, _ptr, ctypes.c_int])
+    lib.atlas_oracle_attention_head_aligned.restype = ctypes.c_int
+    lib.atlas_oracle_attention_head_aligned.argtypes = (
+        [_i64] * 10 + [_f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr, _i64, _ptr, _ptr, _ptr, _ptr,
+                       ctypes.c_int])
     lib.atlas_oracle_attention_head.restype = ctypes.c_int
     lib.atlas_oracle_attention_head.argtypes = (
         [_i64, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
@@ -202,6 +206,57 @@ class Oracle:
         if st != 0:
             raise MemoryError("oracle allocation failed")
         return o, lse
+
+    def attention_head_aligned(self, grid, cube, global_grid, scale, k_d, v_d, kd_lo: int,
+                               k_g, v_g, q_ids, q, n_threads: int = 1):
+        """"Aligned proxy tokens only" variant for one head: detail rows in
+        cube order of ``grid`` cut into ``cube``; global rows in raster order
+        of ``global_grid``. A detail query sees its own cube and the global
+        keys whose scaled position lies in that cube; a global query sees
+        every global key. Arguments and results as :meth:`attention_head`."""
+        f = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+        q = f(q)
+        n_q, D = q.shape
+        k_d = f(k_d).reshape(-1, D) if k_d is not None else np.zeros((0, D))
+        v_d = f(v_d).reshape(-1, D) if v_d is not None else np.zeros((0, D))
+        k_g = f(k_g).reshape(-1, D) if k_g is not None else np.zeros((0, D))
+        v_g = f(v_g).reshape(-1, D) if v_g is not None else np.zeros((0, D))
+        assert k_d.shape == v_d.shape and k_g.shape == v_g.shape
+        assert k_g.shape[0] == global_grid[0] * global_grid[1] * global_grid[2]
+        ids = np.ascontiguousarray(np.asarray(q_ids, dtype=np.int64))
+        assert ids.shape == (n_q,)
+        o = np.empty((n_q, D), dtype=np.float64)
+        lse = np.empty(n_q, dtype=np.float64)
+        st = self.lib.atlas_oracle_attention_head_aligned(
+            *grid, *cube, *global_grid, D, float(scale), k_d.ctypes.data, v_d.ctypes.data,
+            kd_lo, kd_lo + k_d.shape[0], k_g.ctypes.data, v_g.ctypes.data, n_q,
+            ids.ctypes.data, q.ctypes.data, o.ctypes.data, lse.ctypes.data, int(n_threads))
+        if st == 1:
+            raise ValueError("an allowed detail key lies outside the rows given")
+        if st == 3:
+            raise RuntimeError("cube positions are not a permutation")
+        if st != 0:
+            raise MemoryError("oracle allocation failed")
+        return o, lse
+
+    def attention_full_aligned(self, q_d, k_d, v_d, grid, cube, q_g, k_g, v_g, global_grid,
+                               scale, n_threads: int = 1):
+        """All rows, all heads, of the aligned variant. Detail tensors
+        [N, heads, D] in cube order, global [G, heads, D] in raster order.
+        Returns (o_d, o_g, lse [heads, N+G])."""
+        q_d = np.asarray(q_d, dtype=np.float64)
+        q_g = np.asarray(q_g, dtype=np.float64)
+        N, heads, D = q_d.shape
+        G = q_g.shape[0]
+        o_d, o_g, lse = np.empty((N, heads, D)), np.empty((G, heads, D)), np.empty((heads, N + G))
+        for hh in range(heads):
+            q_all = np.concatenate([q_d[:, hh, :], q_g[:, hh, :]], axis=0)
+            o, l = self.attention_head_aligned(
+                grid, cube, global_grid, scale, np.asarray(k_d)[:, hh, :],
+                np.asarray(v_d)[:, hh, :], 0, np.asarray(k_g)[:, hh, :],
+                np.asarray(v_g)[:, hh, :], np.arange(N + G, dtype=np.int64), q_all, n_threads)
+            o_d[:, hh, :], o_g[:, hh, :], lse[hh] = o[:N], o[N:], l
+        return o_d, o_g, lse
 
     def attention_full(self, q_d, k_d, v_d, window_len, q_g, k_g, v_g,
                        scale, n_threads: int = 1, win_off=None):

@@ -37,7 +37,10 @@
  *     angle p * theta^(-2k/d), p = index * scale for that axis;
  *   - one joint softmax per query row over every allowed key; a detail
  *     query is allowed the keys of its own cube and every global key; a
- *     global query is allowed every global key and no detail key.
+ *     global query is allowed every global key and no detail key;
+ *   - in the "aligned proxy tokens only" variant a detail query is allowed,
+ *     of the global keys, only those whose scaled position falls inside its
+ *     cube (see atlas_oracle_attention_head_aligned).
  *
  * Arithmetic is fp64 throughout, with no intermediate rounding.
  */
@@ -213,13 +216,46 @@ static int64_t window_of(int64_t x, int64_t L, const int64_t *win_off, int64_t n
     return lo;
 }
 
-static int allowed(int64_t q, int64_t k, int64_t N, int64_t L,
-                   const int64_t *win_off, int64_t n_win)
+/* "Aligned proxy tokens only" variant ([TS] Methodologie 2: a detail query
+ * sees the global tokens aligned with it; position alignment puts global
+ * token (tg, hg, wg) of a t x h x w grid at detail-grid coordinates
+ * (tg*T/t, hg*H/h, wg*W/w)). Reading: a global key is aligned with a detail
+ * cube when that scaled position lies inside the cube, i.e. on each axis
+ * a <= tg*T/t < a + e for the cube's start a and extent e, compared exactly
+ * as a*t <= tg*T < (a+e)*t. */
+struct mask {
+    int64_t N, L, n_win;
+    const int64_t *win_off;
+    int aligned;                 /* 0: a detail query sees every global key */
+    int64_t T, H, W, ct, ch, cw; /* aligned only: detail grid and cube */
+    int64_t t, h, w;             /* aligned only: global grid */
+    const int64_t *cube_of;      /* aligned only: cube id of each detail position */
+};
+
+static int axis_aligned(int64_t a, int64_t e, int64_t g, int64_t E, int64_t e_glob)
 {
-    int q_detail = q < N, k_detail = k < N;
-    if (q_detail && k_detail)
-        return window_of(q, L, win_off, n_win) == window_of(k, L, win_off, n_win);
-    if (q_detail && !k_detail) return 1;
+    return a * e_glob <= g * E && g * E < (a + e) * e_glob;
+}
+
+static int global_aligned(const struct mask *m, int64_t c, int64_t g)
+{
+    int64_t nh = (m->H + m->ch - 1) / m->ch, nw = (m->W + m->cw - 1) / m->cw;
+    int64_t bt = c / (nh * nw), bh = (c / nw) % nh, bw = c % nw;
+    int64_t gt = g / (m->h * m->w), gh = (g / m->w) % m->h, gw = g % m->w;
+    return axis_aligned(bt * m->ct, cube_extent(m->T, m->ct, bt), gt, m->T, m->t) &&
+           axis_aligned(bh * m->ch, cube_extent(m->H, m->ch, bh), gh, m->H, m->h) &&
+           axis_aligned(bw * m->cw, cube_extent(m->W, m->cw, bw), gw, m->W, m->w);
+}
+
+static int allowed(const struct mask *m, int64_t q, int64_t k)
+{
+    int q_detail = q < m->N, k_detail = k < m->N;
+    if (q_detail && k_detail) {
+        if (m->aligned) return m->cube_of[q] == m->cube_of[k];
+        return window_of(q, m->L, m->win_off, m->n_win) ==
+               window_of(k, m->L, m->win_off, m->n_win);
+    }
+    if (q_detail && !k_detail) return m->aligned ? global_aligned(m, m->cube_of[q], k - m->N) : 1;
     if (!q_detail && k_detail) return 0;
     return 1;
 }
@@ -236,18 +272,13 @@ static int allowed(int64_t q, int64_t k, int64_t N, int64_t L,
  * k_g/v_g hold all G global rows. If an allowed detail key falls outside
  * the rows supplied the function returns 1 (caller error); 2 on allocation
  * failure; 0 on success. */
-int atlas_oracle_attention_head_windows(int64_t n_detail, int64_t window_len,
-                                        const int64_t *win_off, int64_t n_win,
-                                        int64_t n_global, int64_t head_dim,
-                                        double scale,
-                                        const double *k_d, const double *v_d,
-                                        int64_t kd_lo, int64_t kd_hi,
-                                        const double *k_g, const double *v_g,
-                                        int64_t n_q, const int64_t *q_ids,
-                                        const double *q, double *o, double *lse,
-                                        int n_threads)
+static int attention_core(const struct mask *msk, int64_t n_global, int64_t head_dim,
+                          double scale, const double *k_d, const double *v_d,
+                          int64_t kd_lo, int64_t kd_hi, const double *k_g, const double *v_g,
+                          int64_t n_q, const int64_t *q_ids, const double *q, double *o,
+                          double *lse, int n_threads)
 {
-    int64_t N = n_detail, G = n_global, D = head_dim;
+    int64_t N = msk->N, G = n_global, D = head_dim;
     int status = 0;
     if (n_threads < 1) n_threads = 1;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
@@ -266,7 +297,7 @@ int atlas_oracle_attention_head_windows(int64_t n_detail, int64_t window_len,
         int64_t n_allowed = 0;
         int bad = 0;
         for (int64_t kid = 0; kid < N + G; ++kid) {
-            if (!allowed(qid, kid, N, window_len, win_off, n_win)) continue;
+            if (!allowed(msk, qid, kid)) continue;
             const double *kr, *vr;
             if (kid < N) {
                 if (kid < kd_lo || kid >= kd_hi) { bad = 1; break; }
@@ -306,6 +337,68 @@ int atlas_oracle_attention_head_windows(int64_t n_detail, int64_t window_len,
         free(vrow);
     }
     return status;
+}
+
+int atlas_oracle_attention_head_windows(int64_t n_detail, int64_t window_len,
+                                        const int64_t *win_off, int64_t n_win,
+                                        int64_t n_global, int64_t head_dim,
+                                        double scale,
+                                        const double *k_d, const double *v_d,
+                                        int64_t kd_lo, int64_t kd_hi,
+                                        const double *k_g, const double *v_g,
+                                        int64_t n_q, const int64_t *q_ids,
+                                        const double *q, double *o, double *lse,
+                                        int n_threads)
+{
+    struct mask m;
+    memset(&m, 0, sizeof m);
+    m.N = n_detail;
+    m.L = window_len;
+    m.win_off = win_off;
+    m.n_win = n_win;
+    return attention_core(&m, n_global, head_dim, scale, k_d, v_d, kd_lo, kd_hi, k_g, v_g,
+                          n_q, q_ids, q, o, lse, n_threads);
+}
+
+/* One head of the aligned variant. Detail grid T x H x W cut into cubes
+ * ct x ch x cw (partial cubes at the far edges), detail rows in cube order;
+ * global grid t x h x w (G = t*h*w rows, raster order). A detail query sees
+ * its own cube and the global keys aligned with that cube; a global query
+ * sees every global key. Arguments and return value otherwise as
+ * atlas_oracle_attention_head_windows; 3 if the cube positions are not a
+ * permutation (defensive; cannot happen with a correct position map). */
+int atlas_oracle_attention_head_aligned(int64_t T, int64_t H, int64_t W,
+                                        int64_t ct, int64_t ch, int64_t cw,
+                                        int64_t t, int64_t h, int64_t w,
+                                        int64_t head_dim, double scale,
+                                        const double *k_d, const double *v_d,
+                                        int64_t kd_lo, int64_t kd_hi,
+                                        const double *k_g, const double *v_g,
+                                        int64_t n_q, const int64_t *q_ids,
+                                        const double *q, double *o, double *lse,
+                                        int n_threads)
+{
+    struct mask m;
+    memset(&m, 0, sizeof m);
+    m.N = T * H * W;
+    m.aligned = 1;
+    m.T = T; m.H = H; m.W = W;
+    m.ct = ct; m.ch = ch; m.cw = cw;
+    m.t = t; m.h = h; m.w = w;
+    int64_t *cube_of = (int64_t *)malloc((size_t)(m.N > 0 ? m.N : 1) * sizeof(int64_t));
+    if (!cube_of) return 2;
+    int64_t nh = (H + ch - 1) / ch, nw = (W + cw - 1) / cw;
+    for (int64_t r = 0; r < m.N; ++r) {
+        int64_t tt = r / (H * W), hh = (r / W) % H, ww = r % W;
+        int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        if (j < 0 || j >= m.N) { free(cube_of); return 3; }   /* not a permutation */
+        cube_of[j] = ((tt / ct) * nh + hh / ch) * nw + ww / cw;
+    }
+    m.cube_of = cube_of;
+    int st = attention_core(&m, t * h * w, head_dim, scale, k_d, v_d, kd_lo, kd_hi, k_g, v_g,
+                            n_q, q_ids, q, o, lse, n_threads);
+    free(cube_of);
+    return st;
 }
 
 /* Windows of window_len consecutive detail positions (the cube divides the

@@ -490,7 +490,95 @@ def pin_attention_offsets_equal_fixed_windows(o):
         assert np.array_equal(x, y)
 
 
+# "Aligned proxy tokens only": detail grid, cube, global grid.
+ALIGNED_CASES = [
+    ((4, 8, 8), (2, 4, 4), (2, 4, 4)),     # ratios 2, 2, 2; they divide the cube
+    ((3, 8, 12), (3, 4, 4), (3, 2, 3)),    # ratios 1, 4, 4
+    ((5, 7, 9), (2, 3, 4), (2, 3, 4)),     # ratios 2.5, 7/3, 9/4; partial cubes
+    ((4, 6, 10), (2, 4, 4), (4, 3, 5)),    # ratios 1, 2, 2; partial cubes along h and w
+]
+
+
+def aligned_mask(grid, cube, global_grid):
+    """Allowed-matrix of the aligned variant from token coordinates: detail
+    cube ids by floor division, detail tokens in lexsort cube order; a global
+    token's cube is the one holding its scaled position, floor(g*T/(t*c)) on
+    each axis."""
+    T, H, W = grid
+    ct, ch, cw = cube
+    t, h, w = global_grid
+    N, G = T * H * W, t * h * w
+    order = lexsort_order(grid, cube)
+    dkey = np.stack([order // (H * W) // ct, (order // W) % H // ch, order % W // cw], -1)
+    g = np.arange(G)
+    gkey = np.stack([(g // (h * w)) * T // (t * ct), ((g // w) % h) * H // (h * ch),
+                     (g % w) * W // (w * cw)], -1)
+    mask = np.zeros((N + G, N + G), dtype=bool)
+    mask[:N, :N] = np.all(dkey[:, None, :] == dkey[None, :, :], -1)
+    mask[:N, N:] = np.all(dkey[:, None, :] == gkey[None, :, :], -1)
+    mask[N:, N:] = True
+    return mask
+
+
+def pin_attention_aligned_dense_sdpa(o):
+    """Aligned variant equal to dense masked attention (mask above)."""
+    for ci, (grid, cube, gg) in enumerate(ALIGNED_CASES):
+        G, heads, D = gg[0] * gg[1] * gg[2], 2, 16
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 400 + ci)
+        od, og, lse = o.attention_full_aligned(qd, kd, vd, grid, cube, qg, kg, vg, gg, 0.3)
+        mask = torch.from_numpy(aligned_mask(grid, cube, gg))
+        q = torch.from_numpy(np.concatenate([qd, qg])).permute(1, 0, 2)
+        k = torch.from_numpy(np.concatenate([kd, kg])).permute(1, 0, 2)
+        v = torch.from_numpy(np.concatenate([vd, vg])).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k, v, attn_mask=mask, scale=0.3).permute(1, 0, 2).numpy()
+        assert np.max(np.abs(ref - np.concatenate([od, og]))) < 1e-12, (grid, cube, gg)
+        logits = np.where(mask.numpy()[None], (q @ k.transpose(1, 2)).numpy() * 0.3, -np.inf)
+        mx = logits.max(-1, keepdims=True)
+        ref_lse = (mx + np.log(np.exp(logits - mx).sum(-1, keepdims=True)))[..., 0]
+        assert np.max(np.abs(ref_lse - lse)) < 1e-12, (grid, cube, gg)
+
+
+def pin_attention_aligned_counts(o):
+    """K = 0: LSE = log(number of allowed keys). Along an axis of E detail
+    and e global tokens, the global indices whose scaled position g*E/e lies
+    in [a, a+x) number ceil((a+x)*e/E) - ceil(a*e/E)."""
+    for ci, (grid, cube, gg) in enumerate(ALIGNED_CASES):
+        G, heads, D = gg[0] * gg[1] * gg[2], 1, 8
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 410 + ci)
+        kd[:] = 0.0
+        kg[:] = 0.0
+        _, _, lse = o.attention_full_aligned(qd, kd, vd, grid, cube, qg, kg, vg, gg, 0.7)
+        order = lexsort_order(grid, cube)
+        n_allowed = np.empty(N)
+        for j, r in enumerate(order):
+            coords = (r // (grid[1] * grid[2]), (r // grid[2]) % grid[1], r % grid[2])
+            n_det, n_glob = 1, 1
+            for x, E, c, e in zip(coords, grid, cube, gg):
+                a = (x // c) * c
+                ext = min(c, E - a)
+                n_det *= ext
+                n_glob *= -(-(a + ext) * e // E) - -(-a * e // E)
+            n_allowed[j] = n_det + n_glob
+        assert np.max(np.abs(lse[0, :N] - np.log(n_allowed))) < 1e-12, (grid, cube, gg)
+        assert np.max(np.abs(lse[0, N:] - math.log(G))) < 1e-12
+
+
+def pin_attention_aligned_one_cube_sees_all(o):
+    """A single cube covering the volume is aligned with every global token:
+    the aligned variant equals the all-global-keys one."""
+    grid, gg, heads, D = (2, 4, 6), (1, 2, 3), 2, 16
+    G = 6
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 420)
+    a = o.attention_full_aligned(qd, kd, vd, grid, grid, qg, kg, vg, gg, 0.25)
+    b = o.attention_full(qd, kd, vd, N, qg, kg, vg, 0.25)
+    for x, y in zip(a, b):
+        assert np.max(np.abs(x - y)) < 1e-12
+
+
 ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
+             pin_attention_aligned_dense_sdpa, pin_attention_aligned_counts,
+             pin_attention_aligned_one_cube_sees_all,
              pin_attention_offsets_equal_fixed_windows, pin_attention_full_when_one_cube,
              pin_attention_single_token_windows, pin_attention_zero_keys_mean,
              pin_attention_rows_sum_to_one, pin_attention_global_ignores_detail,

@@ -15,7 +15,17 @@ MUTANTS = [
      "if (win_off[mid] < x) lo = mid; else hi = mid - 1;"),
     ("partial_cube_extent", "return (b + 1) * c <= E ? c : E - b * c;", "return c;"),
     ("global_sees_detail", "if (!q_detail && k_detail) return 0;", "if (!q_detail && k_detail) return 1;"),
-    ("detail_misses_global", "if (q_detail && !k_detail) return 1;", "if (q_detail && !k_detail) return 0;"),
+    ("detail_misses_global", "return m->aligned ? global_aligned(m, m->cube_of[q], k - m->N) : 1;",
+     "return m->aligned ? global_aligned(m, m->cube_of[q], k - m->N) : 0;"),
+    ("aligned_sees_all", "return m->aligned ? global_aligned(m, m->cube_of[q], k - m->N) : 1;",
+     "return 1;"),
+    ("aligned_upper_bound_inclusive", "g * E < (a + e) * e_glob;", "g * E <= (a + e) * e_glob;"),
+    ("aligned_ratio_inverted", "return a * e_glob <= g * E && g * E < (a + e) * e_glob;",
+     "return a * E <= g * e_glob && g * e_glob < (a + e) * E;"),
+    ("aligned_axis_mixup", "int64_t gt = g / (m->h * m->w), gh = (g / m->w) % m->h, gw = g % m->w;",
+     "int64_t gt = g / (m->h * m->w), gh = (g / m->h) % m->w, gw = g % m->w;"),
+    ("aligned_cube_coords", "int64_t bt = c / (nh * nw), bh = (c / nw) % nh, bw = c % nw;",
+     "int64_t bt = c / (nh * nw), bh = (c / nh) % nw, bw = c % nw;"),
     ("rope_sign", "y[off + 2 * k] = x0 * c - x1 * s;", "y[off + 2 * k] = x0 * c + x1 * s;"),
     ("rope_freq_width", "pow(theta, -2.0 * (double)k / (double)d)", "pow(theta, -2.0 * (double)k / (double)(d + 2))"),
     ("rope_wrong_axis", "rope_segment(xr, yr, d_t + d_h, d_w, p_w, theta);", "rope_segment(xr, yr, d_t + d_h, d_w, p_h, theta);"),
