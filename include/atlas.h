@@ -240,6 +240,105 @@ atlas_status atlas_local_global_attn_windows(
     int32_t head_dim, float softmax_scale, atlas_dtype dtype, void *o_d,
     void *o_g, float *lse, atlas_stream_t stream);
 
+/*
+ * Layout of a call to atlas_local_global_attn_ex.
+ *
+ * batch: number of problems of the same shape stacked along the rows (>= 1).
+ *   Detail tensors hold batch*n_detail rows (problem b at rows
+ *   [b*n_detail, (b+1)*n_detail)), global tensors batch*n_global rows. A
+ *   query sees only keys of its own problem.
+ * Detail windows, the same for every problem:
+ *   window_offsets == NULL: windows of window_len rows (n_detail %
+ *     window_len == 0);
+ *   window_offsets != NULL: DEVICE array of n_windows+1 int32 offsets over
+ *     one problem's rows, increasing, [0] = 0, [n_windows] = n_detail
+ *     (window_len is ignored).
+ * global_window_offsets: NULL: a detail query sees every global key of its
+ *   problem. Otherwise the "aligned proxy tokens only" variant: DEVICE array
+ *   of n_windows+1 int32 offsets over one problem's global rows,
+ *   non-decreasing, [0] = 0, [n_windows] = n_global; the queries of window
+ *   w see the global keys [global_window_offsets[w],
+ *   global_window_offsets[w+1]) of their problem. n_windows must then be the
+ *   window count (n_detail / window_len without window_offsets). Global
+ *   queries always see every global key of their problem.
+ * The library never reads the offset arrays on the host. Contents other
+ * than described give undefined rows, but every access stays inside the
+ * tensors: a detail row always sees its own key, and ranges are clamped.
+ */
+typedef struct {
+    int64_t batch;
+    int64_t window_len;
+    const int32_t *window_offsets;
+    int64_t n_windows;
+    const int32_t *global_window_offsets;
+} atlas_attn_layout;
+
+/*
+ * atlas_local_global_attn_ex -- steps (3) and (4), general layout: batch of
+ * problems, windows of fixed or variable length, and the all-global-keys or
+ * the aligned-global-keys variant.
+ *
+ * Passages: as atlas_local_global_attn; for the aligned variant also
+ * Methodologie 2, position alignment (global token (tg, hg, wg) of a t x h x w
+ * grid sits at detail-grid position (tg*T/t, hg*H/h, wg*W/w); it is aligned
+ * with the cube holding that point). When the ratios T/t, H/h, W/w are
+ * integers dividing the cube sizes, the aligned global tokens of cube c are
+ * cube c of the global grid cut into atlas_aligned_global_cube's cube: reorder
+ * the global Q/K/V with atlas_cube_reorder using that cube, pass
+ * atlas_cube_window_offsets of it as global_window_offsets, and unorder o_g.
+ *
+ * n_detail, n_global: rows of ONE problem. layout: see atlas_attn_layout
+ * (NULL is an error). lse: optional fp32 [batch, heads, n_detail +
+ * n_global], per problem detail rows first, then global rows. Everything
+ * else as atlas_local_global_attn.
+ * Errors: NULL layout or required pointer (NULL); batch < 1, inconsistent
+ * windows, more than 2^31-1 rows in a tensor (SHAPE); misaligned offsets
+ * (ALIGN); as atlas_local_global_attn otherwise.
+ */
+atlas_status atlas_local_global_attn_ex(
+    const void *q_d, const void *k_d, const void *v_d, int64_t n_detail,
+    const void *q_g, const void *k_g, const void *v_g, int64_t n_global,
+    const atlas_attn_layout *layout, int32_t heads, int32_t head_dim,
+    float softmax_scale, atlas_dtype dtype, void *o_d, void *o_g, float *lse,
+    atlas_stream_t stream);
+
+/*
+ * atlas_aligned_global_cube -- the global-grid cube whose cubes are the
+ * aligned sets of the detail cubes (host).
+ *
+ * Passage: Methodologie 2, position alignment (see atlas_local_global_attn_ex).
+ * With ratios r = (T/t, H/h, W/w) integral and dividing (ct, ch, cw), global
+ * cube c of the global grid cut into (ct/r_t, ch/r_h, cw/r_w) holds exactly
+ * the global tokens aligned with detail cube c, partial cubes included, and
+ * both grids have the same number of cubes. *global_cube receives that cube.
+ * Errors: NULL global_cube (NULL); non-positive extents (SHAPE); ratios not
+ * integral or not dividing the cube (UNSUPPORTED). Host only.
+ */
+atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 cube,
+                                       atlas_grid3 global_grid,
+                                       atlas_cube3 *global_cube);
+
+/*
+ * Batched permutations: `batch` problems of the same grid stacked along the
+ * rows ([batch * T*H*W, heads, head_dim]); each problem is permuted (and
+ * rotated) on its own, exactly as the unbatched call would. batch >= 1;
+ * batch * T*H*W must stay below 2^31. Errors as the unbatched calls, SHAPE
+ * for batch < 1.
+ */
+atlas_status atlas_cube_reorder_batched(const void *src, void *dst, int64_t batch,
+                                        atlas_grid3 grid, atlas_cube3 cube,
+                                        int32_t heads, int32_t head_dim,
+                                        atlas_dtype dtype, const atlas_rope *rope,
+                                        atlas_stream_t stream);
+atlas_status atlas_cube_unorder_batched(const void *src, void *dst, int64_t batch,
+                                        atlas_grid3 grid, atlas_cube3 cube,
+                                        int32_t heads, int32_t head_dim,
+                                        atlas_dtype dtype, atlas_stream_t stream);
+atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t batch,
+                                  atlas_grid3 grid, int32_t heads, int32_t head_dim,
+                                  atlas_dtype dtype, const atlas_rope *rope,
+                                  atlas_stream_t stream);
+
 /* Human-readable name of a status. Never NULL. */
 const char *atlas_status_string(atlas_status status);
 

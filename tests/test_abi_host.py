@@ -165,3 +165,79 @@ def test_windows_attention_validation(lib):
     assert call(n_win=0) == atlas.ERR_SHAPE
     assert call(n_win=300) == atlas.ERR_SHAPE
     assert call(off=FAKE + (8 << 28) + 2) == atlas.ERR_ALIGN
+
+
+def test_attention_ex_validation(lib):
+    base = [FAKE, FAKE + (1 << 28), FAKE + (2 << 28), 256, FAKE + (3 << 28), FAKE + (4 << 28),
+            FAKE + (5 << 28), 32]
+    outs = [FAKE + (6 << 28), FAKE + (7 << 28)]
+
+    def call(ly, n_d=256, heads=2, lse=None):
+        args = list(base)
+        args[3] = n_d
+        return lib.atlas_local_global_attn_ex(*args, ctypes.byref(ly) if ly else None, heads, 64,
+                                              0.0, atlas.BF16, *outs, lse, None)
+    L = atlas.AttnLayout
+    assert call(None) == atlas.ERR_NULL
+    assert call(L(0, 32, None, 0, None)) == atlas.ERR_SHAPE            # batch < 1
+    assert call(L(1, 30, None, 0, None)) == atlas.ERR_SHAPE            # 256 % 30
+    assert call(L(1, 32, None, 7, FAKE + (8 << 28))) == atlas.ERR_SHAPE  # 8 windows, not 7
+    assert call(L(1, 32, None, 8, FAKE + (8 << 28) + 2)) == atlas.ERR_ALIGN
+    assert call(L(1, 0, FAKE + (8 << 28), 0, None)) == atlas.ERR_SHAPE   # no windows
+    assert call(L(1 << 30, 32, None, 0, None)) == atlas.ERR_SHAPE      # too many rows
+    # batch 2: the tensors hold 512 detail rows; the outputs overlap k_d's second half
+    assert lib.atlas_local_global_attn_ex(
+        FAKE, FAKE + 256 * 256, FAKE + (2 << 28), 256, FAKE + (3 << 28), FAKE + (4 << 28),
+        FAKE + (5 << 28), 32, ctypes.byref(L(2, 32, None, 0, None)), 1, 64, 0.0, atlas.BF16,
+        FAKE + 384 * 256, FAKE + (7 << 28), None, None) == atlas.ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        assert call(L(2, 32, None, 8, FAKE + (8 << 28))) == atlas.ERR_DEVICE
+
+
+def test_aligned_global_cube_host(lib):
+    assert atlas.aligned_global_cube((21, 48, 80), (3, 16, 16), (21, 12, 20)) == (3, 4, 4)
+    assert atlas.aligned_global_cube((42, 144, 240), (6, 16, 16), (21, 18, 30)) == (3, 2, 2)
+    out = atlas.Cube3()
+    G3, C3 = atlas.Grid3, atlas.Cube3
+    assert lib.atlas_aligned_global_cube(G3(5, 7, 9), C3(2, 3, 4), G3(2, 3, 4),
+                                         ctypes.byref(out)) == atlas.ERR_UNSUPPORTED
+    assert lib.atlas_aligned_global_cube(G3(4, 8, 8), C3(2, 4, 3), G3(2, 4, 4),
+                                         ctypes.byref(out)) == atlas.ERR_UNSUPPORTED
+    assert lib.atlas_aligned_global_cube(G3(4, 8, 8), C3(2, 4, 4), G3(0, 4, 4),
+                                         ctypes.byref(out)) == atlas.ERR_SHAPE
+    assert lib.atlas_aligned_global_cube(G3(4, 8, 8), C3(2, 4, 4), G3(2, 4, 4),
+                                         None) == atlas.ERR_NULL
+
+
+def test_aligned_global_cube_matches_oracle(lib):
+    """For integral ratios, cube c of the global grid cut into the returned
+    cube holds exactly the global tokens the oracle's aligned predicate
+    gives detail cube c (K = 0 makes the oracle's LSE a key count, and the
+    probe below names the keys)."""
+    import numpy as np
+    import oracle
+    orc = oracle.Oracle()
+    for grid, cube, gg in (((4, 8, 8), (2, 4, 4), (2, 4, 4)), ((5, 12, 20), (2, 8, 8), (5, 3, 5)),
+                           ((6, 16, 16), (3, 8, 8), (6, 4, 4))):
+        gcube = atlas.aligned_global_cube(grid, cube, gg)
+        goff = atlas.cube_window_offsets(gg, gcube).numpy()
+        doff = atlas.cube_window_offsets(grid, cube).numpy()
+        assert goff.size == doff.size
+        gpos = orc.cube_positions(gg, gcube)   # raster -> global cube order
+        G = gg[0] * gg[1] * gg[2]
+        D = 8
+        # V_g = one-hot of the raster index (first D rows only carry mass
+        # visibility): use indicator of "global cube order position in window w"
+        for w in range(doff.size - 1):
+            lo, hi = int(doff[w]), int(doff[w + 1])
+            vg = np.zeros((G, D))
+            inside = (gpos >= goff[w]) & (gpos < goff[w + 1])
+            vg[inside, 0] = 1.0
+            vg[~inside, 1] = 1.0
+            kd = np.zeros((hi - lo, D))
+            o, _ = orc.attention_head_aligned(grid, cube, gg, 1.0, kd, kd, lo, np.zeros((G, D)),
+                                              vg, np.arange(lo, hi), np.zeros((hi - lo, D)))
+            assert np.all(o[:, 1] == 0.0), (grid, w)
+            n_in = int(inside.sum())
+            assert np.allclose(o[:, 0], n_in / (hi - lo + n_in)), (grid, w)

@@ -39,6 +39,12 @@ class Rope(ctypes.Structure):
                 ("scale_h", ctypes.c_double), ("scale_w", ctypes.c_double)]
 
 
+class AttnLayout(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("window_len", ctypes.c_int64),
+                ("window_offsets", ctypes.c_void_p), ("n_windows", ctypes.c_int64),
+                ("global_window_offsets", ctypes.c_void_p)]
+
+
 def make_rope(theta, split, scales) -> Rope:
     d_t, d_h, d_w = (int(v) for v in split)
     s_t, s_h, s_w = (float(v) for v in scales)
@@ -78,6 +84,21 @@ def _declare(lib):
     lib.atlas_local_global_attn_windows.argtypes = [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp,
                                                     _i64, _i32, _i32, ctypes.c_float, ctypes.c_int,
                                                     _vp, _vp, _vp, _vp]
+    lib.atlas_local_global_attn_ex.restype = ctypes.c_int
+    lib.atlas_local_global_attn_ex.argtypes = [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
+                                               ctypes.POINTER(AttnLayout), _i32, _i32,
+                                               ctypes.c_float, ctypes.c_int, _vp, _vp, _vp, _vp]
+    lib.atlas_aligned_global_cube.restype = ctypes.c_int
+    lib.atlas_aligned_global_cube.argtypes = [Grid3, Cube3, Grid3, ctypes.POINTER(Cube3)]
+    lib.atlas_cube_reorder_batched.restype = ctypes.c_int
+    lib.atlas_cube_reorder_batched.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
+                                               ctypes.c_int, ctypes.POINTER(Rope), _vp]
+    lib.atlas_cube_unorder_batched.restype = ctypes.c_int
+    lib.atlas_cube_unorder_batched.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
+                                               ctypes.c_int, _vp]
+    lib.atlas_rope3d_batched.restype = ctypes.c_int
+    lib.atlas_rope3d_batched.argtypes = [_vp, _vp, _i64, Grid3, _i32, _i32, ctypes.c_int,
+                                         ctypes.POINTER(Rope), _vp]
     lib.atlas_cube_window_offsets.restype = ctypes.c_int
     lib.atlas_cube_window_offsets.argtypes = [Grid3, Cube3, _vp, _i64, ctypes.POINTER(_i64)]
     lib.atlas_status_string.restype = ctypes.c_char_p
@@ -233,6 +254,76 @@ def local_global_attn_windows(q_d, k_d, v_d, window_offsets, q_g, k_g, v_g, o_d,
         _dtype_code(ref), nz(o_d, n_d), nz(o_g, n_g), _ptr(lse), _stream(ref, stream))
     _check(st, "atlas_local_global_attn_windows")
     return o_d, o_g, lse
+
+
+def local_global_attn_ex(q_d, k_d, v_d, q_g, k_g, v_g, o_d, o_g, lse=None, *, batch=1,
+                         window_len=0, window_offsets=None, global_window_offsets=None,
+                         softmax_scale: float = 0.0, stream=None):
+    """General layout: ``batch`` problems stacked along the rows (detail
+    tensors [batch*N, heads, D], global [batch*G, heads, D], lse [batch,
+    heads, N+G]); windows of ``window_len`` rows or the device int32
+    ``window_offsets`` of one problem; with ``global_window_offsets`` (device
+    int32 [n_windows+1], one problem) the queries of window w see only those
+    global keys (the aligned variant)."""
+    ref = q_d if q_d is not None and q_d.shape[0] > 0 else q_g
+    heads, hd = ref.shape[1], ref.shape[2]
+    n_d = (q_d.shape[0] if q_d is not None else 0) // batch
+    n_g = (q_g.shape[0] if q_g is not None else 0) // batch
+    nz = lambda t, n: _ptr(t) if (t is not None and n > 0) else None
+    if window_offsets is not None:
+        n_win = window_offsets.numel() - 1
+    elif global_window_offsets is not None:
+        n_win = global_window_offsets.numel() - 1
+    else:
+        n_win = 0
+    wo = _ptr(window_offsets) if window_offsets is not None else None
+    gwo = _ptr(global_window_offsets) if global_window_offsets is not None else None
+    ly = AttnLayout(int(batch), int(window_len), wo.value if wo is not None else None,
+                    int(n_win), gwo.value if gwo is not None else None)
+    st = lib().atlas_local_global_attn_ex(
+        nz(q_d, n_d), nz(k_d, n_d), nz(v_d, n_d), n_d, nz(q_g, n_g), nz(k_g, n_g), nz(v_g, n_g),
+        n_g, ctypes.byref(ly), heads, hd, float(softmax_scale), _dtype_code(ref),
+        nz(o_d, n_d), nz(o_g, n_g), _ptr(lse), _stream(ref, stream))
+    _check(st, "atlas_local_global_attn_ex")
+    return o_d, o_g, lse
+
+
+def aligned_global_cube(grid, cube, global_grid):
+    """The global-grid cube whose cubes are the aligned sets of the detail
+    cubes (ratios must be integers dividing the cube)."""
+    out = Cube3()
+    _check(lib().atlas_aligned_global_cube(Grid3(*grid), Cube3(*cube), Grid3(*global_grid),
+                                           ctypes.byref(out)), "atlas_aligned_global_cube")
+    return (out.ct, out.ch, out.cw)
+
+
+def cube_reorder_batched(src, dst, batch, grid, cube, rope: Rope | None = None, stream=None):
+    """``cube_reorder`` of ``batch`` problems stacked along the rows."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_reorder_batched(
+        _ptr(src), _ptr(dst), int(batch), Grid3(*grid), Cube3(*cube), heads, hd,
+        _dtype_code(src), ctypes.byref(rope) if rope is not None else None, _stream(src, stream))
+    _check(st, "atlas_cube_reorder_batched")
+    return dst
+
+
+def cube_unorder_batched(src, dst, batch, grid, cube, stream=None):
+    """``cube_unorder`` of ``batch`` problems stacked along the rows."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_unorder_batched(_ptr(src), _ptr(dst), int(batch), Grid3(*grid),
+                                          Cube3(*cube), heads, hd, _dtype_code(src),
+                                          _stream(src, stream))
+    _check(st, "atlas_cube_unorder_batched")
+    return dst
+
+
+def rope3d_batched(src, dst, batch, grid, rope: Rope, stream=None):
+    """``rope3d`` of ``batch`` problems stacked along the rows."""
+    n, heads, hd = src.shape
+    st = lib().atlas_rope3d_batched(_ptr(src), _ptr(dst), int(batch), Grid3(*grid), heads, hd,
+                                    _dtype_code(src), ctypes.byref(rope), _stream(src, stream))
+    _check(st, "atlas_rope3d_batched")
+    return dst
 
 
 def last_device_error(stream=None) -> int:

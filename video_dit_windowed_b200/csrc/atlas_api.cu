@@ -103,22 +103,74 @@ atlas_status check_rope(const atlas_rope &r, int32_t head_dim, atlas_dtype dt) {
 
 using namespace atlas;
 
+namespace atlas {
+namespace {
+
+// Shared validation of the permutation entry points; `bytes` receives the
+// size of one tensor (all problems).
+atlas_status check_permute(const void *src, const void *dst, int64_t batch, atlas_grid3 grid,
+                           int32_t heads, int32_t head_dim, atlas_dtype dtype, size_t *bytes) {
+    if (!src || !dst) return ATLAS_ERR_NULL;
+    atlas_status st = check_grid(grid, heads, head_dim, dtype);
+    if (st != ATLAS_OK) return st;
+    if (batch < 1 || batch > kMaxRows || grid.T * grid.H * grid.W > kMaxRows / batch)
+        return ATLAS_ERR_SHAPE;
+    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
+    *bytes = static_cast<size_t>(batch * grid.T * grid.H * grid.W) * heads * head_dim *
+             elem_bytes(dtype);
+    return ATLAS_OK;
+}
+
+atlas_status reorder(const void *src, void *dst, int64_t batch, atlas_grid3 grid,
+                     atlas_cube3 cube, int32_t heads, int32_t head_dim, atlas_dtype dtype,
+                     const atlas_rope *rope, atlas_stream_t stream, bool noalloc) {
+    size_t bytes = 0;
+    atlas_status st = check_permute(src, dst, batch, grid, heads, head_dim, dtype, &bytes);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), 0, rope, batch};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return noalloc ? launch_permute_rope_noalloc(a, s) : launch_permute_rope(a, s);
+}
+
+atlas_status unorder(const void *src, void *dst, int64_t batch, atlas_grid3 grid,
+                     atlas_cube3 cube, int32_t heads, int32_t head_dim, atlas_dtype dtype,
+                     atlas_stream_t stream) {
+    size_t bytes = 0;
+    atlas_status st = check_permute(src, dst, batch, grid, heads, head_dim, dtype, &bytes);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), 1, nullptr, batch};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+atlas_status rope3d(const void *src, void *dst, int64_t batch, atlas_grid3 grid, int32_t heads,
+                    int32_t head_dim, atlas_dtype dtype, const atlas_rope *rope,
+                    atlas_stream_t stream) {
+    if (!rope) return ATLAS_ERR_NULL;
+    size_t bytes = 0;
+    atlas_status st = check_permute(src, dst, batch, grid, heads, head_dim, dtype, &bytes);
+    if (st != ATLAS_OK) return st;
+    if ((st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (src != dst && ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, 1, 1, 1,
+                  heads, head_dim, elem_bytes(dtype), 2, rope, batch};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace atlas
+
 ATLAS_API atlas_status atlas_cube_reorder(const void *src, void *dst, atlas_grid3 grid,
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, const atlas_rope *rope,
                                           atlas_stream_t stream) {
-    if (!src || !dst) return ATLAS_ERR_NULL;
-    atlas_status st = check_grid(grid, heads, head_dim, dtype);
-    if (st != ATLAS_OK) return st;
-    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
-    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
-    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
-    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
-                         elem_bytes(dtype);
-    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
-    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
-                  heads, head_dim, elem_bytes(dtype), 0, rope};
-    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+    return atlas::reorder(src, dst, 1, grid, cube, heads, head_dim, dtype, rope, stream, false);
 }
 
 ATLAS_API atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, atlas_grid3 grid,
@@ -126,74 +178,77 @@ ATLAS_API atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, at
                                                   int32_t head_dim, atlas_dtype dtype,
                                                   const atlas_rope *rope,
                                                   atlas_stream_t stream) {
-    if (!src || !dst) return ATLAS_ERR_NULL;
-    atlas_status st = check_grid(grid, heads, head_dim, dtype);
-    if (st != ATLAS_OK) return st;
-    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
-    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
-    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
-    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
-                         elem_bytes(dtype);
-    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
-    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
-                  heads, head_dim, elem_bytes(dtype), 0, rope};
-    return launch_permute_rope_noalloc(a, reinterpret_cast<cudaStream_t>(stream));
+    return atlas::reorder(src, dst, 1, grid, cube, heads, head_dim, dtype, rope, stream, true);
 }
 
 ATLAS_API atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, atlas_stream_t stream) {
-    if (!src || !dst) return ATLAS_ERR_NULL;
-    atlas_status st = check_grid(grid, heads, head_dim, dtype);
-    if (st != ATLAS_OK) return st;
-    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
-    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
-    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
-                         elem_bytes(dtype);
-    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
-    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
-                  heads, head_dim, elem_bytes(dtype), 1, nullptr};
-    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+    return atlas::unorder(src, dst, 1, grid, cube, heads, head_dim, dtype, stream);
 }
 
 ATLAS_API atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid, int32_t heads,
                                     int32_t head_dim, atlas_dtype dtype, const atlas_rope *rope,
                                     atlas_stream_t stream) {
-    if (!src || !dst || !rope) return ATLAS_ERR_NULL;
-    atlas_status st = check_grid(grid, heads, head_dim, dtype);
-    if (st != ATLAS_OK) return st;
-    if ((st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
-    if (!aligned16(src) || !aligned16(dst)) return ATLAS_ERR_ALIGN;
-    const size_t bytes = static_cast<size_t>(grid.T * grid.H * grid.W) * heads * head_dim *
-                         elem_bytes(dtype);
-    if (src != dst && ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
-    PermuteArgs a{src, dst, grid.T, grid.H, grid.W, 1, 1, 1,
-                  heads, head_dim, elem_bytes(dtype), 2, rope};
-    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+    return atlas::rope3d(src, dst, 1, grid, heads, head_dim, dtype, rope, stream);
+}
+
+ATLAS_API atlas_status atlas_cube_reorder_batched(const void *src, void *dst, int64_t batch,
+                                                  atlas_grid3 grid, atlas_cube3 cube,
+                                                  int32_t heads, int32_t head_dim,
+                                                  atlas_dtype dtype, const atlas_rope *rope,
+                                                  atlas_stream_t stream) {
+    return atlas::reorder(src, dst, batch, grid, cube, heads, head_dim, dtype, rope, stream,
+                          false);
+}
+
+ATLAS_API atlas_status atlas_cube_unorder_batched(const void *src, void *dst, int64_t batch,
+                                                  atlas_grid3 grid, atlas_cube3 cube,
+                                                  int32_t heads, int32_t head_dim,
+                                                  atlas_dtype dtype, atlas_stream_t stream) {
+    return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, stream);
+}
+
+ATLAS_API atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t batch,
+                                            atlas_grid3 grid, int32_t heads, int32_t head_dim,
+                                            atlas_dtype dtype, const atlas_rope *rope,
+                                            atlas_stream_t stream) {
+    return atlas::rope3d(src, dst, batch, grid, heads, head_dim, dtype, rope, stream);
 }
 
 namespace atlas {
 namespace {
 
-// Shared validation and dispatch of the two attention entry points. With
-// win_off (device, n_win+1 int32) the windows are its ranges; otherwise
-// windows of window_len rows.
+// Shared validation and dispatch of the attention entry points. n_detail
+// and n_global are rows of one problem; see atlas_attn_layout.
 atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d,
-                               int64_t n_detail, int64_t window_len, const int32_t *win_off,
-                               int64_t n_win, const void *q_g, const void *k_g, const void *v_g,
-                               int64_t n_global, int32_t heads, int32_t head_dim,
-                               float softmax_scale, atlas_dtype dtype, void *o_d, void *o_g,
-                               float *lse, atlas_stream_t stream) {
-    if (n_detail < 0 || n_global < 0 || heads < 1) return ATLAS_ERR_SHAPE;
-    if (win_off == nullptr) {
-        if (n_detail > 0 && (window_len < 1 || n_detail % window_len != 0)) return ATLAS_ERR_SHAPE;
+                               int64_t n_detail, const void *q_g, const void *k_g,
+                               const void *v_g, int64_t n_global, const atlas_attn_layout &ly,
+                               int32_t heads, int32_t head_dim, float softmax_scale,
+                               atlas_dtype dtype, void *o_d, void *o_g, float *lse,
+                               atlas_stream_t stream) {
+    if (n_detail < 0 || n_global < 0 || heads < 1 || ly.batch < 1) return ATLAS_ERR_SHAPE;
+    if (ly.batch > kMaxRows || n_detail > kMaxRows / ly.batch ||
+        n_global > kMaxRows / ly.batch || static_cast<int64_t>(heads) > 65535)
+        return ATLAS_ERR_SHAPE;
+    int64_t window_len = ly.window_len, n_win = 0;
+    const int32_t *win_off = n_detail > 0 ? ly.window_offsets : nullptr;
+    const int32_t *gwin_off = n_detail > 0 ? ly.global_window_offsets : nullptr;
+    if (n_detail > 0) {
+        if (win_off == nullptr) {
+            if (window_len < 1 || n_detail % window_len != 0) return ATLAS_ERR_SHAPE;
+            n_win = n_detail / window_len;
+            if (gwin_off && ly.n_windows != n_win) return ATLAS_ERR_SHAPE;
+        } else {
+            n_win = ly.n_windows;
+            if (n_win < 1 || n_win > n_detail) return ATLAS_ERR_SHAPE;
+            if (reinterpret_cast<uintptr_t>(win_off) & 3u) return ATLAS_ERR_ALIGN;
+            window_len = 1;
+        }
+        if (gwin_off && (reinterpret_cast<uintptr_t>(gwin_off) & 3u)) return ATLAS_ERR_ALIGN;
     } else {
-        if (n_win < 1 || n_win > n_detail) return ATLAS_ERR_SHAPE;
-        if (reinterpret_cast<uintptr_t>(win_off) & 3u) return ATLAS_ERR_ALIGN;
         window_len = 1;
     }
-    if (n_detail + n_global > kMaxRows || static_cast<int64_t>(heads) > 65535)
-        return ATLAS_ERR_SHAPE;
     if (n_detail > 0 && (!q_d || !k_d || !v_d || !o_d)) return ATLAS_ERR_NULL;
     if (n_global > 0 && (!q_g || !k_g || !v_g || !o_g)) return ATLAS_ERR_NULL;
     if (elem_bytes(dtype) == 0) return ATLAS_ERR_UNSUPPORTED;
@@ -204,7 +259,8 @@ atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATLAS_ERR_ALIGN;
     // Outputs must not overlap inputs.
     const size_t eb = static_cast<size_t>(elem_bytes(dtype)) * heads * head_dim;
-    const size_t bd = eb * static_cast<size_t>(n_detail), bg = eb * static_cast<size_t>(n_global);
+    const size_t bd = eb * static_cast<size_t>(n_detail * ly.batch),
+                 bg = eb * static_cast<size_t>(n_global * ly.batch);
     const void *ins[] = {q_d, k_d, v_d, q_g, k_g, v_g};
     const size_t in_bytes[] = {bd, bd, bd, bg, bg, bg};
     for (int i = 0; i < 6; ++i) {
@@ -218,8 +274,8 @@ atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d
     if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
     float scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(head_dim));
     AttnArgs a{q_d, k_d, v_d, n_detail, window_len, q_g, k_g, v_g, n_global,
-               heads, head_dim, scale, o_d, o_g, lse, n_detail > 0 ? win_off : nullptr,
-               n_detail > 0 ? n_win : 0};
+               heads, head_dim, scale, o_d, o_g, lse, win_off, win_off ? n_win : 0,
+               ly.batch, gwin_off, n_win};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dtype == ATLAS_BF16 ? launch_attn_tc_bf16(a, s) : launch_attn_simt_f32(a, s);
 }
@@ -233,9 +289,9 @@ ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d,
                                                int64_t n_global, int32_t heads, int32_t head_dim,
                                                float softmax_scale, atlas_dtype dtype, void *o_d,
                                                void *o_g, float *lse, atlas_stream_t stream) {
-    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, window_len, nullptr, 0, q_g, k_g,
-                                    v_g, n_global, heads, head_dim, softmax_scale, dtype, o_d,
-                                    o_g, lse, stream);
+    atlas_attn_layout ly{1, window_len, nullptr, 0, nullptr};
+    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, ly, heads,
+                                    head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
 }
 
 ATLAS_API atlas_status atlas_local_global_attn_windows(
@@ -244,10 +300,40 @@ ATLAS_API atlas_status atlas_local_global_attn_windows(
     const void *v_g, int64_t n_global, int32_t heads, int32_t head_dim, float softmax_scale,
     atlas_dtype dtype, void *o_d, void *o_g, float *lse, atlas_stream_t stream) {
     if (n_detail > 0 && window_offsets == nullptr) return ATLAS_ERR_NULL;
-    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, 1, n_detail > 0 ? window_offsets
-                                                                            : nullptr,
-                                    n_windows, q_g, k_g, v_g, n_global, heads, head_dim,
-                                    softmax_scale, dtype, o_d, o_g, lse, stream);
+    atlas_attn_layout ly{1, 1, window_offsets, n_windows, nullptr};
+    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, ly, heads,
+                                    head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
+}
+
+ATLAS_API atlas_status atlas_local_global_attn_ex(
+    const void *q_d, const void *k_d, const void *v_d, int64_t n_detail, const void *q_g,
+    const void *k_g, const void *v_g, int64_t n_global, const atlas_attn_layout *layout,
+    int32_t heads, int32_t head_dim, float softmax_scale, atlas_dtype dtype, void *o_d,
+    void *o_g, float *lse, atlas_stream_t stream) {
+    if (!layout) return ATLAS_ERR_NULL;
+    return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, *layout,
+                                    heads, head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
+}
+
+ATLAS_API atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 cube,
+                                                 atlas_grid3 global_grid,
+                                                 atlas_cube3 *global_cube) {
+    if (!global_cube) return ATLAS_ERR_NULL;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1 || global_grid.T < 1 || global_grid.H < 1 ||
+        global_grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1)
+        return ATLAS_ERR_SHAPE;
+    const int64_t E[3] = {grid.T, grid.H, grid.W};
+    const int64_t e[3] = {global_grid.T, global_grid.H, global_grid.W};
+    const int64_t c[3] = {cube.ct, cube.ch, cube.cw};
+    int32_t out[3];
+    for (int i = 0; i < 3; ++i) {
+        if (E[i] % e[i] != 0) return ATLAS_ERR_UNSUPPORTED;
+        const int64_t r = E[i] / e[i];
+        if (c[i] % r != 0) return ATLAS_ERR_UNSUPPORTED;
+        out[i] = static_cast<int32_t>(c[i] / r);
+    }
+    *global_cube = atlas_cube3{out[0], out[1], out[2]};
+    return ATLAS_OK;
 }
 
 ATLAS_API atlas_status atlas_cube_window_offsets(atlas_grid3 grid, atlas_cube3 cube,

@@ -69,6 +69,7 @@ struct PermuteArgs {
     int32_t heads, head_dim, elem_bytes;
     int mode;               // 0 reorder (raster -> cube), 1 unorder, 2 raster RoPE
     const atlas_rope *rope; // may be NULL (pure permutation)
+    int64_t batch = 1;      // problems of this grid stacked along the rows
 };
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
 atlas_status release_rope_tables();
@@ -86,7 +87,11 @@ struct AttnArgs {
     void *o_d, *o_g;
     float *lse;
     const int32_t *win_off = nullptr;  // window offsets (device), NULL: windows of window_len
-    int64_t n_win = 0;
+    int64_t n_win = 0;                 // windows of win_off
+    int64_t batch = 1;                 // problems stacked along the rows; n_detail, n_global
+                                       // and the offsets are per problem
+    const int32_t *gwin_off = nullptr; // per-window global key offsets (device), NULL: all
+    int64_t n_gwin = 0;                // window count (with gwin_off)
 };
 atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
 // One-shot request (atlas_debug_stall_next_attention): true once, for the

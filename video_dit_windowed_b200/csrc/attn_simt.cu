@@ -15,11 +15,13 @@ constexpr int kWarps = 8;
 struct Params {
     const float *q_d, *k_d, *v_d, *q_g, *k_g, *v_g;
     float *o_d, *o_g, *lse;
-    int64_t N, L, G;
+    int64_t N, L, G;         // detail rows, window length, global rows of ONE problem
+    int64_t batch;           // problems stacked along the rows
     int32_t heads;
     float scale;
-    const int32_t *win_off;  // window offsets (NULL: windows of L rows)
+    const int32_t *win_off;  // window offsets over one problem (NULL: windows of L rows)
     int64_t n_win;
+    const int32_t *gwin_off; // global key offsets per window (NULL: every global key)
 };
 
 template <int HD>
@@ -47,15 +49,24 @@ __device__ __forceinline__ void accumulate_keys(const float *k, const float *v, 
     }
 }
 
+// x limited to [lo, hi] (lo <= hi).
+__device__ __forceinline__ int64_t clamp64(int64_t x, int64_t lo, int64_t hi) {
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const Params p) {
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + threadIdx.x / 32;
     const int head = blockIdx.y;
-    if (row >= p.N + p.G) return;
-    const bool detail = row < p.N;
+    const int64_t nd_all = p.batch * p.N;
+    if (row >= nd_all + p.batch * p.G) return;
+    const bool detail = row < nd_all;
+    // Problem b, and the row's index within its problem's detail or global rows.
+    const int64_t b = detail ? row / p.N : (row - nd_all) / p.G;
+    const int64_t local = detail ? row - b * p.N : row - nd_all - b * p.G;
     const int64_t stride = static_cast<int64_t>(p.heads) * HD;
-    const float *qr = (detail ? p.q_d + row * stride : p.q_g + (row - p.N) * stride) + head * HD;
+    const float *qr = (detail ? p.q_d + row * stride : p.q_g + (row - nd_all) * stride) + head * HD;
     float q[HD / 32], o[HD / 32];
 #pragma unroll
     for (int e = 0; e < HD / 32; ++e) {
@@ -63,36 +74,46 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const Params p) 
         o[e] = 0.f;
     }
     float m = -__builtin_huge_valf(), l = 0.f;
+    int64_t g_lo = 0, g_hi = p.G;
     if (detail) {
-        int64_t lo, hi;
+        int64_t lo, hi, w;
         if (p.win_off == nullptr) {
-            lo = (row / p.L) * p.L;
+            w = local / p.L;
+            lo = w * p.L;
             hi = lo + p.L;
-        } else {  // last window whose start is <= row
-            int64_t a = 0, b = p.n_win - 1;
-            while (a < b) {
-                const int64_t mid = (a + b + 1) / 2;
-                if (p.win_off[mid] <= row) a = mid; else b = mid - 1;
+        } else {  // last window whose start is <= local; range clamped to hold it
+            int64_t a = 0, c = p.n_win - 1;
+            while (a < c) {
+                const int64_t mid = (a + c + 1) / 2;
+                if (p.win_off[mid] <= local) a = mid; else c = mid - 1;
             }
-            lo = p.win_off[a];
-            hi = p.win_off[a + 1];
+            w = a;
+            lo = clamp64(p.win_off[a], 0, local);
+            hi = clamp64(p.win_off[a + 1], local + 1, p.N);
         }
-        accumulate_keys<HD>(p.k_d + head * HD, p.v_d + head * HD, lo, hi, stride, q, p.scale,
+        if (p.gwin_off != nullptr) {
+            g_lo = clamp64(p.gwin_off[w], 0, p.G);
+            g_hi = clamp64(p.gwin_off[w + 1], g_lo, p.G);
+        }
+        accumulate_keys<HD>(p.k_d + (b * p.N) * stride + head * HD,
+                            p.v_d + (b * p.N) * stride + head * HD, lo, hi, stride, q, p.scale,
                             m, l, o);
     }
-    if (p.G > 0)
-        accumulate_keys<HD>(p.k_g + head * HD, p.v_g + head * HD, 0, p.G, stride, q, p.scale, m,
-                            l, o);
-    float *out = (detail ? p.o_d + row * stride : p.o_g + (row - p.N) * stride) + head * HD;
+    if (g_hi > g_lo)
+        accumulate_keys<HD>(p.k_g + (b * p.G) * stride + head * HD,
+                            p.v_g + (b * p.G) * stride + head * HD, g_lo, g_hi, stride, q,
+                            p.scale, m, l, o);
+    float *out = (detail ? p.o_d + row * stride : p.o_g + (row - nd_all) * stride) + head * HD;
     const float inv = 1.f / l;
 #pragma unroll
     for (int e = 0; e < HD / 32; ++e) out[lane + 32 * e] = o[e] * inv;
-    if (p.lse != nullptr && lane == 0) p.lse[head * (p.N + p.G) + row] = m + logf(l);
+    if (p.lse != nullptr && lane == 0)
+        p.lse[(b * p.heads + head) * (p.N + p.G) + (detail ? local : p.N + local)] = m + logf(l);
 }
 
 template <int HD>
 atlas_status launch_hd(const Params &p, cudaStream_t stream) {
-    const int64_t rows = p.N + p.G;
+    const int64_t rows = p.batch * (p.N + p.G);
     if (rows == 0) return ATLAS_OK;
     dim3 grid(static_cast<unsigned>((rows + kWarps - 1) / kWarps), static_cast<unsigned>(p.heads));
     attn_simt_kernel<HD><<<grid, kWarps * 32, 0, stream>>>(p);
@@ -119,6 +140,8 @@ atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream) {
     p.scale = a.scale;
     p.win_off = a.win_off;
     p.n_win = a.n_win;
+    p.batch = a.batch;
+    p.gwin_off = a.gwin_off;
     if (a.head_dim == 64) return launch_hd<64>(p, stream);
     if (a.head_dim == 128) return launch_hd<128>(p, stream);
     return ATLAS_ERR_UNSUPPORTED;

@@ -87,15 +87,17 @@ struct Params {
     __nv_bfloat16 *o_d, *o_g;
     float *lse;
     uint32_t *err_word;
-    int32_t N, L, G, heads;
+    int32_t N, L, G, heads;  // N, G: detail and global rows of ONE problem
     float scale_log2;
-    int32_t n_dunits, n_gunits, units_per_head, n_units, n_gtiles;
+    int32_t n_dunits, n_gunits;          // units of one problem
+    int32_t units_per_prob, units_per_head, n_units, n_gtiles;
     int32_t stall_unit;   // test hook: this unit's first K tile is never loaded (-1: off)
-    const int32_t *win_off;  // window offsets [n_win + 1] (NULL: windows of L rows)
+    const int32_t *win_off;   // window offsets [n_win + 1] of one problem (NULL: L rows)
+    const int32_t *gwin_off;  // global key offsets [n_win + 1] per window (NULL: all keys)
     int32_t n_win;
 };
 
-// The window holding detail row x, and its row range [start, end).
+// The window holding detail row x (of one problem).
 __device__ __forceinline__ int32_t window_of(const Params &p, int32_t x) {
     if (p.win_off == nullptr) return x / p.L;
     int32_t lo = 0, hi = p.n_win - 1;
@@ -105,36 +107,62 @@ __device__ __forceinline__ int32_t window_of(const Params &p, int32_t x) {
     }
     return lo;
 }
-__device__ __forceinline__ int32_t window_start(const Params &p, int32_t w) {
-    return p.win_off == nullptr ? w * p.L : __ldg(p.win_off + w);
+// Row range [start, end) of window w, which holds row x. With offsets the
+// range is clamped to [0, N) and to contain x, so that offsets other than
+// described still keep every access in bounds.
+__device__ __forceinline__ int32_t window_start(const Params &p, int32_t w, int32_t x) {
+    return p.win_off == nullptr ? w * p.L : min(max(__ldg(p.win_off + w), 0), x);
 }
-__device__ __forceinline__ int32_t window_end(const Params &p, int32_t w) {
-    return p.win_off == nullptr ? min(p.N, (w + 1) * p.L) : __ldg(p.win_off + w + 1);
+__device__ __forceinline__ int32_t window_end(const Params &p, int32_t w, int32_t x) {
+    return p.win_off == nullptr ? min(p.N, (w + 1) * p.L)
+                                : max(min(__ldg(p.win_off + w + 1), p.N), x + 1);
+}
+// Global keys [start, end) seen by the queries of window w (one problem).
+__device__ __forceinline__ int32_t global_start(const Params &p, int32_t w) {
+    return p.gwin_off == nullptr ? 0 : min(max(__ldg(p.gwin_off + w), 0), p.G);
+}
+__device__ __forceinline__ int32_t global_end(const Params &p, int32_t w, int32_t start) {
+    return p.gwin_off == nullptr ? p.G : min(max(__ldg(p.gwin_off + w + 1), start), p.G);
 }
 
+// Work unit: one head, one problem of the batch, kUnitRows query rows.
+// Rows are per problem (q0, rows); row0 is the problem's first row in the
+// stacked tensors; kw0 / kg0 are absolute first key rows.
 struct Unit {
-    int32_t head, detail, q0, rows, kw0, n_wtiles, n_tiles;
+    int32_t head, detail, b, q0, rows, row0, kw0, n_wtiles, kg0, n_tiles;
 };
 
 __device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
     Unit U;
     U.head = u / p.units_per_head;
     int32_t lu = u - U.head * p.units_per_head;
+    U.b = lu / p.units_per_prob;
+    lu -= U.b * p.units_per_prob;
     U.detail = lu < p.n_dunits;
+    int32_t n_gtiles = p.n_gtiles;
+    U.kg0 = U.b * p.G;
     if (U.detail) {
         U.q0 = lu * kUnitRows;
         U.rows = p.N;
+        U.row0 = U.b * p.N;
         const int32_t q_last = min(U.q0 + kUnitRows, p.N) - 1;
-        U.kw0 = window_start(p, window_of(p, U.q0));
-        const int32_t kw1 = window_end(p, window_of(p, q_last));
+        const int32_t w0 = window_of(p, U.q0), w1 = window_of(p, q_last);
+        U.kw0 = U.row0 + window_start(p, w0, U.q0);
+        const int32_t kw1 = U.row0 + window_end(p, w1, q_last);
         U.n_wtiles = (kw1 - U.kw0 + kBN - 1) / kBN;
+        if (p.gwin_off != nullptr) {
+            const int32_t g0 = global_start(p, w0), g1 = global_end(p, w1, g0);
+            U.kg0 += g0;
+            n_gtiles = (g1 - g0 + kBN - 1) / kBN;
+        }
     } else {
         U.q0 = (lu - p.n_dunits) * kUnitRows;
         U.rows = p.G;
+        U.row0 = U.b * p.G;
         U.kw0 = 0;
         U.n_wtiles = 0;
     }
-    U.n_tiles = U.n_wtiles + p.n_gtiles;
+    U.n_tiles = U.n_wtiles + n_gtiles;
     return U;
 }
 
@@ -161,7 +189,7 @@ __device__ __forceinline__ bool wait_phase(Smem<HD> &sm, uint64_t &bar, uint32_t
 
 // Key tile j of unit U: first row and whether it is a window (detail) tile.
 __device__ __forceinline__ int32_t key_row(const Unit &U, int32_t j) {
-    return j < U.n_wtiles ? U.kw0 + j * kBN : (j - U.n_wtiles) * kBN;
+    return j < U.n_wtiles ? U.kw0 + j * kBN : U.kg0 + (j - U.n_wtiles) * kBN;
 }
 
 // ---------------------------------------------------------------------------
@@ -210,7 +238,7 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 #pragma unroll
             for (int db = 0; db < HD / 64; ++db)
                 ptx::tma_load_3d(ptx::smem_addr(sm.q[i] + db * kBM * 128), tq, bar, db * 64,
-                                 U.head, U.q0 + i * kBM);
+                                 U.head, U.row0 + U.q0 + i * kBM);
         }
         q_armed = unit_iter + 1;
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
@@ -433,11 +461,18 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         const Unit U = decode_unit(p, u);
         const int32_t q = U.q0 + qt * kBM + static_cast<int32_t>(r);
         const bool row_valid = q < U.rows;
-        int32_t lo = 0, hi = p.N;
+        // Allowed keys (absolute rows): detail [lo, hi), global [glo, ghi).
+        int32_t lo = 0, hi = 0, glo = U.b * p.G, ghi = glo + p.G;
         if (U.detail) {
-            const int32_t w = window_of(p, min(q, p.N - 1));
-            lo = window_start(p, w);
-            hi = window_end(p, w);
+            const int32_t qc = min(q, p.N - 1);
+            const int32_t w = window_of(p, qc);
+            lo = U.row0 + window_start(p, w, qc);
+            hi = U.row0 + window_end(p, w, qc);
+            if (p.gwin_off != nullptr) {
+                const int32_t g0 = global_start(p, w);
+                ghi = U.b * p.G + global_end(p, w, g0);
+                glo = U.b * p.G + g0;
+            }
         }
         float m_run = kNegInf, l_run = 0.f;
         for (int32_t j = 0; j < U.n_tiles; ++j, ++cnt) {
@@ -447,8 +482,8 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             ptx::tmem_ld128(t_s, sr);
             // Mask keys outside this row's allowed range.
             const int32_t k0 = key_row(U, j);
-            const int32_t klo = j < U.n_wtiles ? lo : 0;
-            const int32_t khi = j < U.n_wtiles ? hi : p.G;
+            const int32_t klo = j < U.n_wtiles ? lo : glo;
+            const int32_t khi = j < U.n_wtiles ? hi : ghi;
             const bool row_masked = k0 < klo || k0 + kBN > khi;
             if (row_masked) {
 #pragma unroll
@@ -498,7 +533,7 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         __nv_bfloat16 *out = U.detail ? p.o_d : p.o_g;
         uint4 *dst = reinterpret_cast<uint4 *>(
-            out + (static_cast<int64_t>(row_valid ? q : 0) * p.heads + U.head) * HD);
+            out + (static_cast<int64_t>(U.row0 + (row_valid ? q : 0)) * p.heads + U.head) * HD);
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
@@ -521,7 +556,7 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         }
         if (p.lse != nullptr && row_valid) {
             const int64_t col = U.detail ? q : static_cast<int64_t>(p.N) + q;
-            p.lse[static_cast<int64_t>(U.head) * (p.N + p.G) + col] =
+            p.lse[(static_cast<int64_t>(U.b) * p.heads + U.head) * (p.N + p.G) + col] =
                 (m_run + __log2f(l_run)) * 0.69314718055994531f;
         }
         ptx::tc_fence_before();
@@ -635,7 +670,8 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
                *vd = has_d ? a.v_d : a.v_g;
     const void *qg = has_g ? a.q_g : a.q_d, *kg = has_g ? a.k_g : a.k_d,
                *vg = has_g ? a.v_g : a.v_d;
-    const int64_t nd = has_d ? a.n_detail : a.n_global, ng = has_g ? a.n_global : a.n_detail;
+    const int64_t nd = (has_d ? a.n_detail : a.n_global) * a.batch,
+                  ng = (has_g ? a.n_global : a.n_detail) * a.batch;
     if (!make_map(&p.tm_qd, qd, nd, a.heads, HD) || !make_map(&p.tm_kd, kd, nd, a.heads, HD) ||
         !make_map(&p.tm_vd, vd, nd, a.heads, HD) || !make_map(&p.tm_qg, qg, ng, a.heads, HD) ||
         !make_map(&p.tm_kg, kg, ng, a.heads, HD) || !make_map(&p.tm_vg, vg, ng, a.heads, HD))
@@ -652,13 +688,17 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.n_dunits = static_cast<int32_t>((a.n_detail + kUnitRows - 1) / kUnitRows);
     p.n_gunits = static_cast<int32_t>((a.n_global + kUnitRows - 1) / kUnitRows);
-    p.units_per_head = p.n_dunits + p.n_gunits;
+    p.units_per_prob = p.n_dunits + p.n_gunits;
+    if (p.units_per_prob == 0) return ATLAS_OK;
+    if (static_cast<int64_t>(p.units_per_prob) * a.batch * a.heads > INT32_MAX)
+        return ATLAS_ERR_SHAPE;
+    p.units_per_head = p.units_per_prob * static_cast<int32_t>(a.batch);
     p.n_units = p.units_per_head * a.heads;
     p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
     p.stall_unit = take_stall_request() ? 0 : -1;
     p.win_off = a.win_off;
-    p.n_win = static_cast<int32_t>(a.n_win);
-    if (p.n_units == 0) return ATLAS_OK;
+    p.gwin_off = a.gwin_off;
+    p.n_win = static_cast<int32_t>(a.win_off ? a.n_win : a.n_gwin);
     const size_t smem = sizeof(Smem<HD>) + 1024;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;

@@ -57,7 +57,9 @@ struct Geom {
 struct Params {
     const uint8_t *src;
     uint8_t *dst;
-    uint32_t rows;          // tokens
+    uint32_t rows;          // tokens of one problem
+    uint32_t total_rows;    // tokens of all problems (batch * rows)
+    FastDiv by_rows;
     uint32_t row_vecs;      // 16-byte vectors per row
     uint32_t vph;           // 16-byte vectors per head (power of two <= 128)
     uint32_t heads;
@@ -230,7 +232,10 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) 
         }
     }
 
-    for (uint32_t row = blockIdx.x * 2 + group; row < p.rows; row += gridDim.x * 2) {
+    for (uint32_t rr = blockIdx.x * 2 + group; rr < p.total_rows; rr += gridDim.x * 2) {
+        // Problem b of the batch, and the row within it.
+        const uint32_t b = p.by_rows.div(rr);
+        const uint32_t row = rr - b * p.rows;
         uint32_t t = 0, h = 0, w = 0, src_row;
         if (MODE == 0) {
             cube_coords(p.g, row, t, h, w);
@@ -248,8 +253,9 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) 
             raster_coords(p.g, row, t, h, w);
             src_row = row;
         }
-        const uint8_t *s = p.src + static_cast<uint64_t>(src_row) * row_bytes;
-        uint8_t *d = p.dst + static_cast<uint64_t>(row) * row_bytes;
+        const uint8_t *s =
+            p.src + (static_cast<uint64_t>(b) * p.rows + src_row) * row_bytes;
+        uint8_t *d = p.dst + static_cast<uint64_t>(rr) * row_bytes;
 
         if (!ROPE) {
             for (uint32_t v0 = tid; v0 < p.row_vecs; v0 += kGroup * kMaxInFlight) {
@@ -347,7 +353,7 @@ atlas_status rope_table(int device, int64_t T, int64_t H, int64_t W, const atlas
 
 template <int EB, bool ROPE, int MODE>
 atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream) {
-    uint32_t blocks_needed = (p.rows + 1) / 2;
+    uint32_t blocks_needed = (p.total_rows + 1) / 2;
     uint32_t grid = std::min<uint32_t>(blocks_needed, static_cast<uint32_t>(dev.sm_count) * 8u);
     if (grid == 0) return ATLAS_OK;
     permute_rope_kernel<EB, ROPE, MODE><<<grid, kThreads, 0, stream>>>(p);
@@ -421,6 +427,8 @@ void fill_geometry(Params &p, const PermuteArgs &a) {
     p.src = static_cast<const uint8_t *>(a.src);
     p.dst = static_cast<uint8_t *>(a.dst);
     p.rows = static_cast<uint32_t>(a.T * a.H * a.W);
+    p.total_rows = static_cast<uint32_t>(a.batch * a.T * a.H * a.W);
+    p.by_rows = FastDiv(p.rows);
     p.heads = static_cast<uint32_t>(a.heads);
     p.row_vecs = static_cast<uint32_t>(static_cast<int64_t>(a.heads) * a.head_dim *
                                        a.elem_bytes / 16);
@@ -453,33 +461,7 @@ atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream) {
     DeviceInfo dev;
     if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
     Params p{};
-    p.src = static_cast<const uint8_t *>(a.src);
-    p.dst = static_cast<uint8_t *>(a.dst);
-    p.rows = static_cast<uint32_t>(a.T * a.H * a.W);
-    p.heads = static_cast<uint32_t>(a.heads);
-    p.row_vecs = static_cast<uint32_t>(static_cast<int64_t>(a.heads) * a.head_dim *
-                                       a.elem_bytes / 16);
-    p.vph = static_cast<uint32_t>(a.head_dim * a.elem_bytes / 16);
-    Geom &g = p.g;
-    g.T = static_cast<uint32_t>(a.T);
-    g.H = static_cast<uint32_t>(a.H);
-    g.W = static_cast<uint32_t>(a.W);
-    g.ct = static_cast<uint32_t>(a.ct);
-    g.ch = static_cast<uint32_t>(a.ch);
-    g.cw = static_cast<uint32_t>(a.cw);
-    // (cube counts of the divisible path; at least 1 so the dividers stay
-    // defined when a partial cube covers a whole axis)
-    g.cubes_h = std::max(1u, g.H / g.ch);
-    g.cubes_w = std::max(1u, g.W / g.cw);
-    g.L = g.ct * g.ch * g.cw;
-    g.by_W = FastDiv(g.W);
-    g.by_H = FastDiv(g.H);
-    g.by_ct = FastDiv(g.ct);
-    g.by_ch = FastDiv(g.ch);
-    g.by_cw = FastDiv(g.cw);
-    g.by_cubes_w = FastDiv(g.cubes_w);
-    g.by_cubes_h = FastDiv(g.cubes_h);
-    g.by_L = FastDiv(g.L);
+    fill_geometry(p, a);
     const bool rope = a.rope != nullptr;
     if (rope) {
         float2 *tab = nullptr;
