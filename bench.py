@@ -120,64 +120,168 @@ class ClockSampler:
 # the GPU path
 # ---------------------------------------------------------------------------
 class Path:
-    """Device buffers and the seven C-ABI calls of one step."""
+    """Device buffers and the C-ABI calls of one step.
 
-    def __init__(self, w, device, stream):
+    mask "all" (the headline): reorder (+RoPE) detail Q and K, reorder V; RoPE
+      of global Q and K; attention (own window + every global key of the
+      problem); unorder O_d.
+    "aligned": the aligned-proxy-tokens variant. As "all", but global Q, K
+      (+RoPE) and V are reordered by the aligned global cube, each window sees
+      only its aligned global keys, and O_g is unordered too.
+    "raster": naive block attention for comparison. RoPE of detail Q and K
+      in raster order, no reorder; windows of window_len consecutive raster
+      rows (+ every global key); no unorder.
+    "dense": full attention for comparison. RoPE of every Q and K into one
+      buffer of N+G rows, one attention call in which every row sees every row.
+    Windows that the cube does not divide (partial cubes) go through the
+    window-offset form of the attention."""
+
+    def __init__(self, w, device, stream, mask="all", batch=1):
         from video_dit_windowed_b200 import atlas
-        self.atlas = atlas
-        self.w = w
-        self.dev = device
-        self.stream = stream
-        x = make_inputs(w, device=device)
-        self.x = x
+        if mask == "dense" and batch != 1:
+            raise ValueError("--mask dense runs one problem (batch 1)")
+        if mask in ("raster", "dense") and w.partial:
+            raise ValueError(f"--mask {mask} needs a cube that divides the grid")
+        self.atlas, self.w, self.dev, self.stream = atlas, w, device, stream
+        self.mask, self.B = mask, batch
+        self.gcube = None
         self.rd = atlas.make_rope(w.theta, w.split, w.detail_scales)
         self.rg = atlas.make_rope(w.theta, w.split, w.global_scales)
         e = lambda t: torch.empty_like(t)
+        N, G, B = w.n_detail, w.n_global, batch
+        if mask == "dense":
+            # every Q, K and V in one [N+G] buffer, detail rows first
+            shp = (N + G, w.heads, w.head_dim)
+            self.q_all = torch.empty(shp, dtype=w.torch_dtype, device=device)
+            self.k_all, self.v_all = e(self.q_all), e(self.q_all)
+            self.o_all = e(self.q_all)
+            x = make_inputs(w, device=device)
+            self.v_all[:N].copy_(x["v_d"])
+            self.v_all[N:].copy_(x["v_g"])
+            x["v_d"], x["v_g"] = self.v_all[:N], self.v_all[N:]
+            self.x = x
+            self.o_raster, self.o_g = self.o_all[:N], self.o_all[N:]
+            return
+        x = make_inputs(w, device=device, batch=B)
+        self.x = x
         self.q_d, self.k_d, self.v_d = e(x["q_d"]), e(x["k_d"]), e(x["v_d"])
         self.q_g, self.k_g = e(x["q_g"]), e(x["k_g"])
         self.o_d, self.o_g = e(x["q_d"]), e(x["q_g"])
         self.o_raster = e(x["q_d"])
+        self.win = (atlas.cube_window_offsets(w.grid, w.cube).to(device)
+                    if w.partial or mask == "aligned" else None)
+        self.gwin = self.gcube = None
+        if mask == "aligned":
+            self.gcube = atlas.aligned_global_cube(w.grid, w.cube, w.global_grid)
+            self.gwin = atlas.cube_window_offsets(w.global_grid, self.gcube).to(device)
+            self.v_g = e(x["v_g"])
+            self.o_graster = e(x["q_g"])
 
     def step(self, ev=None):
         """One pass; ``ev`` (5 CUDA events) brackets the phases if given."""
-        a, w, s, x = self.atlas, self.w, self.stream, self.x
+        a, w, s, x, B = self.atlas, self.w, self.stream, self.x, self.B
         rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        N, G = w.n_detail, w.n_global
+        if self.mask == "dense":
+            rec(0)
+            if N:
+                a.rope3d(x["q_d"], self.q_all[:N], w.grid, self.rd, stream=s)
+                a.rope3d(x["k_d"], self.k_all[:N], w.grid, self.rd, stream=s)
+            rec(1)
+            a.rope3d(x["q_g"], self.q_all[N:], w.global_grid, self.rg, stream=s)
+            a.rope3d(x["k_g"], self.k_all[N:], w.global_grid, self.rg, stream=s)
+            rec(2)
+            a.local_global_attn(None, None, None, 1, self.q_all, self.k_all, self.v_all, None,
+                                self.o_all, None, stream=s)
+            rec(3)
+            rec(4)
+            return
         rec(0)
-        if w.n_detail:
-            a.cube_reorder(x["q_d"], self.q_d, w.grid, w.cube, self.rd, stream=s)
-            a.cube_reorder(x["k_d"], self.k_d, w.grid, w.cube, self.rd, stream=s)
-            a.cube_reorder(x["v_d"], self.v_d, w.grid, w.cube, None, stream=s)
+        if N:
+            if self.mask == "raster":
+                a.rope3d_batched(x["q_d"], self.q_d, B, w.grid, self.rd, stream=s)
+                a.rope3d_batched(x["k_d"], self.k_d, B, w.grid, self.rd, stream=s)
+            else:
+                a.cube_reorder_batched(x["q_d"], self.q_d, B, w.grid, w.cube, self.rd, stream=s)
+                a.cube_reorder_batched(x["k_d"], self.k_d, B, w.grid, w.cube, self.rd, stream=s)
+                a.cube_reorder_batched(x["v_d"], self.v_d, B, w.grid, w.cube, None, stream=s)
         rec(1)
-        if w.n_global:
-            a.rope3d(x["q_g"], self.q_g, w.global_grid, self.rg, stream=s)
-            a.rope3d(x["k_g"], self.k_g, w.global_grid, self.rg, stream=s)
+        v_g = x["v_g"]
+        if G:
+            if self.mask == "aligned":
+                gg, gc = w.global_grid, self.gcube
+                a.cube_reorder_batched(x["q_g"], self.q_g, B, gg, gc, self.rg, stream=s)
+                a.cube_reorder_batched(x["k_g"], self.k_g, B, gg, gc, self.rg, stream=s)
+                a.cube_reorder_batched(x["v_g"], self.v_g, B, gg, gc, None, stream=s)
+                v_g = self.v_g
+            else:
+                a.rope3d_batched(x["q_g"], self.q_g, B, w.global_grid, self.rg, stream=s)
+                a.rope3d_batched(x["k_g"], self.k_g, B, w.global_grid, self.rg, stream=s)
         rec(2)
-        a.local_global_attn(self.q_d, self.k_d, self.v_d, w.window_len, self.q_g, self.k_g,
-                            x["v_g"], self.o_d, self.o_g, None, stream=s)
+        v_d = x["v_d"] if self.mask == "raster" else self.v_d
+        if B == 1 and self.win is None:
+            a.local_global_attn(self.q_d, self.k_d, v_d, w.window_len, self.q_g, self.k_g, v_g,
+                                self.o_d, self.o_g, None, stream=s)
+        else:
+            a.local_global_attn_ex(self.q_d, self.k_d, v_d, self.q_g, self.k_g, v_g, self.o_d,
+                                   self.o_g, None, batch=B, window_len=w.window_len,
+                                   window_offsets=self.win, global_window_offsets=self.gwin,
+                                   stream=s)
         rec(3)
-        if w.n_detail:
-            a.cube_unorder(self.o_d, self.o_raster, w.grid, w.cube, stream=s)
+        if N and self.mask != "raster":
+            a.cube_unorder_batched(self.o_d, self.o_raster, B, w.grid, w.cube, stream=s)
+        if self.mask == "aligned" and G:
+            a.cube_unorder_batched(self.o_g, self.o_graster, B, w.global_grid, self.gcube,
+                                   stream=s)
         rec(4)
 
+    def outputs(self):
+        """Step results in raster order (the tensors a user reads back)."""
+        if self.mask == "raster":
+            return self.o_d, self.o_g
+        if self.mask == "aligned":
+            return self.o_raster, self.o_graster
+        return self.o_raster, self.o_g
+
     def launches_per_step(self):
+        w, m = self.w, self.mask
+        nd, ng = bool(w.n_detail), bool(w.n_global)
+        if m == "dense":
+            return 2 * nd + 2 + 1
+        if m == "raster":
+            return 2 * nd + 2 * ng + 1
+        if m == "aligned":
+            return 3 * nd + 3 * ng + 1 + nd + ng
+        return 3 * nd + 2 * ng + 1 + nd
+
+    def flops(self):
+        return self.B * self.w.unmasked_flops(self.mask, self.gcube)
+
+    def prep_bytes(self):
+        """Algorithmic bytes of the reorder/RoPE phase: one read and one
+        write of every tensor it touches."""
+        w, m = self.w, self.mask
+        row = w.heads * w.head_dim * w.elem_bytes
+        det = (2 if m in ("raster", "dense") else 3) * w.n_detail
+        glob = (3 if m == "aligned" else 2) * w.n_global
+        return self.B * 2 * (det + glob) * row
+
+    def unorder_bytes(self):
+        w, m = self.w, self.mask
+        row = w.heads * w.head_dim * w.elem_bytes
+        rows = {"all": w.n_detail, "aligned": w.n_detail + w.n_global}.get(m, 0)
+        return self.B * 2 * rows * row
+
+    def attn_bytes(self):
+        """Minimum DRAM bytes of one attention launch: Q, K, V read once, O
+        written once."""
         w = self.w
-        return (3 if w.n_detail else 0) + (2 if w.n_global else 0) + 1 + (1 if w.n_detail else 0)
+        return self.B * 4 * (w.n_detail + w.n_global) * w.heads * w.head_dim * w.elem_bytes
 
     @staticmethod
     def phase_ms(ev):
         return {"reorder": ev[0].elapsed_time(ev[1]), "rope_g": ev[1].elapsed_time(ev[2]),
                 "attn": ev[2].elapsed_time(ev[3]), "unorder": ev[3].elapsed_time(ev[4])}
-
-
-def bytes_reorder_rope(w):
-    row = w.heads * w.head_dim * w.elem_bytes
-    return 2 * 3 * w.n_detail * row, 2 * 2 * w.n_global * row
-
-
-def attn_bytes(w):
-    """Minimum DRAM bytes of one attention launch: Q, K, V read once, O written."""
-    row = w.heads * w.head_dim * w.elem_bytes
-    return (3 * (w.n_detail + w.n_global) + (w.n_detail + w.n_global)) * row
 
 
 def kernel_source_hash():
@@ -291,12 +395,12 @@ def max_over_ranks(v, world):
     return float(t.item())
 
 
-def config_of(w, world):
-    c = {"workload": w.name, "detail_grid": list(w.grid), "cube": list(w.cube),
+def config_of(w, world, mask="all", batch=1):
+    c = {"workload": w.name, "mask": mask, "detail_grid": list(w.grid), "cube": list(w.cube),
          "global_grid": list(w.global_grid), "n_detail": w.n_detail, "window_len": w.window_len,
          "n_global": w.n_global, "heads": w.heads, "head_dim": w.head_dim,
          "rope_split": list(w.split), "detail_scales": list(w.detail_scales),
-         "global_scales": list(w.global_scales), "batch_per_gpu": 1,
+         "global_scales": list(w.global_scales), "batch_per_gpu": batch,
          "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"}
     per_tensor = max(w.n_detail, w.n_global) * w.heads * w.head_dim * w.elem_bytes
     c["l2"] = (f"inputs larger than L2 ({per_tensor / 1e6:.0f} MB per tensor)"
@@ -307,6 +411,9 @@ def config_of(w, world):
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    if args.mask != "all" or args.batch != 1:
+        raise SystemExit("the oracle arm times the method's own mask, one problem per step "
+                         "(--mask all --batch 1)")
     w = workload(args)
     times = []
     # each step a bounded sample: the whole --steps/--warmup run stays near a minute
@@ -344,7 +451,7 @@ def run_atlas(args, world, rank, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
-        path = Path(w, dev, stream)
+        path = Path(w, dev, stream, args.mask, args.batch)
     torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         path.step()
@@ -389,33 +496,32 @@ def run_atlas(args, world, rank, local):
         return
     pk, pk_kind = peaks()
     ms = elapsed / args.steps
-    flops = w.unmasked_flops()
+    flops = path.flops()
     value = world * flops / (ms * 1e-3) / 1e12
     attn_ms = statistics.median(phases["attn"])
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
-    b_d, b_g = bytes_reorder_rope(w)
     rr_ms = statistics.median(phases["reorder"]) + statistics.median(phases["rope_g"])
-    rr_gbs = (b_d + b_g) / (rr_ms * 1e-3) / 1e9 if rr_ms > 0 else None
+    rr_gbs = path.prep_bytes() / (rr_ms * 1e-3) / 1e9 if rr_ms > 0 else None
     un_ms = statistics.median(phases["unorder"])
-    un_bytes = 2 * w.n_detail * w.heads * w.head_dim * w.elem_bytes
-    traffic = measured_traffic(w)
+    un_bytes = path.unorder_bytes()
+    traffic = measured_traffic(w) if (args.mask, args.batch) == ("all", 1) else None
     peak_tf = pk["bf16_tflops_sustained"]
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world),
+        "config": config_of(w, world, args.mask, args.batch),
         "attn_tflops": attn_tf, "attn_ms": attn_ms,
         "attn_frac_of_bf16_peak": {"sustained": attn_tf / pk["bf16_tflops_sustained"],
                                    "burst": attn_tf / pk["bf16_tflops"], "peaks": pk_kind},
         "reorder_rope_gbs": rr_gbs, "reorder_rope_ms": rr_ms,
         "reorder_rope_frac_of_hbm": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
-        "unorder_gbs": un_bytes / (un_ms * 1e-3) / 1e9 if un_ms > 0 else None,
+        "unorder_gbs": un_bytes / (un_ms * 1e-3) / 1e9 if un_ms > 0 and un_bytes else None,
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": attn_tf,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
                      "peak_kind": f"{pk_kind} bf16 sustained",
                      "traffic": traffic,
-                     "algorithmic_bytes": attn_bytes(w)},
+                     "algorithmic_bytes": path.attn_bytes()},
         "roofline_reorder_rope": {"bound": "hbm", "achieved": rr_gbs, "peak": pk["hbm_gbs"],
                                   "unit": "GB/s",
                                   "frac": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
@@ -425,7 +531,7 @@ def run_atlas(args, world, rank, local):
     }
     if e2e:
         out["e2e"] = e2e
-    if not args.no_cpu_baseline and world == 1:
+    if not args.no_cpu_baseline and world == 1 and args.mask == "all":
         tf, cores, sample, _ = time_oracle(w, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
@@ -439,8 +545,9 @@ def run_e2e(path, w, dev, stream, args, world):
             for k, v in path.x.items()}
     for k in host:
         host[k].copy_(path.x[k].cpu())
-    out_d = torch.empty(path.o_raster.shape, dtype=path.o_raster.dtype, pin_memory=True)
-    out_g = torch.empty(path.o_g.shape, dtype=path.o_g.dtype, pin_memory=True)
+    res_d, res_g = path.outputs()
+    out_d = torch.empty(res_d.shape, dtype=res_d.dtype, pin_memory=True)
+    out_g = torch.empty(res_g.shape, dtype=res_g.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_d.numel() * out_d.element_size() + out_g.numel() * out_g.element_size()
 
@@ -449,8 +556,8 @@ def run_e2e(path, w, dev, stream, args, world):
             for k in host:
                 path.x[k].copy_(host[k], non_blocking=True)
             path.step()
-            out_d.copy_(path.o_raster, non_blocking=True)
-            out_g.copy_(path.o_g, non_blocking=True)
+            out_d.copy_(res_d, non_blocking=True)
+            out_g.copy_(res_g, non_blocking=True)
 
     for _ in range(min(args.warmup, 3)):
         one()
@@ -466,7 +573,7 @@ def run_e2e(path, w, dev, stream, args, world):
     torch.cuda.synchronize(dev)
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b) / steps, world)
-    return {"value": world * w.unmasked_flops() / (ms * 1e-3) / 1e12, "unit": UNIT,
+    return {"value": world * path.flops() / (ms * 1e-3) / 1e12, "unit": UNIT,
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps}
 
@@ -481,6 +588,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--mask", default="all", choices=["all", "aligned", "raster", "dense"],
+                    help="all: the method (every global key); aligned: aligned global keys "
+                         "only; raster / dense: comparison modes (naive raster-order blocks, "
+                         "full attention)")
+    ap.add_argument("--batch", type=int, default=1, help="problems per GPU")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of its own "
                          "(smaller cases for profiler captures; reported in config)")

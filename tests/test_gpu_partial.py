@@ -144,3 +144,53 @@ def test_partial_cubes_at_scale_sampled():
                                           f64(v_d[lo:hi, head]), lo, kg, vg, rows,
                                           f64(q_d[lo:hi, head]), n_threads(), win_off=offs)
             assert_attn_close(f64(o_d[lo:hi, head]), ref, "bf16", f"window {w} head {head}")
+
+
+@pytest.mark.parametrize("name", ["8k29", "2k321"])
+def test_long_shapes_full_size_sampled(name):
+    """The 8K / 29-frame and 2K / 321-frame shapes at full size (40 heads,
+    partial cubes) through the window-offset entry the benchmark times:
+    sampled windows (first, smallest, last) and global rows on the first and
+    last head against the oracle; V = 1 gives 1 on every row."""
+    from video_dit_windowed_b200.workloads import WORKLOADS
+    w = WORKLOADS[name]
+    torch.cuda.empty_cache()
+    N, G, heads, hd = w.n_detail, w.n_global, w.heads, w.head_dim
+    mk = lambda rows, s: normal((rows, heads, hd), s, torch.bfloat16, seed=4, device=DEV)
+    q_d, k_d, v_d = mk(N, "q_d"), mk(N, "k_d"), mk(N, "v_d")
+    q_g, k_g, v_g = mk(G, "q_g"), mk(G, "k_g"), mk(G, "v_g")
+    off_h = atlas.cube_window_offsets(w.grid, w.cube)
+    off = off_h.to(DEV)
+    o_d, o_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    lse = torch.empty(heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_windows(q_d, k_d, v_d, off, q_g, k_g, v_g, o_d, o_g, lse)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    offs = off_h.numpy().astype(np.int64)
+    sizes = np.diff(offs)
+    assert sizes.min() < w.window_len and offs.size - 1 == w.n_windows
+    g_rows = np.array([0, 1, G // 2, G - 2, G - 1])
+    for head in (0, heads - 1):
+        kg, vg = f64(k_g[:, head]), f64(v_g[:, head])
+        for win in (0, int(np.argmin(sizes)), len(sizes) - 1):
+            lo, hi = int(offs[win]), int(offs[win + 1])
+            ref, ref_l = orc().attention_head(N, 1, G, hd ** -0.5, f64(k_d[lo:hi, head]),
+                                              f64(v_d[lo:hi, head]), lo, kg, vg,
+                                              np.arange(lo, hi), f64(q_d[lo:hi, head]),
+                                              n_threads(), win_off=offs)
+            assert_attn_close(f64(o_d[lo:hi, head]), ref, "bf16", f"{name} window {win}")
+            assert np.max(np.abs(f64(lse[head, lo:hi]) - ref_l)) <= 5e-3
+        idx = torch.as_tensor(g_rows, device=DEV)
+        ref, _ = orc().attention_head(N, 1, G, hd ** -0.5, None, None, 0, kg, vg, N + g_rows,
+                                      f64(q_g[idx, head]), n_threads(), win_off=offs)
+        assert_attn_close(f64(o_g[idx, head]), ref, "bf16", f"{name} global rows")
+    del o_d, o_g, lse
+    v_d.fill_(1.0)
+    v_g.fill_(1.0)
+    o_d, o_g = torch.empty_like(q_d), torch.empty_like(q_g)
+    atlas.local_global_attn_windows(q_d, k_d, v_d, off, q_g, k_g, v_g, o_d, o_g)
+    torch.cuda.synchronize()
+    for t in (o_d, o_g):
+        assert float((t.float() - 1).abs().max()) <= 8e-3
+    del q_d, k_d, v_d, q_g, k_g, v_g, o_d, o_g
+    torch.cuda.empty_cache()

@@ -55,7 +55,23 @@ class Workload:
 
     @property
     def n_windows(self) -> int:
-        return self.n_detail // self.window_len if self.n_detail else 0
+        if not self.n_detail:
+            return 0
+        n = 1
+        for E, c in zip(self.grid, self.cube):
+            n *= -(-E // c)
+        return n
+
+    @property
+    def partial(self) -> bool:
+        """True when the cube does not divide the grid (variable windows)."""
+        return bool(self.n_detail) and any(E % c for E, c in zip(self.grid, self.cube))
+
+    def extents(self, axis: int, cube=None, grid=None):
+        """Cube extents along one axis (the last one partial if need be)."""
+        E = (grid or self.grid)[axis]
+        c = (cube or self.cube)[axis]
+        return [min(c, E - b * c) for b in range(-(-E // c))]
 
     @property
     def n_global(self) -> int:
@@ -74,11 +90,31 @@ class Workload:
     def elem_bytes(self) -> int:
         return 2 if self.dtype == "bf16" else 4
 
-    def unmasked_flops(self) -> int:
+    def allowed_pairs(self, mask: str = "all", global_cube=None) -> int:
+        """Allowed (query, key) pairs of one problem and one head. mask:
+        "all" (detail: own cube + every global key), "aligned" (own cube +
+        the global cube of ``global_cube`` with the same index), "raster"
+        (windows of window_len consecutive raster rows + every global key),
+        "dense" (every token sees every token)."""
+        N, G = self.n_detail, self.n_global
+        if mask == "dense":
+            return (N + G) ** 2
+        if mask == "raster":
+            return N * self.window_len + N * G + G * G
+        win = 1
+        for a in range(3):
+            win *= sum(e * e for e in self.extents(a)) if N else 0
+        if mask == "all":
+            return win + N * G + G * G
+        cross = 1
+        for a in range(3):
+            cross *= sum(e * g for e, g in zip(self.extents(a),
+                                               self.extents(a, global_cube, self.global_grid)))
+        return win + cross + G * G
+
+    def unmasked_flops(self, mask: str = "all", global_cube=None) -> int:
         """2*D FLOPs for q.k plus 2*D for p*v, per allowed (query, key) pair."""
-        N, L, G = self.n_detail, max(1, self.window_len), self.n_global
-        pairs = N * (L + G) + G * G if N else G * G
-        return 4 * self.head_dim * self.heads * pairs
+        return 4 * self.head_dim * self.heads * self.allowed_pairs(mask, global_cube)
 
     def reorder_rope_bytes(self) -> int:
         """One read and one write of detail Q, K, V plus global Q, K."""
@@ -107,6 +143,19 @@ WORKLOADS = {
         "4k_long", (42, 144, 240), (6, 16, 16), (21, 18, 30), 40, 128, "bf16",
         (44, 42, 42), (2.0, 1.0, 1.0), (4.0, 8.0, 8.0),
         note="1,451,520 detail tokens, 945 windows of 1,536; 11,340 global"),
+    # Lengths the pages report generating (8K 29 frames, 2K 321 frames). Latent
+    # grid: frames (F-1)/4+1, pixels / 16 per side (8x VAE, 2x2 patches); the
+    # cube does not divide every axis, so windows include partial cubes.
+    "8k29": Workload(
+        "8k29", (8, 270, 480), (3, 16, 16), (8, 27, 48), 40, 128, "bf16",
+        (44, 42, 42), (1.0, 1.0, 1.0), (1.0, 10.0, 10.0),
+        note="7680x4320, 29 frames: 1,036,800 detail tokens (partial cubes along t and h); "
+             "10,368 global tokens at ratio 10"),
+    "2k321": Workload(
+        "2k321", (81, 90, 160), (3, 16, 16), (27, 18, 32), 40, 128, "bf16",
+        (44, 42, 42), (1.0, 1.0, 1.0), (3.0, 5.0, 5.0),
+        note="2560x1440, 321 frames: 1,166,400 detail tokens (partial cubes along h); "
+             "15,552 global tokens at ratios 3, 5, 5"),
 }
 
 # The order the workloads are listed in (small CPU-checkable case first).
@@ -138,11 +187,12 @@ def normal(shape, stream, dtype=torch.bfloat16, seed: int = 0, device="cpu",
     return out
 
 
-def make_inputs(w: Workload, device="cpu", pin: bool = False):
-    """Raster-ordered detail Q/K/V [N, heads, D] and global Q/K/V [G, heads, D]."""
+def make_inputs(w: Workload, device="cpu", pin: bool = False, batch: int = 1):
+    """Raster-ordered detail Q/K/V [batch*N, heads, D] and global Q/K/V
+    [batch*G, heads, D] (problems stacked along the rows)."""
     dt = w.torch_dtype
-    shp_d = (w.n_detail, w.heads, w.head_dim)
-    shp_g = (w.n_global, w.heads, w.head_dim)
+    shp_d = (batch * w.n_detail, w.heads, w.head_dim)
+    shp_g = (batch * w.n_global, w.heads, w.head_dim)
     t = {}
     for name, shp in (("q_d", shp_d), ("k_d", shp_d), ("v_d", shp_d),
                       ("q_g", shp_g), ("k_g", shp_g), ("v_g", shp_g)):
