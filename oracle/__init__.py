@@ -70,6 +70,12 @@ def _declare(lib):
     lib.atlas_oracle_attention_head_aligned.argtypes = (
         [_i64] * 10 + [_f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr, _i64, _ptr, _ptr, _ptr, _ptr,
                        ctypes.c_int])
+    lib.atlas_oracle_attention_bwd_head_windows.restype = ctypes.c_int
+    lib.atlas_oracle_attention_bwd_head_windows.argtypes = (
+        [_i64, _i64, _ptr, _i64, _i64, _i64, _f64] + [_ptr] * 7 + [ctypes.c_int])
+    lib.atlas_oracle_attention_bwd_head_aligned.restype = ctypes.c_int
+    lib.atlas_oracle_attention_bwd_head_aligned.argtypes = (
+        [_i64] * 10 + [_f64] + [_ptr] * 7 + [ctypes.c_int])
     lib.atlas_oracle_attention_head.restype = ctypes.c_int
     lib.atlas_oracle_attention_head.argtypes = (
         [_i64, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
@@ -280,6 +286,51 @@ class Oracle:
             o_g[:, h, :] = o[N:]
             lse[h] = l
         return o_d, o_g, lse
+
+    # -- backward -------------------------------------------------------
+    def _bwd(self, call, q_d, k_d, v_d, q_g, k_g, v_g, do_d, do_g):
+        """Stack detail and global rows per head, run ``call`` (the C
+        backward of one head) and split the gradients again."""
+        a = [np.asarray(t, dtype=np.float64) for t in (q_d, k_d, v_d, do_d)]
+        g = [np.asarray(t, dtype=np.float64) for t in (q_g, k_g, v_g, do_g)]
+        N, heads, D = a[0].shape
+        G = g[0].shape[0]
+        out = [np.empty((N, heads, D)) for _ in range(3)] + [np.empty((G, heads, D))
+                                                            for _ in range(3)]
+        for hh in range(heads):
+            q, k, v, do = (np.ascontiguousarray(np.concatenate([x[:, hh], y[:, hh]]))
+                           for x, y in zip(a, g))
+            dq, dk, dv = (np.empty((N + G, D)) for _ in range(3))
+            st = call(D, q.ctypes.data, k.ctypes.data, v.ctypes.data, do.ctypes.data,
+                      dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+            if st != 0:
+                raise RuntimeError(f"oracle backward failed ({st})")
+            for idx, x in enumerate((dq, dk, dv)):
+                out[idx][:, hh] = x[:N]
+                out[3 + idx][:, hh] = x[N:]
+        return tuple(out)
+
+    def attention_bwd_full(self, q_d, k_d, v_d, window_len, q_g, k_g, v_g, do_d, do_g, scale,
+                           n_threads: int = 1, win_off=None):
+        """Gradients (dq_d, dk_d, dv_d, dq_g, dk_g, dv_g) of the attention
+        output contracted with (do_d, do_g); shapes as attention_full."""
+        N = np.asarray(q_d).shape[0]
+        G = np.asarray(q_g).shape[0]
+        if win_off is not None:
+            off = np.ascontiguousarray(np.asarray(win_off, dtype=np.int64))
+            off_ptr, n_win = off.ctypes.data, off.size - 1
+        else:
+            off, off_ptr, n_win = None, None, 0
+        f = lambda D, *p: self.lib.atlas_oracle_attention_bwd_head_windows(
+            N, window_len, off_ptr, n_win, G, D, float(scale), *p, int(n_threads))
+        return self._bwd(f, q_d, k_d, v_d, q_g, k_g, v_g, do_d, do_g)
+
+    def attention_bwd_full_aligned(self, q_d, k_d, v_d, grid, cube, q_g, k_g, v_g, global_grid,
+                                   do_d, do_g, scale, n_threads: int = 1):
+        """Gradients of the aligned variant (layout as attention_full_aligned)."""
+        f = lambda D, *p: self.lib.atlas_oracle_attention_bwd_head_aligned(
+            *grid, *cube, *global_grid, D, float(scale), *p, int(n_threads))
+        return self._bwd(f, q_d, k_d, v_d, q_g, k_g, v_g, do_d, do_g)
 
     def max_threads(self) -> int:
         return int(self.lib.atlas_oracle_max_threads())

@@ -418,6 +418,153 @@ int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
                                                k_g, v_g, n_q, q_ids, q, o, lse, n_threads);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Backward pass (gradients of the attention above; [TS] Methodologie 2      */
+/* trains the attention projections with LoRA, which needs dQ, dK and dV)    */
+/* ------------------------------------------------------------------------ */
+
+/* One head, all N+G rows. q, k, v, dout: [N+G][D], detail rows first (cube
+ * order), then global rows; dout is the gradient of the loss w.r.t. the
+ * attention output o. With P the row softmax of the allowed logits
+ * s_ij = scale*<q_i,k_j>:
+ *   dP_ij = <dout_i, v_j>,  delta_i = sum_j P_ij dP_ij,
+ *   dS_ij = P_ij (dP_ij - delta_i)            (softmax Jacobian),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dout_i.
+ * Pass 1 (over query rows) takes each row's softmax (two passes, as the
+ * forward), delta_i and dq_i; pass 2 (over key rows) visits every query
+ * that is allowed the key and accumulates dk_j and dv_j from the same
+ * definitions. Returns 0, or 2 on allocation failure. */
+static int attention_bwd_core(const struct mask *msk, int64_t n_global, int64_t D,
+                              double scale, const double *q, const double *k,
+                              const double *v, const double *dout, double *dq, double *dk,
+                              double *dv, int n_threads)
+{
+    int64_t R = msk->N + n_global;
+    int status = 0;
+    double *lse = (double *)malloc((size_t)(R > 0 ? R : 1) * sizeof(double));
+    double *delta = (double *)malloc((size_t)(R > 0 ? R : 1) * sizeof(double));
+    if (!lse || !delta) { free(lse); free(delta); return 2; }
+    if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+    for (int64_t i = 0; i < R; ++i) {
+        const double *qi = q + i * D, *gi = dout + i * D;
+        double *logit = (double *)malloc((size_t)R * sizeof(double));
+        double *dp = (double *)malloc((size_t)R * sizeof(double));
+        int64_t *key = (int64_t *)malloc((size_t)R * sizeof(int64_t));
+        if (!logit || !dp || !key) {
+            free(logit); free(dp); free(key);
+#pragma omp atomic write
+            status = 2;
+            continue;
+        }
+        int64_t n = 0;
+        for (int64_t j = 0; j < R; ++j) {
+            if (!allowed(msk, i, j)) continue;
+            double dot = 0.0, dpo = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                dot += qi[d] * k[j * D + d];
+                dpo += gi[d] * v[j * D + d];
+            }
+            logit[n] = scale * dot;
+            dp[n] = dpo;
+            key[n] = j;
+            ++n;
+        }
+        double m = -INFINITY;
+        for (int64_t a = 0; a < n; ++a)
+            if (logit[a] > m) m = logit[a];
+        double sum = 0.0;
+        for (int64_t a = 0; a < n; ++a) sum += exp(logit[a] - m);
+        lse[i] = log(sum) + m;
+        double dl = 0.0;
+        for (int64_t a = 0; a < n; ++a) dl += exp(logit[a] - lse[i]) * dp[a];
+        delta[i] = dl;
+        for (int64_t d = 0; d < D; ++d) dq[i * D + d] = 0.0;
+        for (int64_t a = 0; a < n; ++a) {
+            double ds = exp(logit[a] - lse[i]) * (dp[a] - dl);
+            for (int64_t d = 0; d < D; ++d) dq[i * D + d] += scale * ds * k[key[a] * D + d];
+        }
+        free(logit); free(dp); free(key);
+    }
+    if (status == 0) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+        for (int64_t j = 0; j < R; ++j) {
+            const double *kj = k + j * D, *vj = v + j * D;
+            for (int64_t d = 0; d < D; ++d) { dk[j * D + d] = 0.0; dv[j * D + d] = 0.0; }
+            for (int64_t i = 0; i < R; ++i) {
+                if (!allowed(msk, i, j)) continue;
+                double dot = 0.0, dpo = 0.0;
+                for (int64_t d = 0; d < D; ++d) {
+                    dot += q[i * D + d] * kj[d];
+                    dpo += dout[i * D + d] * vj[d];
+                }
+                double p = exp(scale * dot - lse[i]);
+                double ds = p * (dpo - delta[i]);
+                for (int64_t d = 0; d < D; ++d) {
+                    dk[j * D + d] += scale * ds * q[i * D + d];
+                    dv[j * D + d] += p * dout[i * D + d];
+                }
+            }
+        }
+    }
+    free(lse);
+    free(delta);
+    return status;
+}
+
+/* Backward of one head with windows of window_len rows, or of the ranges
+ * of win_off when not NULL; every global key allowed to detail queries. */
+int atlas_oracle_attention_bwd_head_windows(int64_t n_detail, int64_t window_len,
+                                            const int64_t *win_off, int64_t n_win,
+                                            int64_t n_global, int64_t head_dim, double scale,
+                                            const double *q, const double *k, const double *v,
+                                            const double *dout, double *dq, double *dk,
+                                            double *dv, int n_threads)
+{
+    struct mask m;
+    memset(&m, 0, sizeof m);
+    m.N = n_detail;
+    m.L = window_len;
+    m.win_off = win_off;
+    m.n_win = n_win;
+    return attention_bwd_core(&m, n_global, head_dim, scale, q, k, v, dout, dq, dk, dv,
+                              n_threads);
+}
+
+/* Backward of one head of the aligned variant (geometry as
+ * atlas_oracle_attention_head_aligned). Returns 0, 2 (allocation) or 3. */
+int atlas_oracle_attention_bwd_head_aligned(int64_t T, int64_t H, int64_t W,
+                                            int64_t ct, int64_t ch, int64_t cw,
+                                            int64_t t, int64_t h, int64_t w,
+                                            int64_t head_dim, double scale,
+                                            const double *q, const double *k, const double *v,
+                                            const double *dout, double *dq, double *dk,
+                                            double *dv, int n_threads)
+{
+    struct mask m;
+    memset(&m, 0, sizeof m);
+    m.N = T * H * W;
+    m.aligned = 1;
+    m.T = T; m.H = H; m.W = W;
+    m.ct = ct; m.ch = ch; m.cw = cw;
+    m.t = t; m.h = h; m.w = w;
+    int64_t *cube_of = (int64_t *)malloc((size_t)(m.N > 0 ? m.N : 1) * sizeof(int64_t));
+    if (!cube_of) return 2;
+    int64_t nh = (H + ch - 1) / ch, nw = (W + cw - 1) / cw;
+    for (int64_t r = 0; r < m.N; ++r) {
+        int64_t tt = r / (H * W), hh = (r / W) % H, ww = r % W;
+        int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        if (j < 0 || j >= m.N) { free(cube_of); return 3; }
+        cube_of[j] = ((tt / ct) * nh + hh / ch) * nw + ww / cw;
+    }
+    m.cube_of = cube_of;
+    int st = attention_bwd_core(&m, t * h * w, head_dim, scale, q, k, v, dout, dq, dk, dv,
+                                n_threads);
+    free(cube_of);
+    return st;
+}
+
 /* Number of threads an OpenMP parallel region of this library would use by
  * default (reported beside CPU timings). */
 int atlas_oracle_max_threads(void)

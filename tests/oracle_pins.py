@@ -576,6 +576,113 @@ def pin_attention_aligned_one_cube_sees_all(o):
         assert np.max(np.abs(x - y)) < 1e-12
 
 
+# ---------------------------------------------------------------------------
+# Backward
+# ---------------------------------------------------------------------------
+
+def _autograd_grads(mask, qd, kd, vd, qg, kg, vg, dod, dog, scale):
+    """torch autograd (float64) of dense masked attention, loss = <dO, O>."""
+    ts = [torch.from_numpy(np.concatenate([a, b])).permute(1, 0, 2).clone().requires_grad_(True)
+          for a, b in ((qd, qg), (kd, kg), (vd, vg))]
+    out = torch.nn.functional.scaled_dot_product_attention(
+        *ts, attn_mask=torch.from_numpy(mask), scale=scale)
+    dout = torch.from_numpy(np.concatenate([dod, dog])).permute(1, 0, 2)
+    (out * dout).sum().backward()
+    N = qd.shape[0]
+    grads = [t.grad.permute(1, 0, 2).numpy() for t in ts]
+    return [g[:N] for g in grads] + [g[N:] for g in grads]
+
+
+def pin_bwd_autograd_dense(o):
+    """Gradients equal torch autograd of dense masked attention (explicit
+    boolean masks built from coordinates), for fixed windows, partial cubes
+    and the aligned variant."""
+    cases = []
+    for ci, (grid, cube, G, heads, D) in enumerate(ATTN_CASES[:4]):
+        cases.append(("fixed", grid, cube, G, None, heads, D, geometric_mask(grid, cube, G)))
+    for grid, cube in PARTIAL_CASES[:2]:
+        T, H, W = grid
+        order = lexsort_order(grid, cube)
+        key = np.stack([order // (H * W) // cube[0], (order // W) % H // cube[1],
+                        order % W // cube[2]], -1)
+        N, G = T * H * W, 5
+        m = np.zeros((N + G, N + G), dtype=bool)
+        m[:N, :N] = np.all(key[:, None] == key[None], -1)
+        m[:N, N:] = True
+        m[N:, N:] = True
+        cases.append(("partial", grid, cube, G, None, 2, 8, m))
+    for grid, cube, gg in ALIGNED_CASES[:3]:
+        cases.append(("aligned", grid, cube, gg[0] * gg[1] * gg[2], gg, 2, 8,
+                      aligned_mask(grid, cube, gg)))
+    for ci, (kind, grid, cube, G, gg, heads, D, mask) in enumerate(cases):
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 500 + ci)
+        dod = _rand_case(grid, G, heads, D, 600 + ci)[1]
+        dog = _rand_case(grid, G, heads, D, 700 + ci)[4]
+        if kind == "fixed":
+            got = o.attention_bwd_full(qd, kd, vd, cube[0] * cube[1] * cube[2], qg, kg, vg, dod,
+                                       dog, 0.4)
+        elif kind == "partial":
+            got = o.attention_bwd_full(qd, kd, vd, 1, qg, kg, vg, dod, dog, 0.4,
+                                       win_off=o.cube_windows(grid, cube))
+        else:
+            got = o.attention_bwd_full_aligned(qd, kd, vd, grid, cube, qg, kg, vg, gg, dod, dog,
+                                               0.4)
+        ref = _autograd_grads(mask, qd, kd, vd, qg, kg, vg, dod, dog, 0.4)
+        for name, a, b in zip(("dq_d", "dk_d", "dv_d", "dq_g", "dk_g", "dv_g"), got, ref):
+            assert np.max(np.abs(a - b), initial=0.0) < 1e-11, (kind, grid, name)
+
+
+def pin_bwd_finite_differences(o):
+    """Central differences of <dO, O> through the FORWARD oracle agree with
+    the backward oracle (fixed windows and aligned variant)."""
+    rng = np.random.default_rng(7)
+    for kind in ("fixed", "aligned"):
+        grid, cube, gg = (2, 4, 4), (1, 2, 2), (2, 2, 2)
+        G, heads, D = 8, 1, 4
+        N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 800)
+        dod = rng.standard_normal(qd.shape)
+        dog = rng.standard_normal(qg.shape)
+        scale = 0.45
+
+        def loss(ts):
+            if kind == "fixed":
+                od, og, _ = o.attention_full(ts[0], ts[1], ts[2], 4, ts[3], ts[4], ts[5], scale)
+            else:
+                od, og, _ = o.attention_full_aligned(ts[0], ts[1], ts[2], grid, cube, ts[3],
+                                                     ts[4], ts[5], gg, scale)
+            return float(np.sum(od * dod) + np.sum(og * dog))
+        base = [qd, kd, vd, qg, kg, vg]
+        if kind == "fixed":
+            grads = o.attention_bwd_full(qd, kd, vd, 4, qg, kg, vg, dod, dog, scale)
+        else:
+            grads = o.attention_bwd_full_aligned(qd, kd, vd, grid, cube, qg, kg, vg, gg, dod,
+                                                 dog, scale)
+        order = [0, 1, 2, 3, 4, 5]   # grads come as (dq_d, dk_d, dv_d, dq_g, dk_g, dv_g)
+        h = 1e-6
+        for t_idx, g_idx in zip(order, order):
+            for _ in range(6):
+                idx = tuple(int(rng.integers(0, n)) for n in base[t_idx].shape)
+                plus = [b.copy() for b in base]
+                minus = [b.copy() for b in base]
+                plus[t_idx][idx] += h
+                minus[t_idx][idx] -= h
+                fd = (loss(plus) - loss(minus)) / (2 * h)
+                an = grads[g_idx][idx]
+                assert abs(fd - an) < 1e-7 * max(1.0, abs(an)), (kind, t_idx, idx, fd, an)
+
+
+def pin_bwd_single_token_windows(o):
+    """1x1x1 cubes, G = 0: O = V, so dV = dO exactly and dQ = dK = 0."""
+    grid, heads, D = (2, 3, 4), 2, 8
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, 0, heads, D, 810)
+    dod = _rand_case(grid, 0, heads, D, 811)[1]
+    dqd, dkd, dvd, _, _, _ = o.attention_bwd_full(qd, kd, vd, 1, qg, kg, vg, dod, qg, 0.5)
+    assert np.array_equal(dvd, dod)
+    assert np.max(np.abs(dqd)) < 1e-14 and np.max(np.abs(dkd)) < 1e-14
+
+
+BWD_PINS = [pin_bwd_autograd_dense, pin_bwd_finite_differences, pin_bwd_single_token_windows]
+
 ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
              pin_attention_aligned_dense_sdpa, pin_attention_aligned_counts,
              pin_attention_aligned_one_cube_sees_all,
@@ -584,4 +691,4 @@ ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
              pin_attention_rows_sum_to_one, pin_attention_global_ignores_detail,
              pin_attention_probe_mass, pin_attention_rejects_missing_rows]
 
-ALL_PINS = CUBE_PINS + ROPE_PINS + ATTN_PINS
+ALL_PINS = CUBE_PINS + ROPE_PINS + ATTN_PINS + BWD_PINS
