@@ -136,10 +136,13 @@ class Path:
     Windows that the cube does not divide (partial cubes) go through the
     window-offset form of the attention."""
 
-    def __init__(self, w, device, stream, mask="all", batch=1):
+    def __init__(self, w, device, stream, mask="all", batch=1, backward=False):
         from video_dit_windowed_b200 import atlas
         if mask == "dense" and batch != 1:
             raise ValueError("--mask dense runs one problem (batch 1)")
+        if backward and mask == "dense":
+            raise ValueError("--backward runs the method's masks (all, aligned, raster)")
+        self.backward = backward
         if mask in ("raster", "dense") and w.partial:
             raise ValueError(f"--mask {mask} needs a cube that divides the grid")
         self.atlas, self.w, self.dev, self.stream = atlas, w, device, stream
@@ -176,6 +179,22 @@ class Path:
             self.gwin = atlas.cube_window_offsets(w.global_grid, self.gcube).to(device)
             self.v_g = e(x["v_g"])
             self.o_graster = e(x["q_g"])
+        self.lse = None
+        if backward:
+            # output gradients (raster order, as a user hands them in), the
+            # forward's LSE, the delta workspace, gradients in the
+            # attention's order and in raster order
+            from video_dit_windowed_b200.workloads import normal
+            self.do = {"d": normal(x["q_d"].shape, 0, w.torch_dtype, 1, device),
+                       "g": normal(x["q_g"].shape, 3, w.torch_dtype, 1, device)}
+            self.do_att = {"d": e(x["q_d"]), "g": e(x["q_g"])}
+            self.lse = torch.empty(B, w.heads, N + G, dtype=torch.float32, device=device)
+            self.delta = torch.empty_like(self.lse)
+            names = ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")
+            self.grad = [e(x[n]) for n in names]
+            self.grad_raster = [e(x[n]) for n in names]
+            self.rd_t = atlas.transpose_rope(self.rd)
+            self.rg_t = atlas.transpose_rope(self.rg)
 
     def step(self, ev=None):
         """One pass; ``ev`` (5 CUDA events) brackets the phases if given."""
@@ -221,10 +240,10 @@ class Path:
         v_d = x["v_d"] if self.mask == "raster" else self.v_d
         if B == 1 and self.win is None:
             a.local_global_attn(self.q_d, self.k_d, v_d, w.window_len, self.q_g, self.k_g, v_g,
-                                self.o_d, self.o_g, None, stream=s)
+                                self.o_d, self.o_g, self.lse, stream=s)
         else:
             a.local_global_attn_ex(self.q_d, self.k_d, v_d, self.q_g, self.k_g, v_g, self.o_d,
-                                   self.o_g, None, batch=B, window_len=w.window_len,
+                                   self.o_g, self.lse, batch=B, window_len=w.window_len,
                                    window_offsets=self.win, global_window_offsets=self.gwin,
                                    stream=s)
         rec(3)
@@ -234,6 +253,49 @@ class Path:
             a.cube_unorder_batched(self.o_g, self.o_graster, B, w.global_grid, self.gcube,
                                    stream=s)
         rec(4)
+        if self.backward:
+            self.step_backward(v_d, v_g, ev)
+
+    def step_backward(self, v_d, v_g, ev=None):
+        """Gradients of the step's outputs w.r.t. its raster inputs: dO to the
+        attention's order, the attention backward, then the gradients back
+        to raster order (the transposed RoPE for dQ and dK)."""
+        a, w, s, B = self.atlas, self.w, self.stream, self.B
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        N, G, m = w.n_detail, w.n_global, self.mask
+        gg, gc = w.global_grid, self.gcube
+        do_d, do_g = self.do["d"], self.do["g"]
+        if N and m != "raster":
+            a.cube_reorder_batched(do_d, self.do_att["d"], B, w.grid, w.cube, stream=s)
+            do_d = self.do_att["d"]
+        if G and m == "aligned":
+            a.cube_reorder_batched(do_g, self.do_att["g"], B, gg, gc, stream=s)
+            do_g = self.do_att["g"]
+        rec(5)
+        g = self.grad
+        a.local_global_attn_bwd(self.q_d, self.k_d, v_d, self.o_d, do_d, self.q_g, self.k_g,
+                                v_g, self.o_g, do_g, self.lse, *g, self.delta, batch=B,
+                                window_len=w.window_len, window_offsets=self.win,
+                                global_window_offsets=self.gwin, stream=s)
+        rec(6)
+        r = self.grad_raster
+        if N:
+            if m == "raster":
+                a.rope3d_batched(g[0], r[0], B, w.grid, self.rd_t, stream=s)
+                a.rope3d_batched(g[1], r[1], B, w.grid, self.rd_t, stream=s)
+            else:
+                a.cube_unorder_rope(g[0], r[0], w.grid, w.cube, self.rd_t, B, stream=s)
+                a.cube_unorder_rope(g[1], r[1], w.grid, w.cube, self.rd_t, B, stream=s)
+                a.cube_unorder_batched(g[2], r[2], B, w.grid, w.cube, stream=s)
+        if G:
+            if m == "aligned":
+                a.cube_unorder_rope(g[3], r[3], gg, gc, self.rg_t, B, stream=s)
+                a.cube_unorder_rope(g[4], r[4], gg, gc, self.rg_t, B, stream=s)
+                a.cube_unorder_batched(g[5], r[5], B, gg, gc, stream=s)
+            else:
+                a.rope3d_batched(g[3], r[3], B, gg, self.rg_t, stream=s)
+                a.rope3d_batched(g[4], r[4], B, gg, self.rg_t, stream=s)
+        rec(7)
 
     def outputs(self):
         """Step results in raster order (the tensors a user reads back)."""
@@ -243,16 +305,35 @@ class Path:
             return self.o_raster, self.o_graster
         return self.o_raster, self.o_g
 
+    def gradients(self):
+        """Backward results in raster order (dq_d, dk_d, dv_d, dq_g, dk_g, dv_g)."""
+        g, r, m = self.grad, self.grad_raster, self.mask
+        return [r[0], r[1], g[2] if m == "raster" else r[2], r[3], r[4],
+                r[5] if m == "aligned" else g[5]]
+
     def launches_per_step(self):
         w, m = self.w, self.mask
         nd, ng = bool(w.n_detail), bool(w.n_global)
         if m == "dense":
             return 2 * nd + 2 + 1
         if m == "raster":
-            return 2 * nd + 2 * ng + 1
-        if m == "aligned":
-            return 3 * nd + 3 * ng + 1 + nd + ng
-        return 3 * nd + 2 * ng + 1 + nd
+            fwd = 2 * nd + 2 * ng + 1
+        elif m == "aligned":
+            fwd = 3 * nd + 3 * ng + 1 + nd + ng
+        else:
+            fwd = 3 * nd + 2 * ng + 1 + nd
+        if not self.backward:
+            return fwd
+        # dO reorder(s); delta + dQ + dK/dV kernels; gradients to raster order
+        pre = (nd if m != "raster" else 0) + (ng if m == "aligned" else 0)
+        post = (2 * nd + (nd if m != "raster" else 0)) + (2 * ng + (ng if m == "aligned" else 0))
+        return fwd + pre + 3 + post
+
+    def bwd_flops(self):
+        """Tensor-core FLOPs the backward kernels execute: per allowed pair
+        6*D in the dQ pass (S, dP, dQ) and 8*D in the dK/dV pass (S, dP, dV,
+        dK), i.e. 3.5 times the forward's 4*D."""
+        return self.flops() * 14 // 4
 
     def flops(self):
         return self.B * self.w.unmasked_flops(self.mask, self.gcube)
@@ -280,8 +361,12 @@ class Path:
 
     @staticmethod
     def phase_ms(ev):
-        return {"reorder": ev[0].elapsed_time(ev[1]), "rope_g": ev[1].elapsed_time(ev[2]),
-                "attn": ev[2].elapsed_time(ev[3]), "unorder": ev[3].elapsed_time(ev[4])}
+        d = {"reorder": ev[0].elapsed_time(ev[1]), "rope_g": ev[1].elapsed_time(ev[2]),
+             "attn": ev[2].elapsed_time(ev[3]), "unorder": ev[3].elapsed_time(ev[4])}
+        if len(ev) > 5:
+            d.update({"bwd_pre": ev[4].elapsed_time(ev[5]), "bwd_attn": ev[5].elapsed_time(ev[6]),
+                      "bwd_post": ev[6].elapsed_time(ev[7])})
+        return d
 
 
 def kernel_source_hash():
@@ -395,8 +480,8 @@ def max_over_ranks(v, world):
     return float(t.item())
 
 
-def config_of(w, world, mask="all", batch=1):
-    c = {"workload": w.name, "mask": mask, "detail_grid": list(w.grid), "cube": list(w.cube),
+def config_of(w, world, mask="all", batch=1, backward=False):
+    c = {"workload": w.name, "mask": mask, "pass": "forward+backward" if backward else "forward", "detail_grid": list(w.grid), "cube": list(w.cube),
          "global_grid": list(w.global_grid), "n_detail": w.n_detail, "window_len": w.window_len,
          "n_global": w.n_global, "heads": w.heads, "head_dim": w.head_dim,
          "rope_split": list(w.split), "detail_scales": list(w.detail_scales),
@@ -411,7 +496,7 @@ def config_of(w, world, mask="all", batch=1):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    if args.mask != "all" or args.batch != 1:
+    if args.mask != "all" or args.batch != 1 or args.backward:
         raise SystemExit("the oracle arm times the method's own mask, one problem per step "
                          "(--mask all --batch 1)")
     w = workload(args)
@@ -451,7 +536,7 @@ def run_atlas(args, world, rank, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
-        path = Path(w, dev, stream, args.mask, args.batch)
+        path = Path(w, dev, stream, args.mask, args.batch, args.backward)
     torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         path.step()
@@ -468,7 +553,8 @@ def run_atlas(args, world, rank, local):
     t_wall0 = time.time()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    n_ev = 8 if args.backward else 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     start.record(stream)
     for i in range(args.steps):
         path.step(evs[i])
@@ -478,10 +564,10 @@ def run_atlas(args, world, rank, local):
     barrier(world)
     clk = clocks.stop()
     elapsed = start.elapsed_time(stop)
-    phases = {"reorder": [], "rope_g": [], "attn": [], "unorder": []}
+    phases = {}
     for ev in evs:
         for k, v in Path.phase_ms(ev).items():
-            phases[k].append(v)
+            phases.setdefault(k, []).append(v)
     elapsed = max_over_ranks(elapsed, world)
     code = atlas.last_device_error(stream)
     if code:
@@ -497,7 +583,9 @@ def run_atlas(args, world, rank, local):
     pk, pk_kind = peaks()
     ms = elapsed / args.steps
     flops = path.flops()
-    value = world * flops / (ms * 1e-3) / 1e12
+    # a training step counts the backward at the usual 2.5x the forward
+    step_flops = flops * 7 // 2 if args.backward else flops
+    value = world * step_flops / (ms * 1e-3) / 1e12
     attn_ms = statistics.median(phases["attn"])
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
     rr_ms = statistics.median(phases["reorder"]) + statistics.median(phases["rope_g"])
@@ -510,7 +598,7 @@ def run_atlas(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world, args.mask, args.batch),
+        "config": config_of(w, world, args.mask, args.batch, args.backward),
         "attn_tflops": attn_tf, "attn_ms": attn_ms,
         "attn_frac_of_bf16_peak": {"sustained": attn_tf / pk["bf16_tflops_sustained"],
                                    "burst": attn_tf / pk["bf16_tflops"], "peaks": pk_kind},
@@ -529,9 +617,21 @@ def run_atlas(args, world, rank, local):
         "gpu_launches": path.launches_per_step() * args.steps,
         "clocks": clk,
     }
+    if args.backward:
+        b_ms = statistics.median(phases["bwd_attn"])
+        b_exec = path.bwd_flops() / (b_ms * 1e-3) / 1e12
+        out["backward"] = {
+            "attn_bwd_ms": b_ms, "pre_ms": statistics.median(phases["bwd_pre"]),
+            "post_ms": statistics.median(phases["bwd_post"]),
+            "attn_bwd_tflops_executed": b_exec,
+            "attn_bwd_tflops_model": flops * 5 / 2 / (b_ms * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "attn_bwd_tc_kernel (dQ + dK/dV, with "
+                         "the delta pass in the timed call)", "achieved": b_exec,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": b_exec / peak_tf,
+                         "peak_kind": f"{pk_kind} bf16 sustained"}}
     if e2e:
         out["e2e"] = e2e
-    if not args.no_cpu_baseline and world == 1 and args.mask == "all":
+    if not args.no_cpu_baseline and world == 1 and args.mask == "all" and not args.backward:
         tf, cores, sample, _ = time_oracle(w, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
@@ -541,23 +641,26 @@ def run_atlas(args, world, rank, local):
 def run_e2e(path, w, dev, stream, args, world):
     """Same step, but inputs start in pinned host memory and the outputs end
     there: H2D of the six raster tensors, the seven calls, D2H of O_d and O_g."""
-    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-            for k, v in path.x.items()}
+    dev_in = dict(path.x)
+    if path.backward:
+        dev_in.update({"do_d": path.do["d"], "do_g": path.do["g"]})
+    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in dev_in.items()}
     for k in host:
-        host[k].copy_(path.x[k].cpu())
-    res_d, res_g = path.outputs()
-    out_d = torch.empty(res_d.shape, dtype=res_d.dtype, pin_memory=True)
-    out_g = torch.empty(res_g.shape, dtype=res_g.dtype, pin_memory=True)
+        host[k].copy_(dev_in[k].cpu())
+    res = list(path.outputs())
+    if path.backward:
+        res += path.gradients()
+    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in res]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_d.numel() * out_d.element_size() + out_g.numel() * out_g.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs)
 
     def one():
         with torch.cuda.stream(stream):
             for k in host:
-                path.x[k].copy_(host[k], non_blocking=True)
+                dev_in[k].copy_(host[k], non_blocking=True)
             path.step()
-            out_d.copy_(res_d, non_blocking=True)
-            out_g.copy_(res_g, non_blocking=True)
+            for o, t in zip(outs, res):
+                o.copy_(t, non_blocking=True)
 
     for _ in range(min(args.warmup, 3)):
         one()
@@ -573,7 +676,8 @@ def run_e2e(path, w, dev, stream, args, world):
     torch.cuda.synchronize(dev)
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b) / steps, world)
-    return {"value": world * path.flops() / (ms * 1e-3) / 1e12, "unit": UNIT,
+    step_flops = path.flops() * 7 // 2 if path.backward else path.flops()
+    return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": UNIT,
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps}
 
@@ -593,6 +697,10 @@ def main():
                          "only; raster / dense: comparison modes (naive raster-order blocks, "
                          "full attention)")
     ap.add_argument("--batch", type=int, default=1, help="problems per GPU")
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step: the forward path plus its backward (gradients "
+                         "w.r.t. the raster inputs); value counts the backward as 2.5x the "
+                         "forward FLOPs")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of its own "
                          "(smaller cases for profiler captures; reported in config)")

@@ -303,6 +303,41 @@ atlas_status atlas_local_global_attn_ex(
     atlas_stream_t stream);
 
 /*
+ * atlas_local_global_attn_bwd -- gradients of steps (3) and (4).
+ *
+ * Passages: as atlas_local_global_attn_ex; the pages train the attention
+ * projections with LoRA ("Technische Samenvatting: AtlasVid", Methodologie
+ * 2, training strategy), which needs the gradients of the attention. With P
+ * the row softmax of the allowed logits s = scale*<q,k> and dO the gradient
+ * of the loss w.r.t. the output O:
+ *   delta_i = sum_d dO_id O_id   (= sum_j P_ij <dO_i, v_j>),
+ *   dS_ij = P_ij (<dO_i, v_j> - delta_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dO_i,
+ * over the same allowed pairs as the forward (same layout, windows, batch
+ * and variant). P is recomputed from q, k and the forward's lse.
+ *
+ * q_*, k_*, v_*: the forward's inputs; o_*: its outputs; do_*: gradients
+ * w.r.t. o_* (same shapes and order). lse: the forward's LSE, fp32 [batch,
+ * heads, n_detail + n_global] (required). delta: caller-owned fp32
+ * workspace of the same shape, overwritten with delta_i. dq_*, dk_*, dv_*:
+ * outputs, same shapes and dtype as q_*; they may not overlap any input.
+ * dtype BF16: tcgen05 kernels (P and dS rounded to bf16 before their
+ * products, fp32 accumulation, gradients rounded to bf16 RNE); FP32: SIMT
+ * fp32 kernels. head_dim 64 or 128.
+ * Errors: as atlas_local_global_attn_ex; NULL lse, delta or a required
+ * gradient pointer (NULL); lse or delta not 4-byte aligned (ALIGN).
+ */
+atlas_status atlas_local_global_attn_bwd(
+    const void *q_d, const void *k_d, const void *v_d, const void *o_d,
+    const void *do_d, int64_t n_detail, const void *q_g, const void *k_g,
+    const void *v_g, const void *o_g, const void *do_g, int64_t n_global,
+    const atlas_attn_layout *layout, int32_t heads, int32_t head_dim,
+    float softmax_scale, atlas_dtype dtype, const float *lse, float *delta,
+    void *dq_d, void *dk_d, void *dv_d, void *dq_g, void *dk_g, void *dv_g,
+    atlas_stream_t stream);
+
+/*
  * atlas_aligned_global_cube -- the global-grid cube whose cubes are the
  * aligned sets of the detail cubes (host).
  *
@@ -338,6 +373,21 @@ atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t batch,
                                   atlas_grid3 grid, int32_t heads, int32_t head_dim,
                                   atlas_dtype dtype, const atlas_rope *rope,
                                   atlas_stream_t stream);
+
+/*
+ * atlas_cube_unorder_rope -- cube order -> raster order with each row rotated
+ * by the RoPE of its raster position: dst[r] = R_rope(r) src[pi(r)].
+ *
+ * Passages: as atlas_cube_reorder. Its use is the backward of step (1)+(2):
+ * R is orthogonal and rotating by -phi is its transpose, so with `rope`'s
+ * scales negated this maps the gradient w.r.t. the reordered, rotated
+ * tokens to the gradient w.r.t. the raster inputs of atlas_cube_reorder.
+ * Batch, layout and errors as atlas_cube_unorder_batched; NULL rope (NULL).
+ */
+atlas_status atlas_cube_unorder_rope(const void *src, void *dst, int64_t batch,
+                                     atlas_grid3 grid, atlas_cube3 cube, int32_t heads,
+                                     int32_t head_dim, atlas_dtype dtype,
+                                     const atlas_rope *rope, atlas_stream_t stream);
 
 /* Human-readable name of a status. Never NULL. */
 const char *atlas_status_string(atlas_status status);

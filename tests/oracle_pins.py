@@ -284,7 +284,23 @@ def pin_rope_heads_identical(o):
         assert np.array_equal(y[:, hd], y[:, 0])
 
 
-ROPE_PINS = [pin_rope_literal_angles, pin_rope_zero_scale_identity,
+def pin_rope_negated_scales_transpose(o):
+    """Rotation with negated scales is the inverse and the transpose of the
+    rotation: R(-s) R(s) x = x and <R(s) x, y> = <x, R(-s) y> (what the
+    backward of the reorder with RoPE uses)."""
+    rng = np.random.default_rng(3)
+    grid, split, sc = (3, 4, 5), (4, 6, 6), (2.0, 1.0, 3.0)
+    neg = tuple(-v for v in sc)
+    x = rng.standard_normal((60, 2, 16))
+    y = rng.standard_normal((60, 2, 16))
+    rx = o.rope3d_grid(x, grid, 100.0, split, sc)
+    assert np.max(np.abs(o.rope3d_grid(rx, grid, 100.0, split, neg) - x)) < 1e-13
+    lhs = np.sum(rx * y)
+    rhs = np.sum(x * o.rope3d_grid(y, grid, 100.0, split, neg))
+    assert abs(lhs - rhs) < 1e-11 * max(1.0, abs(lhs))
+
+
+ROPE_PINS = [pin_rope_literal_angles, pin_rope_negated_scales_transpose, pin_rope_zero_scale_identity,
              pin_rope_pair_norms, pin_rope_relative_position,
              pin_rope_temporal_scale, pin_rope_complex_form,
              pin_rope_heads_identical]

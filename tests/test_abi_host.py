@@ -241,3 +241,35 @@ def test_aligned_global_cube_matches_oracle(lib):
             assert np.all(o[:, 1] == 0.0), (grid, w)
             n_in = int(inside.sum())
             assert np.allclose(o[:, 0], n_in / (hi - lo + n_in)), (grid, w)
+
+
+def test_attention_bwd_validation(lib):
+    ins_d = [FAKE + (i << 27) for i in range(5)]          # q, k, v, o, do (detail)
+    ins_g = [FAKE + ((8 + i) << 27) for i in range(5)]    # global
+    grads = [FAKE + ((16 + i) << 27) for i in range(6)]
+    lse, delta = FAKE + (24 << 27), FAKE + (25 << 27)
+    L = atlas.AttnLayout
+
+    def call(ly=L(1, 32, None, 0, None), i_d=None, i_g=None, g=None, lse_=lse, delta_=delta,
+             hd=64):
+        i_d = i_d or ins_d
+        i_g = i_g or ins_g
+        g = g or grads
+        return lib.atlas_local_global_attn_bwd(*i_d, 256, *i_g, 32,
+                                               ctypes.byref(ly) if ly else None, 2, hd, 0.0,
+                                               atlas.BF16, lse_, delta_, *g, None)
+    assert call(ly=None) == atlas.ERR_NULL
+    assert call(lse_=None) == atlas.ERR_NULL
+    assert call(delta_=None) == atlas.ERR_NULL
+    assert call(delta_=delta + 2) == atlas.ERR_ALIGN
+    assert call(hd=96) == atlas.ERR_UNSUPPORTED
+    assert call(i_d=ins_d[:4] + [None]) == atlas.ERR_NULL             # dO_d missing
+    assert call(g=grads[:5] + [None]) == atlas.ERR_NULL               # dv_g missing
+    assert call(g=[grads[0] + 8] + grads[1:]) == atlas.ERR_ALIGN
+    assert call(g=[ins_d[0]] + grads[1:]) == atlas.ERR_ALIAS          # dq_d over q_d
+    assert call(g=grads[:2] + [grads[1]] + grads[3:]) == atlas.ERR_ALIAS   # dv_d over dk_d
+    assert call(delta_=ins_g[4]) == atlas.ERR_ALIAS                   # delta over dO_g
+    assert call(ly=L(1, 30, None, 0, None)) == atlas.ERR_SHAPE
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == atlas.ERR_DEVICE

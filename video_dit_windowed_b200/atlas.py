@@ -88,6 +88,10 @@ def _declare(lib):
     lib.atlas_local_global_attn_ex.argtypes = [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64,
                                                ctypes.POINTER(AttnLayout), _i32, _i32,
                                                ctypes.c_float, ctypes.c_int, _vp, _vp, _vp, _vp]
+    lib.atlas_local_global_attn_bwd.restype = ctypes.c_int
+    lib.atlas_local_global_attn_bwd.argtypes = (
+        [_vp] * 5 + [_i64] + [_vp] * 5 + [_i64, ctypes.POINTER(AttnLayout), _i32, _i32,
+                                         ctypes.c_float, ctypes.c_int, _vp, _vp] + [_vp] * 7)
     lib.atlas_aligned_global_cube.restype = ctypes.c_int
     lib.atlas_aligned_global_cube.argtypes = [Grid3, Cube3, Grid3, ctypes.POINTER(Cube3)]
     lib.atlas_cube_reorder_batched.restype = ctypes.c_int
@@ -96,6 +100,9 @@ def _declare(lib):
     lib.atlas_cube_unorder_batched.restype = ctypes.c_int
     lib.atlas_cube_unorder_batched.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
                                                ctypes.c_int, _vp]
+    lib.atlas_cube_unorder_rope.restype = ctypes.c_int
+    lib.atlas_cube_unorder_rope.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
+                                            ctypes.c_int, ctypes.POINTER(Rope), _vp]
     lib.atlas_rope3d_batched.restype = ctypes.c_int
     lib.atlas_rope3d_batched.argtypes = [_vp, _vp, _i64, Grid3, _i32, _i32, ctypes.c_int,
                                          ctypes.POINTER(Rope), _vp]
@@ -288,6 +295,42 @@ def local_global_attn_ex(q_d, k_d, v_d, q_g, k_g, v_g, o_d, o_g, lse=None, *, ba
     return o_d, o_g, lse
 
 
+def local_global_attn_bwd(q_d, k_d, v_d, o_d, do_d, q_g, k_g, v_g, o_g, do_g, lse,
+                          dq_d, dk_d, dv_d, dq_g, dk_g, dv_g, delta=None, *, batch=1,
+                          window_len=0, window_offsets=None, global_window_offsets=None,
+                          softmax_scale: float = 0.0, stream=None):
+    """Gradients of ``local_global_attn_ex`` (same layout arguments): fills
+    dq_*, dk_*, dv_* from the forward's inputs, outputs ``o_*``, its ``lse``
+    [batch, heads, N+G] and the output gradients ``do_*``. ``delta`` (fp32,
+    shape of lse) is the workspace; allocated here when not given."""
+    import torch
+    ref = q_d if q_d is not None and q_d.shape[0] > 0 else q_g
+    heads, hd = ref.shape[1], ref.shape[2]
+    n_d = (q_d.shape[0] if q_d is not None else 0) // batch
+    n_g = (q_g.shape[0] if q_g is not None else 0) // batch
+    if delta is None:
+        delta = torch.empty_like(lse)
+    nz = lambda t, n: _ptr(t) if (t is not None and n > 0) else None
+    if window_offsets is not None:
+        n_win = window_offsets.numel() - 1
+    elif global_window_offsets is not None:
+        n_win = global_window_offsets.numel() - 1
+    else:
+        n_win = 0
+    wo = _ptr(window_offsets) if window_offsets is not None else None
+    gwo = _ptr(global_window_offsets) if global_window_offsets is not None else None
+    ly = AttnLayout(int(batch), int(window_len), wo.value if wo is not None else None,
+                    int(n_win), gwo.value if gwo is not None else None)
+    st = lib().atlas_local_global_attn_bwd(
+        nz(q_d, n_d), nz(k_d, n_d), nz(v_d, n_d), nz(o_d, n_d), nz(do_d, n_d), n_d,
+        nz(q_g, n_g), nz(k_g, n_g), nz(v_g, n_g), nz(o_g, n_g), nz(do_g, n_g), n_g,
+        ctypes.byref(ly), heads, hd, float(softmax_scale), _dtype_code(ref), _ptr(lse),
+        _ptr(delta), nz(dq_d, n_d), nz(dk_d, n_d), nz(dv_d, n_d), nz(dq_g, n_g),
+        nz(dk_g, n_g), nz(dv_g, n_g), _stream(ref, stream))
+    _check(st, "atlas_local_global_attn_bwd")
+    return dq_d, dk_d, dv_d, dq_g, dk_g, dv_g
+
+
 def aligned_global_cube(grid, cube, global_grid):
     """The global-grid cube whose cubes are the aligned sets of the detail
     cubes (ratios must be integers dividing the cube)."""
@@ -315,6 +358,24 @@ def cube_unorder_batched(src, dst, batch, grid, cube, stream=None):
                                           _stream(src, stream))
     _check(st, "atlas_cube_unorder_batched")
     return dst
+
+
+def cube_unorder_rope(src, dst, grid, cube, rope: Rope, batch=1, stream=None):
+    """Cube -> raster order with each row rotated at its raster position
+    (with negated scales: the gradient of ``cube_reorder`` with RoPE)."""
+    n, heads, hd = src.shape
+    st = lib().atlas_cube_unorder_rope(_ptr(src), _ptr(dst), int(batch), Grid3(*grid),
+                                       Cube3(*cube), heads, hd, _dtype_code(src),
+                                       ctypes.byref(rope), _stream(src, stream))
+    _check(st, "atlas_cube_unorder_rope")
+    return dst
+
+
+def transpose_rope(rope: Rope) -> Rope:
+    """The same RoPE with negated position scales: rotation by -phi, the
+    transpose (and inverse) of ``rope``."""
+    return Rope(rope.theta, rope.d_t, rope.d_h, rope.d_w, -rope.scale_t, -rope.scale_h,
+                -rope.scale_w)
 
 
 def rope3d_batched(src, dst, batch, grid, rope: Rope, stream=None):

@@ -138,14 +138,15 @@ atlas_status reorder(const void *src, void *dst, int64_t batch, atlas_grid3 grid
 
 atlas_status unorder(const void *src, void *dst, int64_t batch, atlas_grid3 grid,
                      atlas_cube3 cube, int32_t heads, int32_t head_dim, atlas_dtype dtype,
-                     atlas_stream_t stream) {
+                     const atlas_rope *rope, atlas_stream_t stream) {
     size_t bytes = 0;
     atlas_status st = check_permute(src, dst, batch, grid, heads, head_dim, dtype, &bytes);
     if (st != ATLAS_OK) return st;
     if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
     if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
     PermuteArgs a{src, dst, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw,
-                  heads, head_dim, elem_bytes(dtype), 1, nullptr, batch};
+                  heads, head_dim, elem_bytes(dtype), 1, rope, batch};
     return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -184,7 +185,7 @@ ATLAS_API atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, at
 ATLAS_API atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, atlas_stream_t stream) {
-    return atlas::unorder(src, dst, 1, grid, cube, heads, head_dim, dtype, stream);
+    return atlas::unorder(src, dst, 1, grid, cube, heads, head_dim, dtype, nullptr, stream);
 }
 
 ATLAS_API atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid, int32_t heads,
@@ -206,7 +207,16 @@ ATLAS_API atlas_status atlas_cube_unorder_batched(const void *src, void *dst, in
                                                   atlas_grid3 grid, atlas_cube3 cube,
                                                   int32_t heads, int32_t head_dim,
                                                   atlas_dtype dtype, atlas_stream_t stream) {
-    return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, stream);
+    return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, nullptr, stream);
+}
+
+ATLAS_API atlas_status atlas_cube_unorder_rope(const void *src, void *dst, int64_t batch,
+                                               atlas_grid3 grid, atlas_cube3 cube,
+                                               int32_t heads, int32_t head_dim,
+                                               atlas_dtype dtype, const atlas_rope *rope,
+                                               atlas_stream_t stream) {
+    if (!rope) return ATLAS_ERR_NULL;
+    return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, rope, stream);
 }
 
 ATLAS_API atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t batch,
@@ -219,14 +229,14 @@ ATLAS_API atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t 
 namespace atlas {
 namespace {
 
-// Shared validation and dispatch of the attention entry points. n_detail
-// and n_global are rows of one problem; see atlas_attn_layout.
-atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d,
-                               int64_t n_detail, const void *q_g, const void *k_g,
-                               const void *v_g, int64_t n_global, const atlas_attn_layout &ly,
-                               int32_t heads, int32_t head_dim, float softmax_scale,
-                               atlas_dtype dtype, void *o_d, void *o_g, float *lse,
-                               atlas_stream_t stream) {
+// Shared validation of the attention entry points: sizes, windows, dtype
+// and the alignment of the six inputs. Fills `a` (outputs left empty);
+// *bd / *bg receive the bytes of one detail / global tensor (all problems).
+atlas_status attn_layout(const void *q_d, const void *k_d, const void *v_d, int64_t n_detail,
+                         const void *q_g, const void *k_g, const void *v_g, int64_t n_global,
+                         const atlas_attn_layout &ly, int32_t heads, int32_t head_dim,
+                         float softmax_scale, atlas_dtype dtype, AttnArgs *a, size_t *bd,
+                         size_t *bg) {
     if (n_detail < 0 || n_global < 0 || heads < 1 || ly.batch < 1) return ATLAS_ERR_SHAPE;
     if (ly.batch > kMaxRows || n_detail > kMaxRows / ly.batch ||
         n_global > kMaxRows / ly.batch || static_cast<int64_t>(heads) > 65535)
@@ -249,35 +259,120 @@ atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d
     } else {
         window_len = 1;
     }
-    if (n_detail > 0 && (!q_d || !k_d || !v_d || !o_d)) return ATLAS_ERR_NULL;
-    if (n_global > 0 && (!q_g || !k_g || !v_g || !o_g)) return ATLAS_ERR_NULL;
+    if (n_detail > 0 && (!q_d || !k_d || !v_d)) return ATLAS_ERR_NULL;
+    if (n_global > 0 && (!q_g || !k_g || !v_g)) return ATLAS_ERR_NULL;
     if (elem_bytes(dtype) == 0) return ATLAS_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return ATLAS_ERR_UNSUPPORTED;
-    const void *ptrs[] = {q_d, k_d, v_d, o_d, q_g, k_g, v_g, o_g};
+    const void *ptrs[] = {q_d, k_d, v_d, q_g, k_g, v_g};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return ATLAS_ERR_ALIGN;
-    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATLAS_ERR_ALIGN;
-    // Outputs must not overlap inputs.
     const size_t eb = static_cast<size_t>(elem_bytes(dtype)) * heads * head_dim;
-    const size_t bd = eb * static_cast<size_t>(n_detail * ly.batch),
-                 bg = eb * static_cast<size_t>(n_global * ly.batch);
-    const void *ins[] = {q_d, k_d, v_d, q_g, k_g, v_g};
-    const size_t in_bytes[] = {bd, bd, bd, bg, bg, bg};
-    for (int i = 0; i < 6; ++i) {
-        if (!ins[i] || !in_bytes[i]) continue;
-        if (o_d && bd && ranges_overlap(ins[i], in_bytes[i], o_d, bd)) return ATLAS_ERR_ALIAS;
-        if (o_g && bg && ranges_overlap(ins[i], in_bytes[i], o_g, bg)) return ATLAS_ERR_ALIAS;
-    }
-    if (o_d && o_g && bd && bg && ranges_overlap(o_d, bd, o_g, bg)) return ATLAS_ERR_ALIAS;
+    *bd = eb * static_cast<size_t>(n_detail * ly.batch);
+    *bg = eb * static_cast<size_t>(n_global * ly.batch);
+    float scale = softmax_scale > 0.f ? softmax_scale
+                                      : 1.f / std::sqrt(static_cast<float>(head_dim));
+    *a = AttnArgs{q_d, k_d, v_d, n_detail, window_len, q_g, k_g, v_g, n_global,
+                  heads, head_dim, scale, nullptr, nullptr, nullptr, win_off,
+                  win_off ? n_win : 0, ly.batch, gwin_off, n_win};
+    return ATLAS_OK;
+}
+
+// A buffer of `bytes` at `p` (NULL or empty: nothing) overlaps none of `n`
+// others.
+struct Span {
+    const void *p;
+    size_t bytes;
+};
+bool overlaps_any(const Span &x, const Span *others, int n) {
+    if (!x.p || !x.bytes) return false;
+    for (int i = 0; i < n; ++i)
+        if (others[i].p && others[i].bytes && &others[i] != &x &&
+            ranges_overlap(x.p, x.bytes, others[i].p, others[i].bytes))
+            return true;
+    return false;
+}
+
+atlas_status local_global_attn(const void *q_d, const void *k_d, const void *v_d,
+                               int64_t n_detail, const void *q_g, const void *k_g,
+                               const void *v_g, int64_t n_global, const atlas_attn_layout &ly,
+                               int32_t heads, int32_t head_dim, float softmax_scale,
+                               atlas_dtype dtype, void *o_d, void *o_g, float *lse,
+                               atlas_stream_t stream) {
+    AttnArgs a;
+    size_t bd = 0, bg = 0;
+    atlas_status st = attn_layout(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, ly, heads,
+                                  head_dim, softmax_scale, dtype, &a, &bd, &bg);
+    if (st != ATLAS_OK) return st;
+    if ((n_detail > 0 && !o_d) || (n_global > 0 && !o_g)) return ATLAS_ERR_NULL;
+    if ((o_d && !aligned16(o_d)) || (o_g && !aligned16(o_g))) return ATLAS_ERR_ALIGN;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATLAS_ERR_ALIGN;
+    // Outputs must not overlap inputs or each other.
+    const Span all[] = {{q_d, bd}, {k_d, bd}, {v_d, bd}, {q_g, bg}, {k_g, bg}, {v_g, bg},
+                        {o_d, bd}, {o_g, bg}};
+    if (overlaps_any(all[6], all, 8) || overlaps_any(all[7], all, 8)) return ATLAS_ERR_ALIAS;
     if (n_detail + n_global == 0) return ATLAS_OK;
     DeviceInfo dev;
     if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
-    float scale = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(head_dim));
-    AttnArgs a{q_d, k_d, v_d, n_detail, window_len, q_g, k_g, v_g, n_global,
-               heads, head_dim, scale, o_d, o_g, lse, win_off, win_off ? n_win : 0,
-               ly.batch, gwin_off, n_win};
+    a.o_d = o_d;
+    a.o_g = o_g;
+    a.lse = lse;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dtype == ATLAS_BF16 ? launch_attn_tc_bf16(a, s) : launch_attn_simt_f32(a, s);
+}
+
+atlas_status local_global_attn_bwd(const void *const in_d[5], int64_t n_detail,
+                                   const void *const in_g[5], int64_t n_global,
+                                   const atlas_attn_layout &ly, int32_t heads, int32_t head_dim,
+                                   float softmax_scale, atlas_dtype dtype, const float *lse,
+                                   float *delta, void *const grad_d[3], void *const grad_g[3],
+                                   atlas_stream_t stream) {
+    // in_*: q, k, v, o, do; grad_*: dq, dk, dv.
+    AttnArgs a;
+    size_t bd = 0, bg = 0;
+    atlas_status st = attn_layout(in_d[0], in_d[1], in_d[2], n_detail, in_g[0], in_g[1],
+                                  in_g[2], n_global, ly, heads, head_dim, softmax_scale, dtype,
+                                  &a, &bd, &bg);
+    if (st != ATLAS_OK) return st;
+    if (!lse || !delta) return ATLAS_ERR_NULL;
+    for (int i = 3; i < 5; ++i) {
+        if ((n_detail > 0 && !in_d[i]) || (n_global > 0 && !in_g[i])) return ATLAS_ERR_NULL;
+        if ((in_d[i] && !aligned16(in_d[i])) || (in_g[i] && !aligned16(in_g[i])))
+            return ATLAS_ERR_ALIGN;
+    }
+    for (int i = 0; i < 3; ++i) {
+        if ((n_detail > 0 && !grad_d[i]) || (n_global > 0 && !grad_g[i])) return ATLAS_ERR_NULL;
+        if ((grad_d[i] && !aligned16(grad_d[i])) || (grad_g[i] && !aligned16(grad_g[i])))
+            return ATLAS_ERR_ALIGN;
+    }
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(delta) & 3u))
+        return ATLAS_ERR_ALIGN;
+    const size_t bl = sizeof(float) * static_cast<size_t>(ly.batch) * heads *
+                      static_cast<size_t>(n_detail + n_global);
+    Span all[17];
+    int n = 0;
+    for (int i = 0; i < 5; ++i) all[n++] = {in_d[i], bd};
+    for (int i = 0; i < 5; ++i) all[n++] = {in_g[i], bg};
+    all[n++] = {lse, bl};
+    all[n++] = {delta, bl};   // index 11
+    for (int i = 0; i < 3; ++i) all[n++] = {grad_d[i], bd};
+    for (int i = 0; i < 2; ++i) all[n++] = {grad_g[i], bg};
+    Span dv_g{grad_g[2], bg};
+    // Written buffers (delta, the gradients) overlap nothing else.
+    for (int i = 11; i < n; ++i)
+        if (overlaps_any(all[i], all, n) || overlaps_any(all[i], &dv_g, 1))
+            return ATLAS_ERR_ALIAS;
+    if (overlaps_any(dv_g, all, n)) return ATLAS_ERR_ALIAS;
+    if (n_detail + n_global == 0) return ATLAS_OK;
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    a.o_d = const_cast<void *>(in_d[3]);
+    a.o_g = const_cast<void *>(in_g[3]);
+    a.lse = const_cast<float *>(lse);
+    AttnBwdArgs b{a, in_d[4], in_g[4], delta, grad_d[0], grad_d[1], grad_d[2],
+                  grad_g[0], grad_g[1], grad_g[2], elem_bytes(dtype)};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = launch_attn_bwd_delta(b, s)) != ATLAS_OK) return st;
+    return dtype == ATLAS_BF16 ? launch_attn_bwd_tc_bf16(b, s) : launch_attn_bwd_simt_f32(b, s);
 }
 
 }  // namespace
@@ -313,6 +408,23 @@ ATLAS_API atlas_status atlas_local_global_attn_ex(
     if (!layout) return ATLAS_ERR_NULL;
     return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, *layout,
                                     heads, head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
+}
+
+ATLAS_API atlas_status atlas_local_global_attn_bwd(
+    const void *q_d, const void *k_d, const void *v_d, const void *o_d, const void *do_d,
+    int64_t n_detail, const void *q_g, const void *k_g, const void *v_g, const void *o_g,
+    const void *do_g, int64_t n_global, const atlas_attn_layout *layout, int32_t heads,
+    int32_t head_dim, float softmax_scale, atlas_dtype dtype, const float *lse, float *delta,
+    void *dq_d, void *dk_d, void *dv_d, void *dq_g, void *dk_g, void *dv_g,
+    atlas_stream_t stream) {
+    if (!layout) return ATLAS_ERR_NULL;
+    const void *in_d[5] = {q_d, k_d, v_d, o_d, do_d};
+    const void *in_g[5] = {q_g, k_g, v_g, o_g, do_g};
+    void *gd[3] = {dq_d, dk_d, dv_d};
+    void *gg[3] = {dq_g, dk_g, dv_g};
+    return atlas::local_global_attn_bwd(in_d, n_detail, in_g, n_global, *layout, heads,
+                                        head_dim, softmax_scale, dtype, lse, delta, gd, gg,
+                                        stream);
 }
 
 ATLAS_API atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 cube,

@@ -4,6 +4,7 @@
 // instructions (mbarrier, TMA, tcgen05) written for this library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -94,9 +95,28 @@ struct AttnArgs {
     int64_t n_gwin = 0;                // window count (with gwin_off)
 };
 atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
+// [rows, heads, hd] bf16 viewed as a 3-D tensor (hd, heads, rows) with a box
+// of 64 channels x 1 head x 128 rows and 128-byte swizzle (defined in
+// attn_tc.cu). False if the driver entry point is missing or encoding fails.
+bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd);
 // One-shot request (atlas_debug_stall_next_attention): true once, for the
 // next bf16 attention launch, which then leaves one K tile unloaded.
 bool take_stall_request();
 atlas_status launch_attn_simt_f32(const AttnArgs &a, cudaStream_t stream);
+
+// Backward: the forward's arguments (fwd.o_d / fwd.o_g hold the forward's
+// outputs O, fwd.lse its LSE; all are inputs here) plus dO, the delta
+// workspace and the gradient outputs.
+struct AttnBwdArgs {
+    AttnArgs fwd;
+    const void *do_d, *do_g;
+    float *delta;
+    void *dq_d, *dk_d, *dv_d, *dq_g, *dk_g, *dv_g;
+    int elem_bytes;
+};
+// delta_i = <dO_i, O_i> for every row and head, into bwd.delta.
+atlas_status launch_attn_bwd_delta(const AttnBwdArgs &a, cudaStream_t stream);
+atlas_status launch_attn_bwd_simt_f32(const AttnBwdArgs &a, cudaStream_t stream);
+atlas_status launch_attn_bwd_tc_bf16(const AttnBwdArgs &a, cudaStream_t stream);
 
 }  // namespace atlas

@@ -1,0 +1,696 @@
+// attn_bwd_tc.cu -- backward of the asymmetric local-global attention, bf16,
+// tcgen05 + TMA + TMEM.
+//
+// Passages: "Technische Samenvatting: AtlasVid", Methodologie 2 (the
+// asymmetric mask; training adapts the attention projections, so the
+// attention's gradients are needed). With P the row softmax of
+// s = scale*<q,k> over the allowed keys, dO the output gradient and
+// delta_i = <dO_i, O_i>:
+//   dS = P o (dO V^T - delta),  dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
+//
+// One kernel template, two forms:
+//   DQ   -- resident: a 128-row tile of Q and of dO; streamed: K and V tiles
+//           of the keys those rows may see (their windows, then the global
+//           keys); accumulates dQ.
+//   DKDV -- resident: a 128-row tile of K and of V; streamed: Q and dO tiles
+//           of the queries that may see those keys (for a detail key, its
+//           window's queries; for a global key, the detail queries that see
+//           it and every global query); accumulates dV and dK.
+// Either way a streamed tile of 128 rows is taken in two halves of 64. For
+// half h the MMA warp computes  S_h = X X'_h^T  and  dP_h = Y Y'_h^T  into
+// tensor memory (X, Y resident, X', Y' streamed: Q/K and dO/V for DQ, K/Q and
+// V/dO for DKDV); the 128 compute threads (one resident row each) turn them
+// into P_h and dS_h, written back as bf16 over the first half of their own
+// columns; the MMA warp then accumulates from tensor memory:
+//   DQ:    dQ += dS_h K_h
+//   DKDV:  dV += P_h dO_h,  dK += dS_h Q_h        (P_h, dS_h transposed here)
+// and issues the next tile's S_h, dP_h behind them. MMAs issued by one thread
+// execute in order, so the next S_h cannot overwrite P_h before it is read,
+// and the compute threads work on one half while the tensor core works on
+// the other. Tensor memory: S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc.
+// Every wait is bounded, as in the forward kernel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "atlas_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace atlas {
+namespace {
+
+constexpr int kRows = 128;            // resident rows per unit = TMEM lanes
+constexpr int kHalf = 64;             // streamed rows per half tile
+constexpr int kCompute = 128;         // compute threads (warps 0-3)
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum Form { kDQ = 0, kDKDV = 1 };
+
+template <int HD>
+struct Smem {
+    static constexpr int kTile = kRows * HD * 2;                  // one 128-row bf16 tile
+    static constexpr int kStages = (160 * 1024) / (2 * kTile);    // streamed (X', Y') pairs
+    alignas(1024) uint8_t x[kTile];                              // resident X (Q or K)
+    alignas(1024) uint8_t y[kTile];                              // resident Y (dO or V)
+    alignas(1024) uint8_t xs[kStages][kTile];                    // streamed X' (K or Q)
+    alignas(1024) uint8_t ys[kStages][kTile];                    // streamed Y' (V or dO)
+    float lse2[kStages][kRows];   // DKDV: log2-scaled LSE of the streamed queries
+    float delta[kStages][kRows];  // DKDV: delta of the streamed queries
+    uint64_t x_full, x_empty;
+    uint64_t st_full[kStages], st_empty[kStages];
+    uint64_t s_full[2], p_full[2];
+    uint64_t acc_full, acc_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    volatile int abort;
+    uint32_t *err_word;
+};
+
+struct Params {
+    CUtensorMap tm_q[2], tm_k[2], tm_v[2], tm_do[2];   // [0] detail, [1] global
+    __nv_bfloat16 *out0[2], *out1[2];   // DQ: dq (out0); DKDV: dv (out0), dk (out1)
+    const float *lse, *delta;
+    uint32_t *err_word;
+    int32_t N, L, G, heads, batch;      // N, G: rows of ONE problem
+    float scale_log2, scale;
+    const int32_t *win_off, *gwin_off;
+    int32_t n_win;
+    int32_t tiles_d, tiles_g;           // 128-row tiles of one problem's detail / global rows
+    int32_t n_long;                     // DKDV: units over global keys (scheduled first)
+    int32_t n_units;
+};
+
+// ---- window geometry (per problem; as the forward) --------------------------
+__device__ __forceinline__ int32_t window_of(const Params &p, int32_t x) {
+    if (p.win_off == nullptr) return x / p.L;
+    int32_t lo = 0, hi = p.n_win - 1;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.win_off + mid) <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+__device__ __forceinline__ int32_t window_start(const Params &p, int32_t w, int32_t x) {
+    return p.win_off == nullptr ? w * p.L : min(max(__ldg(p.win_off + w), 0), x);
+}
+__device__ __forceinline__ int32_t window_end(const Params &p, int32_t w, int32_t x) {
+    return p.win_off == nullptr ? min(p.N, (w + 1) * p.L)
+                                : max(min(__ldg(p.win_off + w + 1), p.N), x + 1);
+}
+// Rows of window w without a row to hold (the aligned lookup from a key).
+__device__ __forceinline__ void window_rows(const Params &p, int32_t w, int32_t &lo,
+                                            int32_t &hi) {
+    if (p.win_off == nullptr) {
+        lo = w * p.L;
+        hi = min(p.N, lo + p.L);
+    } else {
+        lo = min(max(__ldg(p.win_off + w), 0), p.N);
+        hi = min(max(__ldg(p.win_off + w + 1), lo), p.N);
+    }
+}
+__device__ __forceinline__ int32_t global_start(const Params &p, int32_t w) {
+    return p.gwin_off == nullptr ? 0 : min(max(__ldg(p.gwin_off + w), 0), p.G);
+}
+__device__ __forceinline__ int32_t global_end(const Params &p, int32_t w, int32_t start) {
+    return p.gwin_off == nullptr ? p.G : min(max(__ldg(p.gwin_off + w + 1), start), p.G);
+}
+// Aligned variant: the window whose global range holds global row g (-1:
+// none).
+__device__ __forceinline__ int32_t window_of_global(const Params &p, int32_t g) {
+    int32_t lo = 0, hi = p.n_win - 1;
+    while (lo < hi) {
+        const int32_t mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.gwin_off + mid) <= g) lo = mid; else hi = mid - 1;
+    }
+    const int32_t s = global_start(p, lo);
+    return (s <= g && g < global_end(p, lo, s)) ? lo : -1;
+}
+
+// A work unit: one head, one problem, 128 resident rows, and the streamed
+// tiles: n_a tiles of detail rows from row a0, then n_b tiles of global rows
+// from row b0 (rows within the problem).
+struct Unit {
+    int32_t head, b, detail, r0, rows, a0, n_a, b0, n_b;
+};
+
+template <int FORM>
+__device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
+    Unit U;
+    const int32_t per_prob = p.tiles_d + p.tiles_g;
+    if (FORM == kDQ) {
+        U.head = u / (per_prob * p.batch);
+        int32_t lu = u - U.head * per_prob * p.batch;
+        U.b = lu / per_prob;
+        lu -= U.b * per_prob;
+        U.detail = lu < p.tiles_d;
+        U.r0 = (U.detail ? lu : lu - p.tiles_d) * kRows;
+        U.rows = U.detail ? p.N : p.G;
+        U.n_a = 0;
+        U.a0 = 0;
+        int32_t g0 = 0, g1 = p.G;
+        if (U.detail) {
+            const int32_t last = min(U.r0 + kRows, p.N) - 1;
+            const int32_t w0 = window_of(p, U.r0), w1 = window_of(p, last);
+            U.a0 = window_start(p, w0, U.r0);
+            U.n_a = (window_end(p, w1, last) - U.a0 + kRows - 1) / kRows;
+            if (p.gwin_off != nullptr) {
+                g0 = global_start(p, w0);
+                g1 = max(global_end(p, w1, g0), g0);
+            }
+        }
+        U.b0 = g0;
+        U.n_b = (g1 - g0 + kRows - 1) / kRows;
+    } else {
+        // global-key units first (they stream every query that sees them)
+        const bool long_unit = u < p.n_long;
+        const int32_t span = long_unit ? p.tiles_g : p.tiles_d;
+        const int32_t v = long_unit ? u : u - p.n_long;
+        U.head = v / (span * p.batch);
+        int32_t lv = v - U.head * span * p.batch;
+        U.b = lv / span;
+        lv -= U.b * span;
+        U.detail = !long_unit;
+        U.r0 = lv * kRows;
+        U.rows = U.detail ? p.N : p.G;
+        const int32_t last = min(U.r0 + kRows, U.rows) - 1;
+        if (U.detail) {
+            const int32_t w0 = window_of(p, U.r0), w1 = window_of(p, last);
+            U.a0 = window_start(p, w0, U.r0);
+            U.n_a = (window_end(p, w1, last) - U.a0 + kRows - 1) / kRows;
+            U.b0 = 0;
+            U.n_b = 0;
+        } else {
+            int32_t q0 = 0, q1 = p.N;
+            if (p.gwin_off != nullptr && p.N > 0) {
+                // windows whose global ranges hold the first and last key
+                int32_t wa = -1, wb = -1;
+                for (int32_t g = U.r0; g <= last && wa < 0; ++g) wa = window_of_global(p, g);
+                for (int32_t g = last; g >= U.r0 && wb < 0; --g) wb = window_of_global(p, g);
+                if (wa < 0) {
+                    q0 = q1 = 0;
+                } else {
+                    int32_t lo, hi;
+                    window_rows(p, wa, q0, hi);
+                    window_rows(p, wb, lo, q1);
+                    q1 = max(q1, q0);
+                }
+            }
+            U.a0 = q0;
+            U.n_a = (q1 - q0 + kRows - 1) / kRows;
+            U.b0 = 0;
+            U.n_b = p.tiles_g;
+        }
+    }
+    return U;
+}
+
+// Bounded wait (as the forward): false after flagging `err` when the phase
+// did not complete within the limit, or when another role aborted.
+template <int HD>
+__device__ __forceinline__ bool wait_phase(Smem<HD> &sm, uint64_t &bar, uint32_t parity,
+                                           uint32_t err, bool honor_abort = true) {
+    const uint32_t a = ptx::smem_addr(&bar);
+    if (ptx::mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ptx::mbar_try_wait(a, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (honor_abort && sm.abort) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(sm.err_word, err);
+                sm.abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Streamed tile j of unit U: detail rows (true) or global rows, and its first
+// row within the problem.
+__device__ __forceinline__ bool streamed_detail(const Unit &U, int32_t j) { return j < U.n_a; }
+__device__ __forceinline__ int32_t streamed_row(const Unit &U, int32_t j) {
+    return j < U.n_a ? U.a0 + j * kRows : U.b0 + (j - U.n_a) * kRows;
+}
+
+// ---------------------------------------------------------------------------
+// Producer warp: resident X, Y once per unit; then (X', Y') pairs into the
+// stage ring, with (DKDV) the streamed queries' LSE and delta.
+// ---------------------------------------------------------------------------
+template <int HD, int FORM>
+__device__ void producer(const Params &p, Smem<HD> &sm) {
+    constexpr int kStages = Smem<HD>::kStages;
+    constexpr uint32_t kTile = Smem<HD>::kTile;
+    const uint32_t lane = threadIdx.x & 31;
+    uint32_t it = 0, unit_iter = 0, x_armed = 0;
+    uint32_t armed[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) armed[s] = 0;
+    bool ok = true;
+    auto tile = [&](uint8_t *dst, const CUtensorMap *map, uint32_t bar, int32_t head,
+                    int32_t row) {
+#pragma unroll
+        for (int db = 0; db < HD / 64; ++db)
+            ptx::tma_load_3d(ptx::smem_addr(dst + db * kRows * 128), map, bar, db * 64, head,
+                             row);
+    };
+    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit<FORM>(p, u);
+        // Every lane waits and the warp agrees, so the lanes never diverge
+        // around the warp-wide steps below.
+        if (unit_iter > 0 &&
+            !(ok = __all_sync(0xffffffffu, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
+                                                      kErrTimeoutProducer))))
+            break;
+        const int side = U.detail ? 0 : 1;
+        const int32_t rbase = U.b * (U.detail ? p.N : p.G);
+        if (lane == 0) {
+            const uint32_t bar = ptx::smem_addr(&sm.x_full);
+            ptx::mbar_arrive_expect_tx(bar, 2 * kTile);
+            tile(sm.x, FORM == kDQ ? &p.tm_q[side] : &p.tm_k[side], bar, U.head, rbase + U.r0);
+            tile(sm.y, FORM == kDQ ? &p.tm_do[side] : &p.tm_v[side], bar, U.head, rbase + U.r0);
+        }
+        x_armed = unit_iter + 1;
+        const int32_t n = U.n_a + U.n_b;
+        for (int32_t j = 0; j < n && ok; ++j, ++it) {
+            const uint32_t s = it % kStages, round = it / kStages;
+            if (round > 0 &&
+                !(ok = __all_sync(0xffffffffu, wait_phase(sm, sm.st_empty[s], (round - 1) & 1,
+                                                          kErrTimeoutProducer))))
+                break;
+            const bool det = streamed_detail(U, j);
+            const int32_t row = streamed_row(U, j);
+            const int sside = det ? 0 : 1;
+            if (FORM == kDKDV) {
+                // LSE (log2 units) and delta of the 128 streamed queries; rows
+                // past the problem get +inf (P = 0) and 0.
+                const int32_t nrows = det ? p.N : p.G;
+                const int64_t col0 = (static_cast<int64_t>(U.b) * p.heads + U.head) *
+                                         (p.N + p.G) + (det ? 0 : p.N);
+#pragma unroll
+                for (int i = 0; i < kRows / 32; ++i) {
+                    const int32_t c = i * 32 + lane, q = row + c;
+                    const bool valid = q < nrows;
+                    sm.lse2[s][c] = valid ? __ldg(p.lse + col0 + q) * kLog2e
+                                          : __builtin_huge_valf();
+                    sm.delta[s][c] = valid ? __ldg(p.delta + col0 + q) : 0.f;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                const uint32_t bar = ptx::smem_addr(&sm.st_full[s]);
+                ptx::mbar_arrive_expect_tx(bar, 2 * kTile);
+                const int32_t srow = (det ? U.b * p.N : U.b * p.G) + row;
+                tile(sm.xs[s], FORM == kDQ ? &p.tm_k[sside] : &p.tm_q[sside], bar, U.head, srow);
+                tile(sm.ys[s], FORM == kDQ ? &p.tm_v[sside] : &p.tm_do[sside], bar, U.head,
+                     srow);
+            }
+#pragma unroll
+            for (int t = 0; t < kStages; ++t)
+                if (t == static_cast<int>(s)) armed[t] = round + 1;
+        }
+    }
+    if (!ok && lane == 0) {
+        // Let every copy already issued land before the CTA can exit.
+        if (x_armed) wait_phase(sm, sm.x_full, (x_armed - 1) & 1, kErrTimeoutTeardown, false);
+        for (int t = 0; t < kStages; ++t)
+            if (armed[t])
+                wait_phase(sm, sm.st_full[t], (armed[t] - 1) & 1, kErrTimeoutTeardown, false);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one thread).
+// ---------------------------------------------------------------------------
+template <int HD, int FORM>
+__device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+    constexpr int kStages = Smem<HD>::kStages;
+    constexpr uint32_t kT16 = Smem<HD>::kTile >> 4;
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kRows, kHalf, 0);   // S_h, dP_h
+    constexpr uint32_t kIdAcc = ptx::idesc_bf16_f32(kRows, HD, 1);    // acc += A(tmem) B
+    constexpr uint32_t kHi = ptx::desc_sw128_hi(1024);
+    const uint32_t x_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.x), 16);
+    const uint32_t y_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.y), 16);
+    const uint32_t xs_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), 16);
+    const uint32_t ys_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), 16);
+    // The same streamed tiles as MN-major B operands of the accumulation.
+    const uint32_t xs_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), kRows * 128);
+    const uint32_t ys_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), kRows * 128);
+    const uint32_t t_s = tmem, t_dp = tmem + 2 * kHalf, t_acc = tmem + 4 * kHalf;
+    uint32_t it = 0, unit_iter = 0, p_cnt = 0;
+    bool ok = true;
+
+    // S_h = X X'_h^T and dP_h = Y Y'_h^T from stage s; then a commit.
+    auto issue_sdp = [&](int h, uint32_t s) {
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint32_t a_off = ((ks / 4) * (kRows * 128) + (ks % 4) * 32) >> 4;
+            const uint32_t b_off = a_off + ((h * kHalf * 128) >> 4);
+            ptx::mma_ss(t_s + h * kHalf, ptx::desc_join(x_lo + a_off, kHi),
+                        ptx::desc_join(xs_lo + s * kT16 + b_off, kHi), kIdS, ks > 0);
+            ptx::mma_ss(t_dp + h * kHalf, ptx::desc_join(y_lo + a_off, kHi),
+                        ptx::desc_join(ys_lo + s * kT16 + b_off, kHi), kIdS, ks > 0);
+        }
+        ptx::mma_commit(ptx::smem_addr(&sm.s_full[h]));
+    };
+    // acc += A_h (tensor memory, 64 streamed rows packed in 32 columns) times
+    // the streamed tile's half h as an MN-major B operand.
+    auto issue_acc = [&](uint32_t d, uint32_t a, uint32_t b_lo, int h, uint32_t s,
+                         bool first) {
+#pragma unroll
+        for (int ks = 0; ks < kHalf / 16; ++ks) {
+            const uint32_t off = s * kT16 + ((h * kHalf * 128 + ks * 16 * 128) >> 4);
+            ptx::mma_ts(d, a + ks * 8, ptx::desc_join(b_lo + off, kHi), kIdAcc,
+                        (first && ks == 0) ? 0u : 1u);
+        }
+    };
+    auto next_stage = [&](uint32_t &s) -> bool {
+        s = it % kStages;
+        const bool r = wait_phase(sm, sm.st_full[s], (it / kStages) & 1, kErrTimeoutMma);
+        ++it;
+        ptx::tc_fence_after();
+        return r;
+    };
+
+    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit<FORM>(p, u);
+        const int32_t n = U.n_a + U.n_b;
+        if (!(ok = wait_phase(sm, sm.x_full, unit_iter & 1, kErrTimeoutMma))) break;
+        ptx::tc_fence_after();
+        uint32_t s_cur, s_next = 0;
+        if (!(ok = next_stage(s_cur))) break;
+        issue_sdp(0, s_cur);
+        issue_sdp(1, s_cur);
+        for (int32_t j = 0; j < n && ok; ++j) {
+            const bool more = j + 1 < n;
+            for (int h = 0; h < 2 && ok; ++h) {
+                if (!(ok = wait_phase(sm, sm.p_full[h], p_cnt & 1, kErrTimeoutMma))) break;
+                if (j == 0 && h == 0 && unit_iter > 0 &&
+                    !(ok = wait_phase(sm, sm.acc_empty, (unit_iter - 1) & 1, kErrTimeoutMma)))
+                    break;
+                ptx::tc_fence_after();
+                const bool first = j == 0 && h == 0;
+                if (FORM == kDQ) {
+                    issue_acc(t_acc, t_dp + h * kHalf, xs_mn, h, s_cur, first);     // dQ
+                } else {
+                    issue_acc(t_acc, t_s + h * kHalf, ys_mn, h, s_cur, first);      // dV
+                    issue_acc(t_acc + HD, t_dp + h * kHalf, xs_mn, h, s_cur, first); // dK
+                }
+                if (h == 1) ptx::mma_commit(ptx::smem_addr(&sm.st_empty[s_cur]));
+                if (more) {
+                    if (h == 0 && !(ok = next_stage(s_next))) break;
+                    issue_sdp(h, s_next);
+                }
+            }
+            ++p_cnt;
+            s_cur = s_next;
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_addr(&sm.acc_full));
+        ptx::mma_commit(ptx::smem_addr(&sm.x_empty));
+    }
+    // Drain: every MMA issued must finish before tensor memory is freed.
+    ptx::mma_commit(ptx::smem_addr(&sm.drain));
+    wait_phase(sm, sm.drain, 0, kErrTimeoutTeardown, false);
+}
+
+// ---------------------------------------------------------------------------
+// Compute warps: thread = resident row = tensor-memory lane.
+// ---------------------------------------------------------------------------
+template <int HD, int FORM>
+__device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+    constexpr int kStages = Smem<HD>::kStages;
+    constexpr uint32_t kAll = 0xffffffffu;
+    const uint32_t warp = threadIdx.x / 32, r = threadIdx.x & 127;
+    const uint32_t lane_sel = (warp * 32u) << 16;
+    const uint32_t t_s = tmem + lane_sel, t_dp = tmem + 2 * kHalf + lane_sel;
+    const uint32_t t_acc = tmem + 4 * kHalf + lane_sel;
+    const float c2 = p.scale_log2;
+    uint32_t cnt = 0, unit_iter = 0;
+
+    for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
+        const Unit U = decode_unit<FORM>(p, u);
+        const int32_t row = U.r0 + static_cast<int32_t>(r);   // resident row (in problem)
+        const bool valid = row < U.rows;
+        // Allowed streamed rows: [da, db) of detail tiles, [ga, gb) of global tiles.
+        int32_t da = 0, db = 0, ga = 0, gb = 0;
+        float lse2_own = 0.f, delta_own = 0.f;
+        if (valid) {
+            if (FORM == kDQ) {
+                ga = 0;
+                gb = p.G;
+                if (U.detail) {
+                    const int32_t w = window_of(p, row);
+                    da = window_start(p, w, row);
+                    db = window_end(p, w, row);
+                    ga = global_start(p, w);
+                    gb = global_end(p, w, ga);
+                }
+                const int64_t col = (static_cast<int64_t>(U.b) * p.heads + U.head) *
+                                        (p.N + p.G) + (U.detail ? row : p.N + row);
+                lse2_own = __ldg(p.lse + col) * kLog2e;
+                delta_own = __ldg(p.delta + col);
+            } else if (U.detail) {
+                const int32_t w = window_of(p, row);
+                da = window_start(p, w, row);
+                db = window_end(p, w, row);
+            } else {
+                db = p.N;
+                if (p.gwin_off != nullptr) {
+                    const int32_t w = window_of_global(p, row);
+                    if (w < 0) db = 0; else window_rows(p, w, da, db);
+                }
+                gb = p.G;
+            }
+        } else if (FORM == kDQ) {
+            lse2_own = __builtin_huge_valf();
+        }
+        const int32_t n = U.n_a + U.n_b;
+        for (int32_t j = 0; j < n; ++j, ++cnt) {
+            const bool det = streamed_detail(U, j);
+            const int32_t base = streamed_row(U, j);
+            const int32_t lo = det ? da : ga, hi = det ? db : gb;
+            const uint32_t stage = cnt % kStages;
+            if (FORM == kDKDV &&
+                !__all_sync(kAll, wait_phase(sm, sm.st_full[stage], (cnt / kStages) & 1,
+                                             kErrTimeoutSoftmax)))
+                return;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                if (!__all_sync(kAll, wait_phase(sm, sm.s_full[h], cnt & 1, kErrTimeoutSoftmax)))
+                    return;
+                ptx::tc_fence_after();
+                uint32_t sv[kHalf], dv[kHalf];
+                ptx::tmem_ld64(t_s + h * kHalf, sv);
+                ptx::tmem_ld64(t_dp + h * kHalf, dv);
+                const int32_t c0 = base + h * kHalf;   // streamed row of column 0
+                const bool partial = c0 < lo || c0 + kHalf > hi;
+                uint32_t pk_p[kHalf / 2], pk_ds[kHalf / 2];
+#pragma unroll
+                for (int e = 0; e < kHalf / 2; ++e) {
+                    float pv[2], dsv[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int c = 2 * e + k;
+                        float l2, de;
+                        if (FORM == kDQ) {
+                            l2 = lse2_own;
+                            de = delta_own;
+                        } else {
+                            l2 = sm.lse2[stage][h * kHalf + c];
+                            de = sm.delta[stage][h * kHalf + c];
+                        }
+                        float pr = ptx::ex2(fmaf(__uint_as_float(sv[c]), c2, -l2));
+                        if (partial && (c0 + c < lo || c0 + c >= hi)) pr = 0.f;
+                        pv[k] = pr;
+                        dsv[k] = pr * (__uint_as_float(dv[c]) - de);
+                    }
+                    pk_p[e] = ptx::pack_bf16x2(pv[0], pv[1]);
+                    pk_ds[e] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+                }
+                if (FORM == kDKDV) ptx::tmem_st32_nowait(t_s + h * kHalf, pk_p);
+                ptx::tmem_st32_nowait(t_dp + h * kHalf, pk_ds);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[h]));
+            }
+        }
+        // Epilogue: accumulators -> bf16 rows.
+        if (!__all_sync(kAll, wait_phase(sm, sm.acc_full, unit_iter & 1, kErrTimeoutSoftmax)))
+            return;
+        ptx::tc_fence_after();
+        const int side = U.detail ? 0 : 1;
+        const int64_t out_row = static_cast<int64_t>(U.b) * (U.detail ? p.N : p.G) +
+                                (valid ? row : 0);
+        const int n_acc = FORM == kDQ ? 1 : 2;
+#pragma unroll 1
+        for (int a = 0; a < n_acc; ++a) {
+            // DQ: dQ * scale; DKDV: dV (a = 0), dK * scale (a = 1)
+            const float f = (FORM == kDQ || a == 1) ? p.scale : 1.f;
+            __nv_bfloat16 *out = (a == 0 ? p.out0[side] : p.out1[side]);
+            uint4 *dst = reinterpret_cast<uint4 *>(out + (out_row * p.heads + U.head) * HD);
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(t_acc + a * HD + c * 32, o);
+                if (valid) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * f,
+                                               __uint_as_float(o[8 * v + 1]) * f);
+                        w.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * f,
+                                               __uint_as_float(o[8 * v + 3]) * f);
+                        w.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * f,
+                                               __uint_as_float(o[8 * v + 5]) * f);
+                        w.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * f,
+                                               __uint_as_float(o[8 * v + 7]) * f);
+                        dst[c * 4 + v] = w;
+                    }
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&sm.acc_empty));
+    }
+}
+
+template <int HD, int FORM>
+__global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem<HD> &sm = *reinterpret_cast<Smem<HD> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(ptx::smem_addr(&sm.x_full), 1);
+        ptx::mbar_init(ptx::smem_addr(&sm.x_empty), 1);
+        for (int s = 0; s < Smem<HD>::kStages; ++s) {
+            ptx::mbar_init(ptx::smem_addr(&sm.st_full[s]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.st_empty[s]), 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            ptx::mbar_init(ptx::smem_addr(&sm.s_full[h]), 1);
+            ptx::mbar_init(ptx::smem_addr(&sm.p_full[h]), kCompute);
+        }
+        ptx::mbar_init(ptx::smem_addr(&sm.acc_full), 1);
+        ptx::mbar_init(ptx::smem_addr(&sm.acc_empty), kCompute);
+        ptx::mbar_init(ptx::smem_addr(&sm.drain), 1);
+        sm.abort = 0;
+        sm.err_word = p.err_word;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_addr(&sm.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::prefetch_tmap(&p.tm_q[i]);
+            ptx::prefetch_tmap(&p.tm_k[i]);
+            ptx::prefetch_tmap(&p.tm_v[i]);
+            ptx::prefetch_tmap(&p.tm_do[i]);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const bool tmem_ok = tmem == 0;   // a 512-column allocation starts at column 0
+    if (!tmem_ok && threadIdx.x == 0) atomicOr(p.err_word, kErrTmemAlloc);
+    if (tmem_ok) {
+        if (warp < 4) compute<HD, FORM>(p, sm, tmem);
+        else if (warp == kProducerWarp) producer<HD, FORM>(p, sm);
+        else if (lane == 0) mma_issuer<HD, FORM>(p, sm, tmem);
+    }
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+template <int HD, int FORM>
+atlas_status launch_form(Params p, const DeviceInfo &dev, cudaStream_t stream) {
+    const size_t smem = sizeof(Smem<HD>) + 1024;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [&] {
+        attr = cudaFuncSetAttribute(attn_bwd_tc_kernel<HD, FORM>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+    });
+    if (attr != cudaSuccess) return ATLAS_ERR_CUDA;
+    const int64_t per_prob = p.tiles_d + p.tiles_g;
+    const int64_t units = per_prob * p.batch * p.heads;
+    if (units == 0) return ATLAS_OK;
+    if (units > INT32_MAX) return ATLAS_ERR_SHAPE;
+    p.n_units = static_cast<int32_t>(units);
+    p.n_long = FORM == kDKDV ? p.tiles_g * p.batch * p.heads : 0;
+    const int grid = static_cast<int>(std::min<int64_t>(units, dev.sm_count));
+    attn_bwd_tc_kernel<HD, FORM><<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+template <int HD>
+atlas_status launch_hd(const AttnBwdArgs &b, const DeviceInfo &dev, cudaStream_t stream) {
+    const AttnArgs &a = b.fwd;
+    Params p{};
+    const bool has_d = a.n_detail > 0, has_g = a.n_global > 0;
+    const int64_t nd = a.n_detail * a.batch, ng = a.n_global * a.batch;
+    // Maps of an absent side point at the other side; they are never used.
+    const void *src[2][4] = {{a.q_d, a.k_d, a.v_d, b.do_d}, {a.q_g, a.k_g, a.v_g, b.do_g}};
+    const int64_t rows[2] = {nd, ng};
+    CUtensorMap *maps[4] = {p.tm_q, p.tm_k, p.tm_v, p.tm_do};
+    for (int side = 0; side < 2; ++side) {
+        const int use = (side == 0 ? has_d : has_g) ? side : 1 - side;
+        for (int t = 0; t < 4; ++t)
+            if (!make_rows_map(&maps[t][side], src[use][t], rows[use], a.heads, HD))
+                return ATLAS_ERR_CUDA;
+    }
+    p.lse = a.lse;
+    p.delta = b.delta;
+    p.err_word = device_error_word();
+    if (!p.err_word) return ATLAS_ERR_CUDA;
+    p.N = static_cast<int32_t>(a.n_detail);
+    p.L = static_cast<int32_t>(has_d ? a.window_len : 1);
+    p.G = static_cast<int32_t>(a.n_global);
+    p.heads = a.heads;
+    p.batch = static_cast<int32_t>(a.batch);
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * kLog2e;
+    p.win_off = a.win_off;
+    p.gwin_off = a.gwin_off;
+    p.n_win = static_cast<int32_t>(a.win_off ? a.n_win : a.n_gwin);
+    p.tiles_d = static_cast<int32_t>((a.n_detail + kRows - 1) / kRows);
+    p.tiles_g = static_cast<int32_t>((a.n_global + kRows - 1) / kRows);
+    Params pq = p;
+    pq.out0[0] = static_cast<__nv_bfloat16 *>(b.dq_d);
+    pq.out0[1] = static_cast<__nv_bfloat16 *>(b.dq_g);
+    atlas_status st = launch_form<HD, kDQ>(pq, dev, stream);
+    if (st != ATLAS_OK) return st;
+    Params pk = p;
+    pk.out0[0] = static_cast<__nv_bfloat16 *>(b.dv_d);
+    pk.out0[1] = static_cast<__nv_bfloat16 *>(b.dv_g);
+    pk.out1[0] = static_cast<__nv_bfloat16 *>(b.dk_d);
+    pk.out1[1] = static_cast<__nv_bfloat16 *>(b.dk_g);
+    return launch_form<HD, kDKDV>(pk, dev, stream);
+}
+
+}  // namespace
+
+atlas_status launch_attn_bwd_tc_bf16(const AttnBwdArgs &b, cudaStream_t stream) {
+    DeviceInfo dev;
+    if (!current_device(&dev)) return ATLAS_ERR_DEVICE;
+    if (b.fwd.head_dim == 128) return launch_hd<128>(b, dev, stream);
+    if (b.fwd.head_dim == 64) return launch_hd<64>(b, dev, stream);
+    return ATLAS_ERR_UNSUPPORTED;
+}
+
+}  // namespace atlas

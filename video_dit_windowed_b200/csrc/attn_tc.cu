@@ -43,6 +43,40 @@
 #include "sm100_ptx.cuh"
 
 namespace atlas {
+
+// ---------------------------------------------------------------------------
+// Tensor maps (host).
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(hd) * 2,
+                             static_cast<cuuint64_t>(heads) * hd * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr int kBM = 128;          // query rows per Q tile
@@ -626,41 +660,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-// ---------------------------------------------------------------------------
-// Host side.
-// ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void *ptr = nullptr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
-                                             cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// [rows, heads, hd] bf16 viewed as a 3-D tensor (hd, heads, rows); box of
-// 64 channels x 1 head x 128 rows, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(heads),
-                          static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(hd) * 2,
-                             static_cast<cuuint64_t>(heads) * hd * 2};
-    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBM)};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int HD>
 atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t stream) {
     Params p{};
@@ -672,9 +671,12 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
                *vg = has_g ? a.v_g : a.v_d;
     const int64_t nd = (has_d ? a.n_detail : a.n_global) * a.batch,
                   ng = (has_g ? a.n_global : a.n_detail) * a.batch;
-    if (!make_map(&p.tm_qd, qd, nd, a.heads, HD) || !make_map(&p.tm_kd, kd, nd, a.heads, HD) ||
-        !make_map(&p.tm_vd, vd, nd, a.heads, HD) || !make_map(&p.tm_qg, qg, ng, a.heads, HD) ||
-        !make_map(&p.tm_kg, kg, ng, a.heads, HD) || !make_map(&p.tm_vg, vg, ng, a.heads, HD))
+    if (!make_rows_map(&p.tm_qd, qd, nd, a.heads, HD) ||
+        !make_rows_map(&p.tm_kd, kd, nd, a.heads, HD) ||
+        !make_rows_map(&p.tm_vd, vd, nd, a.heads, HD) ||
+        !make_rows_map(&p.tm_qg, qg, ng, a.heads, HD) ||
+        !make_rows_map(&p.tm_kg, kg, ng, a.heads, HD) ||
+        !make_rows_map(&p.tm_vg, vg, ng, a.heads, HD))
         return ATLAS_ERR_CUDA;
     p.o_d = static_cast<__nv_bfloat16 *>(a.o_d);
     p.o_g = static_cast<__nv_bfloat16 *>(a.o_g);

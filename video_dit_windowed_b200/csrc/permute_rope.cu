@@ -207,7 +207,10 @@ __device__ __forceinline__ uint4 rotate<4>(uint4 v, const float2 *cs) {
 
 // MODE 0: dst in cube order, src raster (reorder). MODE 1: dst raster, src
 // cube order (unorder). MODE 2: dst and src raster (RoPE only). MODE 3 / 4:
-// as 0 / 1 for grids the cube does not divide (partial cubes).
+// as 0 / 1 for grids the cube does not divide (partial cubes). With ROPE the
+// row is rotated for the grid position (t, h, w) of its token, in every mode
+// (unorder + rotation with negated scales is the transpose of reorder +
+// rotation, i.e. its gradient).
 template <int EB, bool ROPE, int MODE>
 __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) {
     constexpr int kPairs = 16 / EB / 2;  // RoPE pairs in one 16-byte vector
@@ -367,6 +370,9 @@ atlas_status dispatch(const Params &p, bool rope, int mode, bool general, const 
                       cudaStream_t stream) {
     if (rope) {
         if (mode == 2) return launch<EB, true, 2>(p, dev, stream);
+        if (mode == 1)
+            return general ? launch<EB, true, 4>(p, dev, stream)
+                           : launch<EB, true, 1>(p, dev, stream);
         return general ? launch<EB, true, 3>(p, dev, stream) : launch<EB, true, 0>(p, dev, stream);
     }
     if (mode == 0)
