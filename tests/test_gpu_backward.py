@@ -7,9 +7,11 @@ inputs) are compared per gradient tensor, relative to the reference's scale:
   rel_max = max|g - ref| / max|ref|,  rel_rms = rms(g - ref) / rms(ref).
 Bounds (derived from the arithmetic): bf16 keeps 8 significant bits, so each
 of P, dS, O (inside delta) and the output is rounded with relative error up
-to 2^-9 ~ 2e-3; dS rows sum to ~0, so dQ and dK lose up to a few bits more
-to cancellation. bf16: rel_rms <= 1.5e-2, rel_max <= 5e-2. fp32 (exact fp32
-products, expf): rel_rms <= 1e-5, rel_max <= 1e-4.
+to 2^-9 ~ 2e-3; rounding the output alone gives rel_rms ~ 2^-9/sqrt(3) ~
+1.1e-3, and the rounded P and dS add about as much again. bf16: rel_rms <=
+6e-3, rel_max <= 1.5e-2 (measured on B200: rel_rms 2.4e-3, rel_max <= 4.5e-3
+over the cases below). fp32 (exact fp32 products, expf, accumulation over up
+to ~1e3 terms): rel_rms <= 2e-6, rel_max <= 5e-6 (measured <= 4e-7 / 7e-7).
 """
 import numpy as np
 import pytest
@@ -21,7 +23,7 @@ from video_dit_windowed_b200.workloads import normal
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-TOL = {"bf16": (1.5e-2, 5e-2), "fp32": (1e-5, 1e-4)}
+TOL = {"bf16": (6e-3, 1.5e-2), "fp32": (2e-6, 5e-6)}
 NAMES = ("dq_d", "dk_d", "dv_d", "dq_g", "dk_g", "dv_g")
 
 

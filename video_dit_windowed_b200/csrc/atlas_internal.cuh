@@ -96,9 +96,10 @@ struct AttnArgs {
 };
 atlas_status launch_attn_tc_bf16(const AttnArgs &a, cudaStream_t stream);
 // [rows, heads, hd] bf16 viewed as a 3-D tensor (hd, heads, rows) with a box
-// of 64 channels x 1 head x 128 rows and 128-byte swizzle (defined in
+// of 64 channels x 1 head x box_rows rows and 128-byte swizzle (defined in
 // attn_tc.cu). False if the driver entry point is missing or encoding fails.
-bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd);
+bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd,
+                   int box_rows = 128);
 // One-shot request (atlas_debug_stall_next_attention): true once, for the
 // next bf16 attention launch, which then leaves one K tile unloaded.
 bool take_stall_request();

@@ -16,7 +16,10 @@
 //           of the queries that may see those keys (for a detail key, its
 //           window's queries; for a global key, the detail queries that see
 //           it and every global query); accumulates dV and dK.
-// Either way a streamed tile of 128 rows is taken in two halves of 64. For
+// Either way a streamed tile of 128 rows is taken in two halves of 64, each
+// loaded into its own stage of the shared-memory ring (so three halves can
+// be in flight while one is used; the streamed queries' LSE and delta ride in
+// the same stage, copied by cp.async). For
 // half h the MMA warp computes  S_h = X X'_h^T  and  dP_h = Y Y'_h^T  into
 // tensor memory (X, Y resident, X', Y' streamed: Q/K and dO/V for DQ, K/Q and
 // V/dO for DKDV); the 128 compute threads (one resident row each) turn them
@@ -27,7 +30,13 @@
 // and issues the next tile's S_h, dP_h behind them. MMAs issued by one thread
 // execute in order, so the next S_h cannot overwrite P_h before it is read,
 // and the compute threads work on one half while the tensor core works on
-// the other. Tensor memory: S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc.
+// the other. Two compute warpgroups share the work: thread r of warpgroup g
+// takes resident row r and columns 32g .. 32g+31 of each half (and, in the
+// epilogue, half of the accumulator columns). Tensor memory:
+// S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc (DQ: dQ, then dS packed;
+// DKDV: dV, dK). In DKDV the packed P and dS overwrite the first half of
+// S_h and dP_h, which the other warpgroup may still be reading: the two
+// groups meet on an mbarrier between their loads and their stores.
 // Every wait is bounded, as in the forward kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -42,10 +51,10 @@ namespace {
 
 constexpr int kRows = 128;            // resident rows per unit = TMEM lanes
 constexpr int kHalf = 64;             // streamed rows per half tile
-constexpr int kCompute = 128;         // compute threads (warps 0-3)
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kCompute = 256;         // compute threads (warps 0-7: two warpgroups)
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -53,17 +62,21 @@ enum Form { kDQ = 0, kDKDV = 1 };
 
 template <int HD>
 struct Smem {
-    static constexpr int kTile = kRows * HD * 2;                  // one 128-row bf16 tile
-    static constexpr int kStages = (160 * 1024) / (2 * kTile);    // streamed (X', Y') pairs
+    static constexpr int kTile = kRows * HD * 2;                  // a 128-row bf16 tile
+    static constexpr int kHalfTile = kHalf * HD * 2;              // a 64-row bf16 tile
+    // streamed (X', Y') half-tile pairs: 128 KB of ring, at most 8 stages
+    static constexpr int kStages = (128 * 1024) / (2 * kHalfTile) < 8
+                                       ? (128 * 1024) / (2 * kHalfTile) : 8;
     alignas(1024) uint8_t x[kTile];                              // resident X (Q or K)
     alignas(1024) uint8_t y[kTile];                              // resident Y (dO or V)
-    alignas(1024) uint8_t xs[kStages][kTile];                    // streamed X' (K or Q)
-    alignas(1024) uint8_t ys[kStages][kTile];                    // streamed Y' (V or dO)
-    float lse2[kStages][kRows];   // DKDV: log2-scaled LSE of the streamed queries
-    float delta[kStages][kRows];  // DKDV: delta of the streamed queries
+    alignas(1024) uint8_t xs[kStages][kHalfTile];                // streamed X' (K or Q)
+    alignas(1024) uint8_t ys[kStages][kHalfTile];                // streamed Y' (V or dO)
+    float lse[kStages][kHalf];    // DKDV: LSE of the streamed queries (natural log)
+    float delta[kStages][kHalf];  // DKDV: delta of the streamed queries
     uint64_t x_full, x_empty;
     uint64_t st_full[kStages], st_empty[kStages];
     uint64_t s_full[2], p_full[2];
+    uint64_t ld_done[2];          // DKDV: both warpgroups have read S_h and dP_h
     uint64_t acc_full, acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
@@ -72,7 +85,8 @@ struct Smem {
 };
 
 struct Params {
-    CUtensorMap tm_q[2], tm_k[2], tm_v[2], tm_do[2];   // [0] detail, [1] global
+    CUtensorMap tm_q[2], tm_k[2], tm_v[2], tm_do[2];   // 128-row boxes; [0] detail, [1] global
+    CUtensorMap hm_q[2], hm_k[2], hm_v[2], hm_do[2];   // the same with 64-row boxes
     __nv_bfloat16 *out0[2], *out1[2];   // DQ: dq (out0); DKDV: dv (out0), dk (out1)
     const float *lse, *delta;
     uint32_t *err_word;
@@ -238,24 +252,28 @@ __device__ __forceinline__ int32_t streamed_row(const Unit &U, int32_t j) {
 }
 
 // ---------------------------------------------------------------------------
-// Producer warp: resident X, Y once per unit; then (X', Y') pairs into the
-// stage ring, with (DKDV) the streamed queries' LSE and delta.
+// Producer warp: resident X, Y once per unit; then the streamed tiles as
+// 64-row halves, (X'_h, Y'_h) per ring stage, with (DKDV) the streamed
+// queries' LSE and delta copied by cp.async and tracked by the same stage
+// barrier.
 // ---------------------------------------------------------------------------
 template <int HD, int FORM>
 __device__ void producer(const Params &p, Smem<HD> &sm) {
     constexpr int kStages = Smem<HD>::kStages;
-    constexpr uint32_t kTile = Smem<HD>::kTile;
+    constexpr uint32_t kTile = Smem<HD>::kTile, kHalfTile = Smem<HD>::kHalfTile;
+    constexpr uint32_t kAll = 0xffffffffu;
     const uint32_t lane = threadIdx.x & 31;
     uint32_t it = 0, unit_iter = 0, x_armed = 0;
     uint32_t armed[kStages];
 #pragma unroll
     for (int s = 0; s < kStages; ++s) armed[s] = 0;
     bool ok = true;
+    // One tile of `rows_box` rows: HD/64 boxes of 64 channels.
     auto tile = [&](uint8_t *dst, const CUtensorMap *map, uint32_t bar, int32_t head,
-                    int32_t row) {
+                    int32_t row, uint32_t box_bytes) {
 #pragma unroll
         for (int db = 0; db < HD / 64; ++db)
-            ptx::tma_load_3d(ptx::smem_addr(dst + db * kRows * 128), map, bar, db * 64, head,
+            ptx::tma_load_3d(ptx::smem_addr(dst + db * box_bytes), map, bar, db * 64, head,
                              row);
     };
     for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
@@ -263,51 +281,55 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
         // Every lane waits and the warp agrees, so the lanes never diverge
         // around the warp-wide steps below.
         if (unit_iter > 0 &&
-            !(ok = __all_sync(0xffffffffu, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
-                                                      kErrTimeoutProducer))))
+            !(ok = __all_sync(kAll, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
+                                               kErrTimeoutProducer))))
             break;
         const int side = U.detail ? 0 : 1;
         const int32_t rbase = U.b * (U.detail ? p.N : p.G);
         if (lane == 0) {
             const uint32_t bar = ptx::smem_addr(&sm.x_full);
             ptx::mbar_arrive_expect_tx(bar, 2 * kTile);
-            tile(sm.x, FORM == kDQ ? &p.tm_q[side] : &p.tm_k[side], bar, U.head, rbase + U.r0);
-            tile(sm.y, FORM == kDQ ? &p.tm_do[side] : &p.tm_v[side], bar, U.head, rbase + U.r0);
+            tile(sm.x, FORM == kDQ ? &p.tm_q[side] : &p.tm_k[side], bar, U.head, rbase + U.r0,
+                 kRows * 128);
+            tile(sm.y, FORM == kDQ ? &p.tm_do[side] : &p.tm_v[side], bar, U.head, rbase + U.r0,
+                 kRows * 128);
         }
         x_armed = unit_iter + 1;
-        const int32_t n = U.n_a + U.n_b;
-        for (int32_t j = 0; j < n && ok; ++j, ++it) {
+        const int32_t n = 2 * (U.n_a + U.n_b);   // half tiles
+        for (int32_t jh = 0; jh < n && ok; ++jh, ++it) {
             const uint32_t s = it % kStages, round = it / kStages;
             if (round > 0 &&
-                !(ok = __all_sync(0xffffffffu, wait_phase(sm, sm.st_empty[s], (round - 1) & 1,
-                                                          kErrTimeoutProducer))))
+                !(ok = __all_sync(kAll, wait_phase(sm, sm.st_empty[s], (round - 1) & 1,
+                                                   kErrTimeoutProducer))))
                 break;
+            const int32_t j = jh >> 1;
             const bool det = streamed_detail(U, j);
-            const int32_t row = streamed_row(U, j);
+            const int32_t row = streamed_row(U, j) + (jh & 1) * kHalf;   // in the problem
             const int sside = det ? 0 : 1;
+            const uint32_t bar = ptx::smem_addr(&sm.st_full[s]);
             if (FORM == kDKDV) {
-                // LSE (log2 units) and delta of the 128 streamed queries; rows
-                // past the problem get +inf (P = 0) and 0.
+                // LSE and delta of the 64 streamed queries. Rows past the
+                // problem copy the last row's values: those columns are
+                // masked by the compute warps.
                 const int32_t nrows = det ? p.N : p.G;
                 const int64_t col0 = (static_cast<int64_t>(U.b) * p.heads + U.head) *
                                          (p.N + p.G) + (det ? 0 : p.N);
 #pragma unroll
-                for (int i = 0; i < kRows / 32; ++i) {
-                    const int32_t c = i * 32 + lane, q = row + c;
-                    const bool valid = q < nrows;
-                    sm.lse2[s][c] = valid ? __ldg(p.lse + col0 + q) * kLog2e
-                                          : __builtin_huge_valf();
-                    sm.delta[s][c] = valid ? __ldg(p.delta + col0 + q) : 0.f;
+                for (int i = 0; i < kHalf / 32; ++i) {
+                    const int32_t c = i * 32 + lane, q = min(row + c, nrows - 1);
+                    ptx::cp_async_4(ptx::smem_addr(&sm.lse[s][c]), p.lse + col0 + q);
+                    ptx::cp_async_4(ptx::smem_addr(&sm.delta[s][c]), p.delta + col0 + q);
                 }
+                ptx::cp_async_mbar_arrive(bar);
                 __syncwarp();
             }
             if (lane == 0) {
-                const uint32_t bar = ptx::smem_addr(&sm.st_full[s]);
-                ptx::mbar_arrive_expect_tx(bar, 2 * kTile);
+                ptx::mbar_arrive_expect_tx(bar, 2 * kHalfTile);
                 const int32_t srow = (det ? U.b * p.N : U.b * p.G) + row;
-                tile(sm.xs[s], FORM == kDQ ? &p.tm_k[sside] : &p.tm_q[sside], bar, U.head, srow);
-                tile(sm.ys[s], FORM == kDQ ? &p.tm_v[sside] : &p.tm_do[sside], bar, U.head,
-                     srow);
+                tile(sm.xs[s], FORM == kDQ ? &p.hm_k[sside] : &p.hm_q[sside], bar, U.head, srow,
+                     kHalf * 128);
+                tile(sm.ys[s], FORM == kDQ ? &p.hm_v[sside] : &p.hm_do[sside], bar, U.head,
+                     srow, kHalf * 128);
             }
 #pragma unroll
             for (int t = 0; t < kStages; ++t)
@@ -324,12 +346,14 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (one thread).
+// MMA issuer (one thread). Per unit: S_0, dP_0, S_1, dP_1 of tile 0; then per
+// half h of tile j: acc += (P_h, dS_h)(j), release the half's stage, and
+// S_h, dP_h of tile j+1.
 // ---------------------------------------------------------------------------
 template <int HD, int FORM>
 __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     constexpr int kStages = Smem<HD>::kStages;
-    constexpr uint32_t kT16 = Smem<HD>::kTile >> 4;
+    constexpr uint32_t kH16 = Smem<HD>::kHalfTile >> 4;
     constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kRows, kHalf, 0);   // S_h, dP_h
     constexpr uint32_t kIdAcc = ptx::idesc_bf16_f32(kRows, HD, 1);    // acc += A(tmem) B
     constexpr uint32_t kHi = ptx::desc_sw128_hi(1024);
@@ -337,33 +361,33 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     const uint32_t y_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.y), 16);
     const uint32_t xs_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), 16);
     const uint32_t ys_lo = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), 16);
-    // The same streamed tiles as MN-major B operands of the accumulation.
-    const uint32_t xs_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), kRows * 128);
-    const uint32_t ys_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), kRows * 128);
+    // The same streamed half tiles as MN-major B operands of the
+    // accumulation (64-channel blocks kHalf * 128 bytes apart).
+    const uint32_t xs_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), kHalf * 128);
+    const uint32_t ys_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), kHalf * 128);
     const uint32_t t_s = tmem, t_dp = tmem + 2 * kHalf, t_acc = tmem + 4 * kHalf;
     uint32_t it = 0, unit_iter = 0, p_cnt = 0;
     bool ok = true;
 
-    // S_h = X X'_h^T and dP_h = Y Y'_h^T from stage s; then a commit.
+    // S_h = X X'^T and dP_h = Y Y'^T from the half tile in stage s; commit.
     auto issue_sdp = [&](int h, uint32_t s) {
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
             const uint32_t a_off = ((ks / 4) * (kRows * 128) + (ks % 4) * 32) >> 4;
-            const uint32_t b_off = a_off + ((h * kHalf * 128) >> 4);
+            const uint32_t b_off = ((ks / 4) * (kHalf * 128) + (ks % 4) * 32) >> 4;
             ptx::mma_ss(t_s + h * kHalf, ptx::desc_join(x_lo + a_off, kHi),
-                        ptx::desc_join(xs_lo + s * kT16 + b_off, kHi), kIdS, ks > 0);
+                        ptx::desc_join(xs_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
             ptx::mma_ss(t_dp + h * kHalf, ptx::desc_join(y_lo + a_off, kHi),
-                        ptx::desc_join(ys_lo + s * kT16 + b_off, kHi), kIdS, ks > 0);
+                        ptx::desc_join(ys_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
         }
         ptx::mma_commit(ptx::smem_addr(&sm.s_full[h]));
     };
-    // acc += A_h (tensor memory, 64 streamed rows packed in 32 columns) times
-    // the streamed tile's half h as an MN-major B operand.
-    auto issue_acc = [&](uint32_t d, uint32_t a, uint32_t b_lo, int h, uint32_t s,
-                         bool first) {
+    // acc += A (tensor memory, 64 streamed rows packed in 32 columns) times
+    // the half tile in stage s as an MN-major B operand.
+    auto issue_acc = [&](uint32_t d, uint32_t a, uint32_t b_lo, uint32_t s, bool first) {
 #pragma unroll
         for (int ks = 0; ks < kHalf / 16; ++ks) {
-            const uint32_t off = s * kT16 + ((h * kHalf * 128 + ks * 16 * 128) >> 4);
+            const uint32_t off = s * kH16 + ((ks * 16 * 128) >> 4);
             ptx::mma_ts(d, a + ks * 8, ptx::desc_join(b_lo + off, kHi), kIdAcc,
                         (first && ks == 0) ? 0u : 1u);
         }
@@ -381,10 +405,11 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         const int32_t n = U.n_a + U.n_b;
         if (!(ok = wait_phase(sm, sm.x_full, unit_iter & 1, kErrTimeoutMma))) break;
         ptx::tc_fence_after();
-        uint32_t s_cur, s_next = 0;
-        if (!(ok = next_stage(s_cur))) break;
-        issue_sdp(0, s_cur);
-        issue_sdp(1, s_cur);
+        uint32_t st[2];   // stages of the current tile's halves
+        if (!(ok = next_stage(st[0]))) break;
+        issue_sdp(0, st[0]);
+        if (!(ok = next_stage(st[1]))) break;
+        issue_sdp(1, st[1]);
         for (int32_t j = 0; j < n && ok; ++j) {
             const bool more = j + 1 < n;
             for (int h = 0; h < 2 && ok; ++h) {
@@ -395,19 +420,18 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                 ptx::tc_fence_after();
                 const bool first = j == 0 && h == 0;
                 if (FORM == kDQ) {
-                    issue_acc(t_acc, t_dp + h * kHalf, xs_mn, h, s_cur, first);     // dQ
+                    issue_acc(t_acc, t_acc + HD + h * (kHalf / 2), xs_mn, st[h], first);
                 } else {
-                    issue_acc(t_acc, t_s + h * kHalf, ys_mn, h, s_cur, first);      // dV
-                    issue_acc(t_acc + HD, t_dp + h * kHalf, xs_mn, h, s_cur, first); // dK
+                    issue_acc(t_acc, t_s + h * kHalf, ys_mn, st[h], first);       // dV
+                    issue_acc(t_acc + HD, t_dp + h * kHalf, xs_mn, st[h], first);  // dK
                 }
-                if (h == 1) ptx::mma_commit(ptx::smem_addr(&sm.st_empty[s_cur]));
+                ptx::mma_commit(ptx::smem_addr(&sm.st_empty[st[h]]));
                 if (more) {
-                    if (h == 0 && !(ok = next_stage(s_next))) break;
-                    issue_sdp(h, s_next);
+                    if (!(ok = next_stage(st[h]))) break;
+                    issue_sdp(h, st[h]);
                 }
             }
             ++p_cnt;
-            s_cur = s_next;
         }
         if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&sm.acc_full));
@@ -424,11 +448,14 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
 template <int HD, int FORM>
 __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     constexpr int kStages = Smem<HD>::kStages;
+    constexpr int kCols = kHalf / 2;                 // columns of a half per warpgroup
     constexpr uint32_t kAll = 0xffffffffu;
     const uint32_t warp = threadIdx.x / 32, r = threadIdx.x & 127;
-    const uint32_t lane_sel = (warp * 32u) << 16;
+    const int part = static_cast<int>(warp / 4);     // warpgroup: column block
+    const uint32_t lane_sel = ((warp & 3) * 32u) << 16;
     const uint32_t t_s = tmem + lane_sel, t_dp = tmem + 2 * kHalf + lane_sel;
     const uint32_t t_acc = tmem + 4 * kHalf + lane_sel;
+    const uint32_t t_ds = t_acc + HD;                 // DQ: packed dS_0 | dS_1
     const float c2 = p.scale_log2;
     uint32_t cnt = 0, unit_iter = 0;
 
@@ -474,24 +501,26 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
             const bool det = streamed_detail(U, j);
             const int32_t base = streamed_row(U, j);
             const int32_t lo = det ? da : ga, hi = det ? db : gb;
-            const uint32_t stage = cnt % kStages;
-            if (FORM == kDKDV &&
-                !__all_sync(kAll, wait_phase(sm, sm.st_full[stage], (cnt / kStages) & 1,
-                                             kErrTimeoutSoftmax)))
-                return;
 #pragma unroll 1
             for (int h = 0; h < 2; ++h) {
+                // ring stage of this half tile (the producer's order)
+                const uint32_t hc = 2 * cnt + h, stage = hc % kStages;
+                if (FORM == kDKDV &&
+                    !__all_sync(kAll, wait_phase(sm, sm.st_full[stage], (hc / kStages) & 1,
+                                                 kErrTimeoutSoftmax)))
+                    return;
                 if (!__all_sync(kAll, wait_phase(sm, sm.s_full[h], cnt & 1, kErrTimeoutSoftmax)))
                     return;
                 ptx::tc_fence_after();
-                uint32_t sv[kHalf], dv[kHalf];
-                ptx::tmem_ld64(t_s + h * kHalf, sv);
-                ptx::tmem_ld64(t_dp + h * kHalf, dv);
-                const int32_t c0 = base + h * kHalf;   // streamed row of column 0
-                const bool partial = c0 < lo || c0 + kHalf > hi;
-                uint32_t pk_p[kHalf / 2], pk_ds[kHalf / 2];
+                uint32_t sv[kCols], dv[kCols];
+                ptx::tmem_ld32(t_s + h * kHalf + part * kCols, sv);
+                ptx::tmem_ld32(t_dp + h * kHalf + part * kCols, dv);
+                if (FORM == kDKDV) ptx::mbar_arrive(ptx::smem_addr(&sm.ld_done[h]));
+                const int32_t c0 = base + h * kHalf + part * kCols;   // row of column 0
+                const bool partial = c0 < lo || c0 + kCols > hi;
+                uint32_t pk_p[kCols / 2], pk_ds[kCols / 2];
 #pragma unroll
-                for (int e = 0; e < kHalf / 2; ++e) {
+                for (int e = 0; e < kCols / 2; ++e) {
                     float pv[2], dsv[2];
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -501,8 +530,8 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                             l2 = lse2_own;
                             de = delta_own;
                         } else {
-                            l2 = sm.lse2[stage][h * kHalf + c];
-                            de = sm.delta[stage][h * kHalf + c];
+                            l2 = sm.lse[stage][part * kCols + c] * kLog2e;
+                            de = sm.delta[stage][part * kCols + c];
                         }
                         float pr = ptx::ex2(fmaf(__uint_as_float(sv[c]), c2, -l2));
                         if (partial && (c0 + c < lo || c0 + c >= hi)) pr = 0.f;
@@ -512,8 +541,16 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                     pk_p[e] = ptx::pack_bf16x2(pv[0], pv[1]);
                     pk_ds[e] = ptx::pack_bf16x2(dsv[0], dsv[1]);
                 }
-                if (FORM == kDKDV) ptx::tmem_st32_nowait(t_s + h * kHalf, pk_p);
-                ptx::tmem_st32_nowait(t_dp + h * kHalf, pk_ds);
+                // packed pairs: this warpgroup's 32 values are columns 16g .. 16g+15
+                if (FORM == kDKDV) {
+                    if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], cnt & 1,
+                                                     kErrTimeoutSoftmax)))
+                        return;
+                    ptx::tmem_st16_nowait(t_s + h * kHalf + part * 16, pk_p);
+                    ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 16, pk_ds);
+                } else {
+                    ptx::tmem_st16_nowait(t_ds + h * (kHalf / 2) + part * 16, pk_ds);
+                }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[h]));
@@ -526,17 +563,20 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         const int side = U.detail ? 0 : 1;
         const int64_t out_row = static_cast<int64_t>(U.b) * (U.detail ? p.N : p.G) +
                                 (valid ? row : 0);
-        const int n_acc = FORM == kDQ ? 1 : 2;
-#pragma unroll 1
-        for (int a = 0; a < n_acc; ++a) {
-            // DQ: dQ * scale; DKDV: dV (a = 0), dK * scale (a = 1)
+        // DQ: warpgroup g stores columns [g*HD/2, (g+1)*HD/2) of dQ * scale;
+        // DKDV: warpgroup 0 stores dV, warpgroup 1 stores dK * scale.
+        {
+            const int a = FORM == kDQ ? 0 : part;
             const float f = (FORM == kDQ || a == 1) ? p.scale : 1.f;
             __nv_bfloat16 *out = (a == 0 ? p.out0[side] : p.out1[side]);
-            uint4 *dst = reinterpret_cast<uint4 *>(out + (out_row * p.heads + U.head) * HD);
+            const int col0 = FORM == kDQ ? part * (HD / 2) : 0;
+            const int ncol = FORM == kDQ ? HD / 2 : HD;
+            uint4 *dst = reinterpret_cast<uint4 *>(out + (out_row * p.heads + U.head) * HD +
+                                                   col0);
 #pragma unroll 1
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int c = 0; c < ncol / 32; ++c) {
                 uint32_t o[32];
-                ptx::tmem_ld32(t_acc + a * HD + c * 32, o);
+                ptx::tmem_ld32(t_acc + a * HD + col0 + c * 32, o);
                 if (valid) {
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
@@ -575,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         for (int h = 0; h < 2; ++h) {
             ptx::mbar_init(ptx::smem_addr(&sm.s_full[h]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.p_full[h]), kCompute);
+            ptx::mbar_init(ptx::smem_addr(&sm.ld_done[h]), kCompute);
         }
         ptx::mbar_init(ptx::smem_addr(&sm.acc_full), 1);
         ptx::mbar_init(ptx::smem_addr(&sm.acc_empty), kCompute);
@@ -593,6 +634,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
             ptx::prefetch_tmap(&p.tm_k[i]);
             ptx::prefetch_tmap(&p.tm_v[i]);
             ptx::prefetch_tmap(&p.tm_do[i]);
+            ptx::prefetch_tmap(&p.hm_q[i]);
+            ptx::prefetch_tmap(&p.hm_k[i]);
+            ptx::prefetch_tmap(&p.hm_v[i]);
+            ptx::prefetch_tmap(&p.hm_do[i]);
         }
     }
     ptx::tc_fence_before();
@@ -602,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     const bool tmem_ok = tmem == 0;   // a 512-column allocation starts at column 0
     if (!tmem_ok && threadIdx.x == 0) atomicOr(p.err_word, kErrTmemAlloc);
     if (tmem_ok) {
-        if (warp < 4) compute<HD, FORM>(p, sm, tmem);
+        if (warp < 8) compute<HD, FORM>(p, sm, tmem);
         else if (warp == kProducerWarp) producer<HD, FORM>(p, sm);
         else if (lane == 0) mma_issuer<HD, FORM>(p, sm, tmem);
     }
@@ -648,10 +693,12 @@ atlas_status launch_hd(const AttnBwdArgs &b, const DeviceInfo &dev, cudaStream_t
     const void *src[2][4] = {{a.q_d, a.k_d, a.v_d, b.do_d}, {a.q_g, a.k_g, a.v_g, b.do_g}};
     const int64_t rows[2] = {nd, ng};
     CUtensorMap *maps[4] = {p.tm_q, p.tm_k, p.tm_v, p.tm_do};
+    CUtensorMap *half_maps[4] = {p.hm_q, p.hm_k, p.hm_v, p.hm_do};
     for (int side = 0; side < 2; ++side) {
         const int use = (side == 0 ? has_d : has_g) ? side : 1 - side;
         for (int t = 0; t < 4; ++t)
-            if (!make_rows_map(&maps[t][side], src[use][t], rows[use], a.heads, HD))
+            if (!make_rows_map(&maps[t][side], src[use][t], rows[use], a.heads, HD, kRows) ||
+                !make_rows_map(&half_maps[t][side], src[use][t], rows[use], a.heads, HD, kHalf))
                 return ATLAS_ERR_CUDA;
     }
     p.lse = a.lse;

@@ -61,14 +61,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd) {
+bool make_rows_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int hd,
+                   int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(heads),
                           static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(hd) * 2,
                              static_cast<cuuint64_t>(heads) * hd * 2};
-    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
