@@ -13,6 +13,10 @@ Pages cited (title, section):
     attention) and 2 (asymmetric hierarchical attention, position alignment).
   * "AtlasVid: Efficient Ultra-High-Resolution Long Video Generation via
     Decoupled Global-Local Modeling", abstract.
+  * The projections on either side of the path (QKV in, output out) are the
+    attention layer's linear maps; the summary's training strategy adapts
+    exactly these ("attention projections"). Their oracle is numpy's matmul
+    composed with the pinned reorder and RoPE functions.
 
 Every function takes and returns numpy arrays; floating-point inputs are
 converted to float64 exactly before the C code sees them.
@@ -331,6 +335,42 @@ class Oracle:
         f = lambda D, *p: self.lib.atlas_oracle_attention_bwd_head_aligned(
             *grid, *cube, *global_grid, D, float(scale), *p, int(n_threads))
         return self._bwd(f, q_d, k_d, v_d, q_g, k_g, v_g, do_d, do_g)
+
+    # -- projections around the path (QKV in, output out) ------------------
+    def qkv_proj_reorder(self, x, w, grid, cube, heads, head_dim, theta=10000.0, split=None,
+                         scales=None):
+        """[Q | K | V] = x w^T (x: [rows, C] raster order, w: [3*heads*head_dim, C]),
+        Q and K rotated by 3D RoPE at their raster positions when ``split``
+        is given, all three reordered to cube order. fp64; returns (q, k, v),
+        each [rows, heads, head_dim]. ``rows`` may hold several problems of
+        ``grid`` stacked."""
+        x = np.asarray(x, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64)
+        y = x @ w.T                              # library matmul, fp64
+        n = grid[0] * grid[1] * grid[2]
+        hd = heads * head_dim
+        out = []
+        for i in range(3):
+            t = y[:, i * hd:(i + 1) * hd].reshape(-1, heads, head_dim)
+            parts = []
+            for b in range(t.shape[0] // n):
+                tb = np.ascontiguousarray(t[b * n:(b + 1) * n])
+                if i < 2 and split is not None:
+                    tb = self.rope3d_grid(tb, grid, theta, split, scales)
+                parts.append(self.cube_reorder(tb, grid, cube))
+            out.append(np.concatenate(parts) if parts else t.copy())
+        return tuple(out)
+
+    def out_proj_unorder(self, o, w, grid, cube):
+        """y = unorder(o) w^T (o: [rows, heads*head_dim] in cube order, w:
+        [C_out, heads*head_dim]); fp64, [rows, C_out] in raster order."""
+        o = np.asarray(o, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64)
+        n = grid[0] * grid[1] * grid[2]
+        raster = np.concatenate([self.cube_unorder(np.ascontiguousarray(o[b * n:(b + 1) * n]),
+                                                   grid, cube)
+                                 for b in range(o.shape[0] // n)])
+        return raster @ w.T
 
     def max_threads(self) -> int:
         return int(self.lib.atlas_oracle_max_threads())

@@ -697,6 +697,63 @@ def pin_bwd_single_token_windows(o):
     assert np.max(np.abs(dqd)) < 1e-14 and np.max(np.abs(dkd)) < 1e-14
 
 
+# ---------------------------------------------------------------------------
+# Projections around the path
+# ---------------------------------------------------------------------------
+
+def pin_proj_matches_loops(o):
+    """QKV projection + RoPE + reorder equals plain loops: each output
+    element a dot product of one x row with one w row, pairs rotated by the
+    literal angle p*theta^(-2k/d) of the token's axis position, the row
+    placed at its lexsort cube position."""
+    rng = np.random.default_rng(9)
+    grid, cube, heads, hd, C = (2, 3, 2), (2, 2, 1), 2, 4, 5
+    split, scales, theta = (2, 0, 2), (1.5, 1.0, 2.0), 100.0
+    T, H, W = grid
+    n = T * H * W
+    x = rng.standard_normal((2 * n, C))            # two problems
+    w = rng.standard_normal((3 * heads * hd, C))
+    q, k, v = o.qkv_proj_reorder(x, w, grid, cube, heads, hd, theta, split, scales)
+    order = lexsort_order(grid, cube)
+    for b in range(2):
+        for j in range(n):
+            r = int(order[j])
+            t_, h_, w_ = r // (H * W), (r // W) % H, r % W
+            for which, got in enumerate((q, k, v)):
+                for hh in range(heads):
+                    vals = [sum(x[b * n + r, c] * w[which * heads * hd + hh * hd + d, c]
+                                for c in range(C)) for d in range(hd)]
+                    if which < 2:
+                        off = 0
+                        for pos, dd, sc in ((t_, split[0], scales[0]), (h_, split[1], scales[1]),
+                                            (w_, split[2], scales[2])):
+                            for kk in range(dd // 2):
+                                ang = pos * sc * theta ** (-2.0 * kk / dd)
+                                a0, a1 = vals[off + 2 * kk], vals[off + 2 * kk + 1]
+                                vals[off + 2 * kk] = a0 * math.cos(ang) - a1 * math.sin(ang)
+                                vals[off + 2 * kk + 1] = a0 * math.sin(ang) + a1 * math.cos(ang)
+                            off += dd
+                    assert np.max(np.abs(got[b * n + j, hh] - np.array(vals))) < 1e-12
+
+
+def pin_out_proj_matches_loops(o):
+    """Output projection of cube-ordered rows equals the raster row's plain
+    dot products (the row a cube position holds goes back to its token)."""
+    rng = np.random.default_rng(10)
+    grid, cube, hdim, C = (3, 2, 3), (2, 2, 2), 6, 4
+    n = 18
+    oc = rng.standard_normal((n, hdim))
+    w = rng.standard_normal((C, hdim))
+    y = o.out_proj_unorder(oc, w, grid, cube)
+    order = lexsort_order(grid, cube)
+    for j in range(n):
+        r = int(order[j])
+        for c in range(C):
+            assert abs(y[r, c] - sum(oc[j, e] * w[c, e] for e in range(hdim))) < 1e-12
+
+
+PROJ_PINS = [pin_proj_matches_loops, pin_out_proj_matches_loops]
+
 BWD_PINS = [pin_bwd_autograd_dense, pin_bwd_finite_differences, pin_bwd_single_token_windows]
 
 ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
@@ -707,4 +764,4 @@ ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
              pin_attention_rows_sum_to_one, pin_attention_global_ignores_detail,
              pin_attention_probe_mass, pin_attention_rejects_missing_rows]
 
-ALL_PINS = CUBE_PINS + ROPE_PINS + ATTN_PINS + BWD_PINS
+ALL_PINS = CUBE_PINS + ROPE_PINS + ATTN_PINS + BWD_PINS + PROJ_PINS
