@@ -369,6 +369,100 @@ class Path:
         return d
 
 
+class ProjPath:
+    """The path with the projections on either side, fused (--proj): QKV
+    projection with RoPE and reorder in the GEMM epilogue (detail tokens, and
+    the global proxy with a 1x1x1 cube), the attention, and the output
+    projection writing rows back to raster order. Model width C =
+    heads*head_dim; weights are seeded, random (N(0,1)/sqrt(C)), bf16.
+    Also times, for comparison only, the same projections unfused: torch's
+    matmul (cuBLAS) then the separate reorder / RoPE / unorder kernels."""
+
+    def __init__(self, w, device, stream):
+        from video_dit_windowed_b200 import atlas
+        from video_dit_windowed_b200.workloads import normal
+        self.atlas, self.w, self.stream = atlas, w, stream
+        C = w.heads * w.head_dim
+        self.C = C
+        N, G = w.n_detail, w.n_global
+        bf = torch.bfloat16
+        self.x_d = normal((N, C), "q_d", bf, 0, device)
+        self.x_g = normal((G, C), "q_g", bf, 0, device)
+        self.w_qkv = (normal((3 * C, C), "k_d", torch.float32, 0, device) / C ** 0.5).to(bf)
+        self.w_o = (normal((C, C), "v_d", torch.float32, 0, device) / C ** 0.5).to(bf)
+        e = lambda rows: torch.empty(rows, w.heads, w.head_dim, dtype=bf, device=device)
+        self.q_d, self.k_d, self.v_d = e(N), e(N), e(N)
+        self.q_g, self.k_g, self.v_g = e(G), e(G), e(G)
+        self.o_d, self.o_g = e(N), e(G)
+        self.y_d = torch.empty(N, C, dtype=bf, device=device)
+        self.y_g = torch.empty(G, C, dtype=bf, device=device)
+        self.rd = atlas.make_rope(w.theta, w.split, w.detail_scales)
+        self.rg = atlas.make_rope(w.theta, w.split, w.global_scales)
+        self.one = (1, 1, 1)
+        self.mask = "all"
+        self.backward = False
+
+    def step(self, ev=None):
+        a, w, s = self.atlas, self.w, self.stream
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec(0)
+        a.qkv_proj_reorder(self.x_d, self.w_qkv, w.grid, w.cube, self.q_d, self.k_d, self.v_d,
+                           self.rd, stream=s)
+        rec(1)
+        a.qkv_proj_reorder(self.x_g, self.w_qkv, w.global_grid, self.one, self.q_g, self.k_g,
+                           self.v_g, self.rg, stream=s)
+        rec(2)
+        a.local_global_attn(self.q_d, self.k_d, self.v_d, w.window_len, self.q_g, self.k_g,
+                            self.v_g, self.o_d, self.o_g, None, stream=s)
+        rec(3)
+        a.out_proj_unorder(self.o_d, self.w_o, w.grid, w.cube, self.y_d, stream=s)
+        a.out_proj_unorder(self.o_g, self.w_o, w.global_grid, self.one, self.y_g, stream=s)
+        rec(4)
+
+    def unfused_ms(self, steps):
+        """Median time of the same projections unfused (cuBLAS matmul, then
+        the separate permutation kernels), QKV and output parts."""
+        a, w, s = self.atlas, self.w, self.stream
+        C, N = self.C, w.n_detail
+        tmp = torch.empty(N, C, dtype=torch.bfloat16, device=self.x_d.device)
+        tmp_o = torch.empty(N, w.heads, w.head_dim, dtype=torch.bfloat16, device=tmp.device)
+        t_qkv, t_out = [], []
+        for i in range(steps + 2):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            with torch.cuda.stream(s):
+                ev[0].record(s)
+                for j, (dst, rope) in enumerate(((self.q_d, self.rd), (self.k_d, self.rd),
+                                                 (self.v_d, None))):
+                    torch.matmul(self.x_d, self.w_qkv[j * C:(j + 1) * C].t(), out=tmp)
+                    a.cube_reorder(tmp.view(N, w.heads, w.head_dim), dst, w.grid, w.cube, rope,
+                                   stream=s)
+                ev[1].record(s)
+                a.cube_unorder(self.o_d, tmp_o, w.grid, w.cube, stream=s)
+                torch.matmul(tmp_o.view(N, C), self.w_o.t(), out=self.y_d)
+                ev[2].record(s)
+            torch.cuda.synchronize()
+            if i >= 2:
+                t_qkv.append(ev[0].elapsed_time(ev[1]))
+                t_out.append(ev[1].elapsed_time(ev[2]))
+        return statistics.median(t_qkv), statistics.median(t_out)
+
+    def flops(self):
+        return self.w.unmasked_flops()
+
+    def proj_flops(self):
+        """(QKV, output) projection FLOPs: 2*rows*C*3C and 2*rows*C*C."""
+        rows = self.w.n_detail + self.w.n_global
+        return 2 * rows * self.C * 3 * self.C, 2 * rows * self.C * self.C
+
+    def launches_per_step(self):
+        return 5
+
+    phase_ms = staticmethod(lambda ev: {"qkv_d": ev[0].elapsed_time(ev[1]),
+                                        "qkv_g": ev[1].elapsed_time(ev[2]),
+                                        "attn": ev[2].elapsed_time(ev[3]),
+                                        "out": ev[3].elapsed_time(ev[4])})
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "video_dit_windowed_b200", "csrc")
@@ -536,7 +630,8 @@ def run_atlas(args, world, rank, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
-        path = Path(w, dev, stream, args.mask, args.batch, args.backward)
+        path = (ProjPath(w, dev, stream) if args.proj
+                else Path(w, dev, stream, args.mask, args.batch, args.backward))
     torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         path.step()
@@ -566,12 +661,15 @@ def run_atlas(args, world, rank, local):
     elapsed = start.elapsed_time(stop)
     phases = {}
     for ev in evs:
-        for k, v in Path.phase_ms(ev).items():
+        for k, v in type(path).phase_ms(ev).items():
             phases.setdefault(k, []).append(v)
     elapsed = max_over_ranks(elapsed, world)
     code = atlas.last_device_error(stream)
     if code:
         raise RuntimeError(f"device error word 0x{code:x} in the timed region")
+
+    if args.proj:
+        return report_proj(args, world, rank, path, elapsed, phases, clk)
 
     # end to end through the C-ABI with host buffers
     e2e = None
@@ -638,6 +736,46 @@ def run_atlas(args, world, rank, local):
     print(json.dumps(out), flush=True)
 
 
+def report_proj(args, world, rank, path, elapsed, phases, clk):
+    """JSON line of a --proj run: the whole step's FLOPs (projections +
+    attention), the fused projections' TFLOP/s and roofline, and the unfused
+    comparison."""
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    ms = elapsed / args.steps
+    f_qkv, f_out = path.proj_flops()
+    f_attn = path.flops()
+    med = lambda k: statistics.median(phases[k])
+    qkv_ms = med("qkv_d") + med("qkv_g")
+    out_ms = med("out")
+    proj_tf = (f_qkv + f_out) / ((qkv_ms + out_ms) * 1e-3) / 1e12
+    un_qkv, un_out = path.unfused_ms(min(args.steps, 10))
+    peak_tf = pk["bf16_tflops_sustained"]
+    out = {
+        "metric": METRIC + " (with fused projections)", "value":
+            world * (f_qkv + f_out + f_attn) / (ms * 1e-3) / 1e12, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded inputs, random weights)",
+        "config": dict(config_of(path.w, world), model_width=path.C, projections="fused"),
+        "qkv_proj_ms": qkv_ms, "out_proj_ms": out_ms, "attn_ms": med("attn"),
+        "qkv_proj_tflops": f_qkv / (qkv_ms * 1e-3) / 1e12,
+        "out_proj_tflops": f_out / (out_ms * 1e-3) / 1e12,
+        "attn_tflops": f_attn / (med("attn") * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "gemm_proj_kernel (QKV + output projections)",
+                     "achieved": proj_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": proj_tf / peak_tf, "peak_kind": f"{pk_kind} bf16 sustained"},
+        "unfused_detail_ms": {"qkv_cublas_plus_reorder": un_qkv,
+                              "unorder_plus_cublas_out": un_out,
+                              "fused_qkv_detail": med("qkv_d"), "fused_out_detail_and_global":
+                                  out_ms},
+        "gpu_launches": path.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(out), flush=True)
+
+
 def run_e2e(path, w, dev, stream, args, world):
     """Same step, but inputs start in pinned host memory and the outputs end
     there: H2D of the six raster tensors, the seven calls, D2H of O_d and O_g."""
@@ -697,6 +835,9 @@ def main():
                          "only; raster / dense: comparison modes (naive raster-order blocks, "
                          "full attention)")
     ap.add_argument("--batch", type=int, default=1, help="problems per GPU")
+    ap.add_argument("--proj", action="store_true",
+                    help="include the QKV and output projections, fused with the reorder, "
+                         "RoPE and unorder (random weights, model width heads*head_dim)")
     ap.add_argument("--backward", action="store_true",
                     help="time a training step: the forward path plus its backward (gradients "
                          "w.r.t. the raster inputs); value counts the backward as 2.5x the "

@@ -389,6 +389,48 @@ atlas_status atlas_cube_unorder_rope(const void *src, void *dst, int64_t batch,
                                      int32_t head_dim, atlas_dtype dtype,
                                      const atlas_rope *rope, atlas_stream_t stream);
 
+/*
+ * atlas_qkv_proj_reorder -- the QKV projection with steps (1) and (2) in its
+ * epilogue: [Q | K | V] = x w^T, Q and K rotated by 3D RoPE at each token's
+ * grid position, all three written in cube order.
+ *
+ * Passages: as atlas_cube_reorder; the projection is the attention layer's
+ * linear map (the summary's training strategy adapts the attention
+ * projections). A GEMM acts on rows independently, so writing its rows at
+ * their cube positions equals reordering its result. The rotation uses the
+ * fp32 accumulator: each output is rounded to bf16 once.
+ * x: [batch*T*H*W, c_in] bf16, raster order per problem. w: [3*heads*
+ * head_dim, c_in] bf16 (rows of W_q, then W_k, then W_v). q, k, v: outputs
+ * [batch*T*H*W, heads, head_dim] in cube order. rope: NULL for no rotation
+ * (the global proxy takes a 1x1x1 cube and its own scales). tcgen05 GEMM,
+ * fp32 accumulation.
+ * Requirements: dtype BF16; c_in a multiple of 64; heads*head_dim a multiple
+ * of 256; head_dim a multiple of 32; 16-byte aligned pointers.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, ALIAS (an output overlapping an
+ * input or another output), DEVICE, CUDA.
+ */
+atlas_status atlas_qkv_proj_reorder(const void *x, const void *w, int64_t batch,
+                                    atlas_grid3 grid, atlas_cube3 cube, int32_t c_in,
+                                    int32_t heads, int32_t head_dim, atlas_dtype dtype,
+                                    const atlas_rope *rope, void *q, void *k, void *v,
+                                    atlas_stream_t stream);
+
+/*
+ * atlas_out_proj_unorder -- the output projection with the exact inverse of
+ * step (1) in its epilogue: y = unorder(o) w^T, computed as o w^T with each
+ * row written at its raster position.
+ *
+ * o: [batch*T*H*W, c_in] bf16 in cube order (c_in = heads*head_dim, the
+ * attention output viewed as rows). w: [c_out, c_in] bf16. y: [batch*T*H*W,
+ * c_out] bf16, raster order. Requirements: dtype BF16; c_in a multiple of 64;
+ * c_out a multiple of 256; 16-byte aligned pointers. Errors as
+ * atlas_qkv_proj_reorder.
+ */
+atlas_status atlas_out_proj_unorder(const void *o, const void *w, int64_t batch,
+                                    atlas_grid3 grid, atlas_cube3 cube, int32_t c_in,
+                                    int32_t c_out, atlas_dtype dtype, void *y,
+                                    atlas_stream_t stream);
+
 /* Human-readable name of a status. Never NULL. */
 const char *atlas_status_string(atlas_status status);
 

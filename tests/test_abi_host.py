@@ -273,3 +273,35 @@ def test_attention_bwd_validation(lib):
     import torch
     if not torch.cuda.is_available():
         assert call() == atlas.ERR_DEVICE
+
+
+def test_projection_validation(lib):
+    G3, C3 = atlas.Grid3, atlas.Cube3
+    x, w = FAKE, FAKE + (1 << 30)
+    q, k, v = FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (4 << 30)
+
+    def qkv(x=x, w=w, batch=1, grid=G3(4, 8, 8), c_in=256, heads=2, hd=128, dt=atlas.BF16,
+            q=q, k=k, v=v, rope=None):
+        return lib.atlas_qkv_proj_reorder(x, w, batch, grid, C3(2, 4, 4), c_in, heads, hd, dt,
+                                          ctypes.byref(rope) if rope else None, q, k, v, None)
+    assert qkv(x=None) == atlas.ERR_NULL
+    assert qkv(v=None) == atlas.ERR_NULL
+    assert qkv(batch=0) == atlas.ERR_SHAPE
+    assert qkv(dt=atlas.FP32) == atlas.ERR_UNSUPPORTED
+    assert qkv(c_in=96) == atlas.ERR_UNSUPPORTED            # not a multiple of 64
+    assert qkv(heads=3, hd=64) == atlas.ERR_UNSUPPORTED     # 192 not a multiple of 256
+    assert qkv(q=q + 8) == atlas.ERR_ALIGN
+    assert qkv(k=q + 64) == atlas.ERR_ALIAS                 # k over q
+    assert qkv(q=x) == atlas.ERR_ALIAS                      # q over x
+    assert qkv(rope=atlas.make_rope(10000, (44, 42, 40), (1, 1, 1))) == atlas.ERR_UNSUPPORTED
+
+    def out(o=x, w=w, c_in=256, c_out=512, y=q, dt=atlas.BF16):
+        return lib.atlas_out_proj_unorder(o, w, 1, G3(4, 8, 8), C3(2, 4, 4), c_in, c_out, dt, y,
+                                          None)
+    assert out(y=None) == atlas.ERR_NULL
+    assert out(c_out=300) == atlas.ERR_UNSUPPORTED
+    assert out(y=w) == atlas.ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        assert qkv() == atlas.ERR_DEVICE
+        assert out() == atlas.ERR_DEVICE

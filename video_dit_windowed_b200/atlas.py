@@ -92,6 +92,13 @@ def _declare(lib):
     lib.atlas_local_global_attn_bwd.argtypes = (
         [_vp] * 5 + [_i64] + [_vp] * 5 + [_i64, ctypes.POINTER(AttnLayout), _i32, _i32,
                                          ctypes.c_float, ctypes.c_int, _vp, _vp] + [_vp] * 7)
+    lib.atlas_qkv_proj_reorder.restype = ctypes.c_int
+    lib.atlas_qkv_proj_reorder.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32, _i32,
+                                           ctypes.c_int, ctypes.POINTER(Rope), _vp, _vp, _vp,
+                                           _vp]
+    lib.atlas_out_proj_unorder.restype = ctypes.c_int
+    lib.atlas_out_proj_unorder.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
+                                           ctypes.c_int, _vp, _vp]
     lib.atlas_aligned_global_cube.restype = ctypes.c_int
     lib.atlas_aligned_global_cube.argtypes = [Grid3, Cube3, Grid3, ctypes.POINTER(Cube3)]
     lib.atlas_cube_reorder_batched.restype = ctypes.c_int
@@ -329,6 +336,32 @@ def local_global_attn_bwd(q_d, k_d, v_d, o_d, do_d, q_g, k_g, v_g, o_g, do_g, ls
         nz(dk_g, n_g), nz(dv_g, n_g), _stream(ref, stream))
     _check(st, "atlas_local_global_attn_bwd")
     return dq_d, dk_d, dv_d, dq_g, dk_g, dv_g
+
+
+def qkv_proj_reorder(x, w, grid, cube, q, k, v, rope: Rope | None = None, batch=1,
+                     stream=None):
+    """[Q | K | V] = x w^T with RoPE on Q and K and every row written at its
+    cube position. x [batch*T*H*W, C] raster order; w [3*heads*head_dim, C];
+    q, k, v [batch*T*H*W, heads, head_dim] (outputs)."""
+    heads, hd = q.shape[1], q.shape[2]
+    st = lib().atlas_qkv_proj_reorder(
+        _ptr(x), _ptr(w), int(batch), Grid3(*grid), Cube3(*cube), x.shape[1], heads, hd,
+        _dtype_code(x), ctypes.byref(rope) if rope is not None else None, _ptr(q), _ptr(k),
+        _ptr(v), _stream(x, stream))
+    _check(st, "atlas_qkv_proj_reorder")
+    return q, k, v
+
+
+def out_proj_unorder(o, w, grid, cube, y, batch=1, stream=None):
+    """y = unorder(o) w^T: o [batch*T*H*W, heads, head_dim] (or [rows, C_in])
+    in cube order, w [C_out, C_in], y [batch*T*H*W, C_out] raster order."""
+    rows = o.shape[0]
+    c_in = o.numel() // rows if rows else w.shape[1]
+    st = lib().atlas_out_proj_unorder(_ptr(o), _ptr(w), int(batch), Grid3(*grid), Cube3(*cube),
+                                      c_in, y.shape[1], _dtype_code(o), _ptr(y),
+                                      _stream(o, stream))
+    _check(st, "atlas_out_proj_unorder")
+    return y
 
 
 def aligned_global_cube(grid, cube, global_grid):

@@ -427,6 +427,71 @@ ATLAS_API atlas_status atlas_local_global_attn_bwd(
                                         stream);
 }
 
+namespace atlas {
+namespace {
+
+// Shared checks of the two projection entry points.
+atlas_status check_proj(const void *x, const void *w, int64_t batch, atlas_grid3 grid,
+                        atlas_cube3 cube, int32_t c_in, atlas_dtype dtype) {
+    if (!x || !w) return ATLAS_ERR_NULL;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1 || batch < 1 || c_in < 1) return ATLAS_ERR_SHAPE;
+    if (grid.T > kMaxRows || grid.H > kMaxRows || grid.W > kMaxRows ||
+        grid.T * grid.H > kMaxRows || grid.T * grid.H * grid.W > kMaxRows / batch)
+        return ATLAS_ERR_SHAPE;
+    atlas_status st = check_cube(grid, cube);
+    if (st != ATLAS_OK) return st;
+    if (dtype != ATLAS_BF16 || c_in % 64 != 0) return ATLAS_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w)) return ATLAS_ERR_ALIGN;
+    return ATLAS_OK;
+}
+
+}  // namespace
+}  // namespace atlas
+
+ATLAS_API atlas_status atlas_qkv_proj_reorder(const void *x, const void *w, int64_t batch,
+                                              atlas_grid3 grid, atlas_cube3 cube, int32_t c_in,
+                                              int32_t heads, int32_t head_dim, atlas_dtype dtype,
+                                              const atlas_rope *rope, void *q, void *k, void *v,
+                                              atlas_stream_t stream) {
+    atlas_status st = atlas::check_proj(x, w, batch, grid, cube, c_in, dtype);
+    if (st != ATLAS_OK) return st;
+    if (!q || !k || !v) return ATLAS_ERR_NULL;
+    if (heads < 1 || head_dim < 1) return ATLAS_ERR_SHAPE;
+    if (head_dim % 32 != 0 || (static_cast<int64_t>(heads) * head_dim) % 256 != 0 ||
+        static_cast<int64_t>(heads) * head_dim * 3 > (1ll << 30))
+        return ATLAS_ERR_UNSUPPORTED;
+    if (rope && (st = atlas::check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (!atlas::aligned16(q) || !atlas::aligned16(k) || !atlas::aligned16(v)) return ATLAS_ERR_ALIGN;
+    const size_t rows = static_cast<size_t>(batch * grid.T * grid.H * grid.W);
+    const size_t bx = rows * c_in * 2, bw = static_cast<size_t>(3) * heads * head_dim * c_in * 2;
+    const size_t bo = rows * heads * head_dim * 2;
+    const atlas::Span all[] = {{x, bx}, {w, bw}, {q, bo}, {k, bo}, {v, bo}};
+    for (int i = 2; i < 5; ++i)
+        if (atlas::overlaps_any(all[i], all, 5)) return ATLAS_ERR_ALIAS;
+    atlas::ProjArgs a{x, w, batch, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw, c_in, 0,
+                      heads, head_dim, rope, {q, k, v}};
+    return atlas::launch_qkv_proj(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ATLAS_API atlas_status atlas_out_proj_unorder(const void *o, const void *w, int64_t batch,
+                                              atlas_grid3 grid, atlas_cube3 cube, int32_t c_in,
+                                              int32_t c_out, atlas_dtype dtype, void *y,
+                                              atlas_stream_t stream) {
+    atlas_status st = atlas::check_proj(o, w, batch, grid, cube, c_in, dtype);
+    if (st != ATLAS_OK) return st;
+    if (!y) return ATLAS_ERR_NULL;
+    if (c_out < 1) return ATLAS_ERR_SHAPE;
+    if (c_out % 256 != 0) return ATLAS_ERR_UNSUPPORTED;
+    if (!atlas::aligned16(y)) return ATLAS_ERR_ALIGN;
+    const size_t rows = static_cast<size_t>(batch * grid.T * grid.H * grid.W);
+    const atlas::Span all[] = {{o, rows * c_in * 2}, {w, static_cast<size_t>(c_out) * c_in * 2},
+                               {y, rows * c_out * 2}};
+    if (atlas::overlaps_any(all[2], all, 3)) return ATLAS_ERR_ALIAS;
+    atlas::ProjArgs a{o, w, batch, grid.T, grid.H, grid.W, cube.ct, cube.ch, cube.cw, c_in,
+                      c_out, 0, 0, nullptr, {y, nullptr, nullptr}};
+    return atlas::launch_out_proj(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 ATLAS_API atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 cube,
                                                  atlas_grid3 global_grid,
                                                  atlas_cube3 *global_cube) {

@@ -74,6 +74,23 @@ struct PermuteArgs {
 };
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
 atlas_status release_rope_tables();
+// The cached cos/sin table of `rope` on a T x H x W grid, current device
+// (layout: axis t [t][k], then h, then w; fp64 angles rounded to fp32).
+atlas_status rope_table_for(int64_t T, int64_t H, int64_t W, const atlas_rope &rope,
+                            const float2 **out);
+
+// Projections with the path's permutation in the GEMM epilogue (bf16).
+struct ProjArgs {
+    const void *x, *w;          // x [batch*T*H*W, c_in]; w [n_out, c_in]
+    int64_t batch, T, H, W;
+    int32_t ct, ch, cw;
+    int32_t c_in, c_out;        // c_out: OUT only
+    int32_t heads, head_dim;    // QKV only
+    const atlas_rope *rope;     // QKV only, may be NULL
+    void *out[3];               // QKV: q, k, v; OUT: y
+};
+atlas_status launch_qkv_proj(const ProjArgs &a, cudaStream_t stream);
+atlas_status launch_out_proj(const ProjArgs &a, cudaStream_t stream);
 // Reorder (+RoPE) with the cos/sin table in a fixed device array (no
 // allocation); ATLAS_ERR_CAPACITY if the table would not fit.
 atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stream);
