@@ -61,7 +61,7 @@ def _declare(lib):
     lib.atlas_oracle_cube_positions.argtypes = [_i64] * 6 + [_ptr]
     for name in ("atlas_oracle_cube_reorder", "atlas_oracle_cube_unorder"):
         fn = getattr(lib, name)
-        fn.restype = None
+        fn.restype = ctypes.c_int
         fn.argtypes = [_ptr, _ptr] + [_i64] * 7
     lib.atlas_oracle_rope3d_rows.restype = None
     lib.atlas_oracle_rope3d_rows.argtypes = (
@@ -140,7 +140,8 @@ class Oracle:
             raise ValueError("leading dim must be T*H*W")
         out = np.empty_like(x)
         row_bytes = x.nbytes // max(1, x.shape[0])
-        fn(x.ctypes.data, out.ctypes.data, T, H, W, *cube, row_bytes)
+        if fn(x.ctypes.data, out.ctypes.data, T, H, W, *cube, row_bytes) != 0:
+            raise RuntimeError("cube positions are not a permutation")
         return out
 
     def cube_reorder(self, x: np.ndarray, grid, cube) -> np.ndarray:

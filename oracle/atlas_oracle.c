@@ -119,30 +119,36 @@ void atlas_oracle_cube_positions(int64_t T, int64_t H, int64_t W,
 }
 
 /* dst[position(r)] = src[r], row by row, as a byte copy: every bit pattern
- * survives, so the inverse below restores the input exactly. */
-void atlas_oracle_cube_reorder(const unsigned char *src, unsigned char *dst,
-                               int64_t T, int64_t H, int64_t W,
-                               int64_t ct, int64_t ch, int64_t cw,
-                               int64_t row_bytes)
+ * survives, so the inverse below restores the input exactly. Returns 0, or
+ * 3 if a position falls outside the grid (defensive; cannot happen with a
+ * correct position map). */
+int atlas_oracle_cube_reorder(const unsigned char *src, unsigned char *dst,
+                              int64_t T, int64_t H, int64_t W,
+                              int64_t ct, int64_t ch, int64_t cw,
+                              int64_t row_bytes)
 {
     int64_t n = T * H * W;
     for (int64_t r = 0; r < n; ++r) {
         int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        if (j < 0 || j >= n) return 3;
         memcpy(dst + j * row_bytes, src + r * row_bytes, (size_t)row_bytes);
     }
+    return 0;
 }
 
-/* The exact inverse: dst[r] = src[position(r)]. */
-void atlas_oracle_cube_unorder(const unsigned char *src, unsigned char *dst,
-                               int64_t T, int64_t H, int64_t W,
-                               int64_t ct, int64_t ch, int64_t cw,
-                               int64_t row_bytes)
+/* The exact inverse: dst[r] = src[position(r)]. Returns as the reorder. */
+int atlas_oracle_cube_unorder(const unsigned char *src, unsigned char *dst,
+                              int64_t T, int64_t H, int64_t W,
+                              int64_t ct, int64_t ch, int64_t cw,
+                              int64_t row_bytes)
 {
     int64_t n = T * H * W;
     for (int64_t r = 0; r < n; ++r) {
         int64_t j = atlas_oracle_cube_position(T, H, W, ct, ch, cw, r);
+        if (j < 0 || j >= n) return 3;
         memcpy(dst + r * row_bytes, src + j * row_bytes, (size_t)row_bytes);
     }
+    return 0;
 }
 
 /* ------------------------------------------------------------------------ */
