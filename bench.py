@@ -630,8 +630,10 @@ def run_atlas(args, world, rank, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
+        mem0 = torch.cuda.memory_allocated(dev)
         path = (ProjPath(w, dev, stream) if args.proj
                 else Path(w, dev, stream, args.mask, args.batch, args.backward))
+        path_bytes = torch.cuda.memory_allocated(dev) - mem0
     torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         path.step()
@@ -674,7 +676,15 @@ def run_atlas(args, world, rank, local):
     # end to end through the C-ABI with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(path, w, dev, stream, args, world)
+        # a second buffer set for the pipelined run, if the device holds two
+        twin = None
+        free, total = torch.cuda.mem_get_info(dev)
+        if path_bytes < 0.8 * free:
+            with torch.cuda.stream(stream):
+                twin = Path(w, dev, stream, args.mask, args.batch, args.backward)
+            torch.cuda.synchronize(dev)
+        e2e = run_e2e(path, w, dev, stream, args, world, twin)
+        del twin
 
     if rank != 0:
         return
@@ -776,48 +786,92 @@ def report_proj(args, world, rank, path, elapsed, phases, clk):
     print(json.dumps(out), flush=True)
 
 
-def run_e2e(path, w, dev, stream, args, world):
-    """Same step, but inputs start in pinned host memory and the outputs end
-    there: H2D of the six raster tensors, the seven calls, D2H of O_d and O_g."""
-    dev_in = dict(path.x)
-    if path.backward:
-        dev_in.update({"do_d": path.do["d"], "do_g": path.do["g"]})
-    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in dev_in.items()}
+def run_e2e(path, w, dev, stream, args, world, twin=None):
+    """The same step through the C-ABI with host buffers: every step uploads
+    its inputs from pinned host memory (the six raster tensors; with
+    --backward also dO) and downloads its results (O_d and O_g; with
+    --backward also the six gradients). With ``twin`` (a second set of device
+    buffers) the steps are pipelined: step i+1's upload (one copy stream) and
+    step i-1's download (another) overlap step i's compute; each step still
+    carries its own copies. Without it the copies and the compute of a step
+    run in order on one stream."""
+    paths = [path] + ([twin] if twin is not None else [])
+
+    def dev_inputs(p):
+        d = dict(p.x)
+        if p.backward:
+            d.update({"do_d": p.do["d"], "do_g": p.do["g"]})
+        return d
+
+    def results(p):
+        r = list(p.outputs())
+        if p.backward:
+            r += p.gradients()
+        return r
+
+    ins = [dev_inputs(p) for p in paths]
+    res = [results(p) for p in paths]
+    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in ins[0].items()}
     for k in host:
-        host[k].copy_(dev_in[k].cpu())
-    res = list(path.outputs())
-    if path.backward:
-        res += path.gradients()
-    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in res]
+        host[k].copy_(ins[0][k].cpu())
+    outs = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in r] for r in res]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs)
+    d2h = sum(t.numel() * t.element_size() for t in outs[0])
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
+    n_sets = len(paths)
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev() for _ in range(n_sets)]
+    comp_done = [ev() for _ in range(n_sets)]
+    out_done = [ev() for _ in range(n_sets)]
 
-    def one():
-        with torch.cuda.stream(stream):
+    def one(i):
+        b = i % n_sets
+        if n_sets == 1:
+            with torch.cuda.stream(stream):
+                for k in host:
+                    ins[0][k].copy_(host[k], non_blocking=True)
+                paths[0].step()
+                for o, t in zip(outs[0], res[0]):
+                    o.copy_(t, non_blocking=True)
+            return
+        with torch.cuda.stream(up):
+            if i >= n_sets:
+                up.wait_event(comp_done[b])        # set b's inputs are free again
             for k in host:
-                dev_in[k].copy_(host[k], non_blocking=True)
-            path.step()
-            for o, t in zip(outs, res):
+                ins[b][k].copy_(host[k], non_blocking=True)
+            in_ready[b].record(up)
+        stream.wait_event(in_ready[b])
+        if i >= n_sets:
+            stream.wait_event(out_done[b])         # set b's results were read
+        paths[b].step()
+        comp_done[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(comp_done[b])
+            for o, t in zip(outs[b], res[b]):
                 o.copy_(t, non_blocking=True)
+            out_done[b].record(down)
 
-    for _ in range(min(args.warmup, 3)):
-        one()
+    for i in range(min(args.warmup, 3)):
+        one(i)
     torch.cuda.synchronize(dev)
     steps = max(1, min(args.steps, 10))
     barrier(world)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    first = up if n_sets > 1 else stream
+    last = down if n_sets > 1 else stream
+    t0.record(first)
+    for i in range(steps):
+        one(i)
+    t1.record(last)
     torch.cuda.synchronize(dev)
     barrier(world)
-    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
     step_flops = path.flops() * 7 // 2 if path.backward else path.flops()
     return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": UNIT,
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": steps}
+            "steps": steps, "pipelined": n_sets > 1}
 
 
 def main():
