@@ -80,6 +80,10 @@ def _declare(lib):
     lib.atlas_oracle_attention_bwd_head_aligned.restype = ctypes.c_int
     lib.atlas_oracle_attention_bwd_head_aligned.argtypes = (
         [_i64] * 10 + [_f64] + [_ptr] * 7 + [ctypes.c_int])
+    lib.atlas_oracle_attention_bwd_head_sampled.restype = ctypes.c_int
+    lib.atlas_oracle_attention_bwd_head_sampled.argtypes = (
+        [_i64, _i64, _ptr, _i64, _i64, _i64, _f64] + [_ptr] * 4 + [_i64, _ptr, _i64, _ptr]
+        + [_ptr] * 3 + [ctypes.c_int])
     lib.atlas_oracle_attention_head.restype = ctypes.c_int
     lib.atlas_oracle_attention_head.argtypes = (
         [_i64, _i64, _i64, _i64, _f64, _ptr, _ptr, _i64, _i64, _ptr, _ptr,
@@ -329,6 +333,32 @@ class Oracle:
         f = lambda D, *p: self.lib.atlas_oracle_attention_bwd_head_windows(
             N, window_len, off_ptr, n_win, G, D, float(scale), *p, int(n_threads))
         return self._bwd(f, q_d, k_d, v_d, q_g, k_g, v_g, do_d, do_g)
+
+    def attention_bwd_sampled(self, q, k, v, do, n_detail, window_len, scale, q_rows, k_rows,
+                              n_threads: int = 1, win_off=None):
+        """One head, all N+G rows given ([N+G, D] each, detail rows first):
+        dq for the query rows ``q_rows`` and (dk, dv) for the key rows
+        ``k_rows``; returns (dq [len(q_rows), D], dk, dv [len(k_rows), D])."""
+        f = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+        q, k, v, do = f(q), f(k), f(v), f(do)
+        R, D = q.shape
+        qs = np.ascontiguousarray(np.asarray(q_rows, dtype=np.int64))
+        ks = np.ascontiguousarray(np.asarray(k_rows, dtype=np.int64))
+        dq = np.empty((qs.size, D))
+        dk = np.empty((ks.size, D))
+        dv = np.empty((ks.size, D))
+        if win_off is not None:
+            off = np.ascontiguousarray(np.asarray(win_off, dtype=np.int64))
+            off_ptr, n_win = off.ctypes.data, off.size - 1
+        else:
+            off, off_ptr, n_win = None, None, 0
+        st = self.lib.atlas_oracle_attention_bwd_head_sampled(
+            n_detail, window_len, off_ptr, n_win, R - n_detail, D, float(scale), q.ctypes.data,
+            k.ctypes.data, v.ctypes.data, do.ctypes.data, qs.size, qs.ctypes.data, ks.size,
+            ks.ctypes.data, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(n_threads))
+        if st != 0:
+            raise RuntimeError(f"oracle backward failed ({st})")
+        return dq, dk, dv
 
     def attention_bwd_full_aligned(self, q_d, k_d, v_d, grid, cube, q_g, k_g, v_g, global_grid,
                                    do_d, do_g, scale, n_threads: int = 1):

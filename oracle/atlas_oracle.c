@@ -444,7 +444,8 @@ int atlas_oracle_attention_head(int64_t n_detail, int64_t window_len,
 static int attention_bwd_core(const struct mask *msk, int64_t n_global, int64_t D,
                               double scale, const double *q, const double *k,
                               const double *v, const double *dout, double *dq, double *dk,
-                              double *dv, int n_threads)
+                              double *dv, int64_t n_qsel, const int64_t *qsel,
+                              int64_t n_ksel, const int64_t *ksel, int n_threads)
 {
     int64_t R = msk->N + n_global;
     int status = 0;
@@ -452,6 +453,18 @@ static int attention_bwd_core(const struct mask *msk, int64_t n_global, int64_t 
     double *delta = (double *)malloc((size_t)(R > 0 ? R : 1) * sizeof(double));
     if (!lse || !delta) { free(lse); free(delta); return 2; }
     if (n_threads < 1) n_threads = 1;
+    /* pass 1: every query row's softmax statistics (the selected keys may be
+     * seen by any row), and dq for the selected rows (all rows without a
+     * selection) */
+    int64_t n_dq = qsel ? n_qsel : R;
+    char *want_dq = (char *)calloc((size_t)(R > 0 ? R : 1), 1);
+    int64_t *dq_slot = (int64_t *)malloc((size_t)(R > 0 ? R : 1) * sizeof(int64_t));
+    if (!want_dq || !dq_slot) { free(lse); free(delta); free(want_dq); free(dq_slot); return 2; }
+    for (int64_t a = 0; a < n_dq; ++a) {
+        int64_t i = qsel ? qsel[a] : a;
+        want_dq[i] = 1;
+        dq_slot[i] = a;
+    }
 #pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
     for (int64_t i = 0; i < R; ++i) {
         const double *qi = q + i * D, *gi = dout + i * D;
@@ -486,18 +499,26 @@ static int attention_bwd_core(const struct mask *msk, int64_t n_global, int64_t 
         double dl = 0.0;
         for (int64_t a = 0; a < n; ++a) dl += exp(logit[a] - lse[i]) * dp[a];
         delta[i] = dl;
-        for (int64_t d = 0; d < D; ++d) dq[i * D + d] = 0.0;
-        for (int64_t a = 0; a < n; ++a) {
-            double ds = exp(logit[a] - lse[i]) * (dp[a] - dl);
-            for (int64_t d = 0; d < D; ++d) dq[i * D + d] += scale * ds * k[key[a] * D + d];
+        if (want_dq[i]) {
+            double *dqi = dq + dq_slot[i] * D;
+            for (int64_t d = 0; d < D; ++d) dqi[d] = 0.0;
+            for (int64_t a = 0; a < n; ++a) {
+                double ds = exp(logit[a] - lse[i]) * (dp[a] - dl);
+                for (int64_t d = 0; d < D; ++d) dqi[d] += scale * ds * k[key[a] * D + d];
+            }
         }
         free(logit); free(dp); free(key);
     }
+    /* pass 2: dk and dv of the selected key rows (all rows without a
+     * selection), over every query allowed to see the key */
+    int64_t n_dk = ksel ? n_ksel : R;
     if (status == 0) {
 #pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
-        for (int64_t j = 0; j < R; ++j) {
+        for (int64_t a = 0; a < n_dk; ++a) {
+            int64_t j = ksel ? ksel[a] : a;
             const double *kj = k + j * D, *vj = v + j * D;
-            for (int64_t d = 0; d < D; ++d) { dk[j * D + d] = 0.0; dv[j * D + d] = 0.0; }
+            double *dkj = dk + a * D, *dvj = dv + a * D;
+            for (int64_t d = 0; d < D; ++d) { dkj[d] = 0.0; dvj[d] = 0.0; }
             for (int64_t i = 0; i < R; ++i) {
                 if (!allowed(msk, i, j)) continue;
                 double dot = 0.0, dpo = 0.0;
@@ -508,14 +529,16 @@ static int attention_bwd_core(const struct mask *msk, int64_t n_global, int64_t 
                 double p = exp(scale * dot - lse[i]);
                 double ds = p * (dpo - delta[i]);
                 for (int64_t d = 0; d < D; ++d) {
-                    dk[j * D + d] += scale * ds * q[i * D + d];
-                    dv[j * D + d] += p * dout[i * D + d];
+                    dkj[d] += scale * ds * q[i * D + d];
+                    dvj[d] += p * dout[i * D + d];
                 }
             }
         }
     }
     free(lse);
     free(delta);
+    free(want_dq);
+    free(dq_slot);
     return status;
 }
 
@@ -534,8 +557,31 @@ int atlas_oracle_attention_bwd_head_windows(int64_t n_detail, int64_t window_len
     m.L = window_len;
     m.win_off = win_off;
     m.n_win = n_win;
-    return attention_bwd_core(&m, n_global, head_dim, scale, q, k, v, dout, dq, dk, dv,
-                              n_threads);
+    return attention_bwd_core(&m, n_global, head_dim, scale, q, k, v, dout, dq, dk, dv, 0, NULL,
+                              0, NULL, n_threads);
+}
+
+/* Backward of one head, windows form, for selected rows only: dq for the
+ * n_qsel query rows qsel (written as n_qsel rows), dk and dv for the n_ksel
+ * key rows ksel. Inputs hold all N+G rows. Every row's softmax statistics
+ * are taken first, as the full version does. */
+int atlas_oracle_attention_bwd_head_sampled(int64_t n_detail, int64_t window_len,
+                                            const int64_t *win_off, int64_t n_win,
+                                            int64_t n_global, int64_t head_dim, double scale,
+                                            const double *q, const double *k, const double *v,
+                                            const double *dout, int64_t n_qsel,
+                                            const int64_t *qsel, int64_t n_ksel,
+                                            const int64_t *ksel, double *dq, double *dk,
+                                            double *dv, int n_threads)
+{
+    struct mask m;
+    memset(&m, 0, sizeof m);
+    m.N = n_detail;
+    m.L = window_len;
+    m.win_off = win_off;
+    m.n_win = n_win;
+    return attention_bwd_core(&m, n_global, head_dim, scale, q, k, v, dout, dq, dk, dv, n_qsel,
+                              qsel, n_ksel, ksel, n_threads);
 }
 
 /* Backward of one head of the aligned variant (geometry as
@@ -565,8 +611,8 @@ int atlas_oracle_attention_bwd_head_aligned(int64_t T, int64_t H, int64_t W,
         cube_of[j] = ((tt / ct) * nh + hh / ch) * nw + ww / cw;
     }
     m.cube_of = cube_of;
-    int st = attention_bwd_core(&m, t * h * w, head_dim, scale, q, k, v, dout, dq, dk, dv,
-                                n_threads);
+    int st = attention_bwd_core(&m, t * h * w, head_dim, scale, q, k, v, dout, dq, dk, dv, 0,
+                                NULL, 0, NULL, n_threads);
     free(cube_of);
     return st;
 }

@@ -754,7 +754,25 @@ def pin_out_proj_matches_loops(o):
 
 PROJ_PINS = [pin_proj_matches_loops, pin_out_proj_matches_loops]
 
-BWD_PINS = [pin_bwd_autograd_dense, pin_bwd_finite_differences, pin_bwd_single_token_windows]
+def pin_bwd_sampled_equals_full(o):
+    """Selected rows of the backward equal the same rows of the full one."""
+    grid, cube, G, heads, D = (2, 4, 8), (1, 2, 4), 11, 1, 8
+    N, qd, kd, vd, qg, kg, vg = _rand_case(grid, G, heads, D, 820)
+    dod = _rand_case(grid, G, heads, D, 821)[1]
+    dog = _rand_case(grid, G, heads, D, 822)[4]
+    full = o.attention_bwd_full(qd, kd, vd, 8, qg, kg, vg, dod, dog, 0.3)
+    cat = lambda a, b: np.concatenate([a[:, 0], b[:, 0]])
+    rows = np.array([0, 5, 17, N - 1, N, N + G - 1])
+    dq, dk, dv = o.attention_bwd_sampled(cat(qd, qg), cat(kd, kg), cat(vd, vg), cat(dod, dog),
+                                         N, 8, 0.3, rows, rows[::-1])
+    for got, a, b, sel in ((dq, full[0], full[3], rows), (dk, full[1], full[4], rows[::-1]),
+                           (dv, full[2], full[5], rows[::-1])):
+        ref = cat(a, b)[sel]
+        assert np.max(np.abs(got - ref)) < 1e-13
+
+
+BWD_PINS = [pin_bwd_autograd_dense, pin_bwd_finite_differences, pin_bwd_single_token_windows,
+            pin_bwd_sampled_equals_full]
 
 ATTN_PINS = [pin_attention_dense_sdpa, pin_attention_partial_cubes_dense_sdpa,
              pin_attention_aligned_dense_sdpa, pin_attention_aligned_counts,

@@ -205,3 +205,32 @@ def test_chain_backward_raster(dtype):
            o.cube_unorder(ref[2], grid, cube),
            rope(ref[3], gg, (-2, -2, -2)), rope(ref[4], gg, (-2, -2, -2)), ref[5]]
     assert_grads_close([f64(t) for t in r], ref, dtype, "chain")
+
+
+def test_backward_full_size_sampled():
+    """720p workload at full size (80,640 detail and 5,040 global tokens, 40
+    heads), the configuration bench.py --backward times: dQ of sampled query
+    rows and dK, dV of sampled key rows (detail keys of two windows, global
+    keys, whose gradients sum over every query) on the first and last head
+    against the oracle."""
+    from video_dit_windowed_b200.workloads import WORKLOADS
+    w = WORKLOADS["720p"]
+    torch.cuda.empty_cache()
+    N, L, G, heads, hd = w.n_detail, w.window_len, w.n_global, w.heads, w.head_dim
+    t = inputs(1, N, G, heads, hd, "bf16", seed=26)
+    got = run_gpu(t, 1, heads, N, G, window_len=L)
+    q_rows = np.concatenate([np.arange(0, 128), 57 * L + np.arange(300, 428), [N - 1],
+                             N + np.array([0, 1, 2500, G - 1])])
+    k_rows = np.concatenate([np.arange(0, 32), 104 * L + np.arange(700, 768),
+                             N + np.array([0, 77, 2500, G - 2, G - 1])])
+    for head in (0, heads - 1):
+        cat = lambda a, b: np.concatenate([f64(a[:, head]), f64(b[:, head])])
+        dq, dk, dv = orc().attention_bwd_sampled(
+            cat(t["q_d"], t["q_g"]), cat(t["k_d"], t["k_g"]), cat(t["v_d"], t["v_g"]),
+            cat(t["do_d"], t["do_g"]), N, L, hd ** -0.5, q_rows, k_rows, n_threads())
+        g_q = cat(got[0], got[3])[q_rows]
+        g_k = cat(got[1], got[4])[k_rows]
+        g_v = cat(got[2], got[5])[k_rows]
+        assert_grads_close([g_q, g_k, g_v], [dq, dk, dv], "bf16", f"720p head {head}")
+    del got, t
+    torch.cuda.empty_cache()

@@ -41,10 +41,10 @@ MUTANTS = [
      "memcpy(dst + j * row_bytes, src + r * row_bytes, (size_t)row_bytes);"),
     ("bwd_lse_missing_max", "lse[i] = log(sum) + m;", "lse[i] = log(sum);"),
     ("bwd_drops_delta", "double ds = p * (dpo - delta[i]);", "double ds = p * dpo;"),
-    ("bwd_dk_unscaled", "dk[j * D + d] += scale * ds * q[i * D + d];", "dk[j * D + d] += ds * q[i * D + d];"),
-    ("bwd_dv_uses_ds", "dv[j * D + d] += p * dout[i * D + d];", "dv[j * D + d] += ds * dout[i * D + d];"),
-    ("bwd_dq_wrong_key", "dq[i * D + d] += scale * ds * k[key[a] * D + d];",
-     "dq[i * D + d] += scale * ds * q[key[a] * D + d];"),
+    ("bwd_dk_unscaled", "dkj[d] += scale * ds * q[i * D + d];", "dkj[d] += ds * q[i * D + d];"),
+    ("bwd_dv_uses_ds", "dvj[d] += p * dout[i * D + d];", "dvj[d] += ds * dout[i * D + d];"),
+    ("bwd_dq_wrong_key", "dqi[d] += scale * ds * k[key[a] * D + d];",
+     "dqi[d] += scale * ds * q[key[a] * D + d];"),
     ("bwd_delta_unweighted", "dl += exp(logit[a] - lse[i]) * dp[a];", "dl += dp[a];"),
     ("dot_drops_last_channel", "for (int64_t d = 0; d < D; ++d) dot += qi[d] * kr[d];",
      "for (int64_t d = 0; d + 1 < D; ++d) dot += qi[d] * kr[d];"),
