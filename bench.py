@@ -574,8 +574,9 @@ def max_over_ranks(v, world):
     return float(t.item())
 
 
-def config_of(w, world, mask="all", batch=1, backward=False):
-    c = {"workload": w.name, "mask": mask, "pass": "forward+backward" if backward else "forward", "detail_grid": list(w.grid), "cube": list(w.cube),
+def config_of(w, world, mask="all", batch=1, backward=False, graph=False):
+    c = {"workload": w.name, "mask": mask, "pass": "forward+backward" if backward else "forward",
+         "launch": "cuda graph" if graph else "stream", "detail_grid": list(w.grid), "cube": list(w.cube),
          "global_grid": list(w.global_grid), "n_detail": w.n_detail, "window_len": w.window_len,
          "n_global": w.n_global, "heads": w.heads, "head_dim": w.head_dim,
          "rope_split": list(w.split), "detail_scales": list(w.detail_scales),
@@ -642,6 +643,18 @@ def run_atlas(args, world, rank, local):
     if code:
         raise RuntimeError(f"device error word 0x{code:x} after warm-up")
 
+    graph = None
+    n_ev = 8 if args.backward else 5
+    if args.graph:
+        # the whole step as one CUDA graph (the first calls above have cached
+        # every table and attribute), replayed once per timed step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            path.step()
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.5)            # let nvidia-smi start sampling before the timed region
@@ -650,11 +663,14 @@ def run_atlas(args, world, rank, local):
     t_wall0 = time.time()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
-    n_ev = 8 if args.backward else 5
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     start.record(stream)
     for i in range(args.steps):
-        path.step(evs[i])
+        if graph is not None:
+            with torch.cuda.stream(stream):       # replay() launches on the current stream
+                graph.replay()
+        else:
+            path.step(evs[i])
     stop.record(stream)
     torch.cuda.synchronize(dev)
     clocks.window(t_wall0, time.time())
@@ -662,6 +678,14 @@ def run_atlas(args, world, rank, local):
     clk = clocks.stop()
     elapsed = start.elapsed_time(stop)
     phases = {}
+    if graph is not None:
+        # phase times from eager steps after the timed region (events inside
+        # a graph cannot be timed)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+               for _ in range(min(args.steps, 10))]
+        for ev in evs:
+            path.step(ev)
+        torch.cuda.synchronize(dev)
     for ev in evs:
         for k, v in type(path).phase_ms(ev).items():
             phases.setdefault(k, []).append(v)
@@ -706,7 +730,7 @@ def run_atlas(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world, args.mask, args.batch, args.backward),
+        "config": config_of(w, world, args.mask, args.batch, args.backward, args.graph),
         "attn_tflops": attn_tf, "attn_ms": attn_ms,
         "attn_frac_of_bf16_peak": {"sustained": attn_tf / pk["bf16_tflops_sustained"],
                                    "burst": attn_tf / pk["bf16_tflops"], "peaks": pk_kind},
@@ -889,6 +913,9 @@ def main():
                          "only; raster / dense: comparison modes (naive raster-order blocks, "
                          "full attention)")
     ap.add_argument("--batch", type=int, default=1, help="problems per GPU")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step in a CUDA graph and time its replays (phase times "
+                         "come from eager steps after the timed region)")
     ap.add_argument("--proj", action="store_true",
                     help="include the QKV and output projections, fused with the reorder, "
                          "RoPE and unorder (random weights, model width heads*head_dim)")
