@@ -464,11 +464,18 @@ class ProjPath:
 
 
 def kernel_source_hash():
+    """Hash of the attention kernel's source with comments and whitespace
+    removed: a comment edit keeps the stored traffic valid, a code edit does
+    not."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "video_dit_windowed_b200", "csrc")
     for name in ("attn_tc.cu", "sm100_ptx.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,12 +7,18 @@
 // global keys; global -> detail is masked with -inf).
 //
 // One softmax per query row over its allowed keys, flash style:
-//   * a work unit is one head and 256 consecutive query rows (two 128-row Q
-//     tiles), either detail rows (cube order) or global rows;
+//   * a work unit is one head of one problem (a batch stacks problems along
+//     the rows) and 256 consecutive query rows (two 128-row Q tiles), either
+//     detail rows (cube order) or global rows;
 //   * its key list is the detail rows of the windows its queries belong to
-//     (128-key tiles from the first window's start), then all global keys;
-//     detail units of windows that are multiples of 256 rows see exactly
-//     their own window, otherwise per-row masks cut the tile;
+//     (128-key tiles from the first window's start), then the global keys of
+//     its problem: all of them, or in the aligned variant the union of its
+//     windows' global ranges; per-row masks cut tiles that straddle a range
+//     edge, so units of windows that are multiples of 256 rows see exactly
+//     their own window;
+//   * windows are L rows or the ranges of an offsets array (partial cubes);
+//     ranges from offsets are clamped so that any offsets keep every access
+//     in bounds;
 //   * persistent CTAs (one per SM) walk the units head-major, so the CTAs in
 //     flight share one head's global K/V in L2.
 // Warp roles per CTA (384 threads):

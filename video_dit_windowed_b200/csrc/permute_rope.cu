@@ -12,7 +12,9 @@
 // its cos/sin table entries, are the same for every head of the row) and
 // moves that slot for heads hg, hg + 128/vph, ... with all loads of a row in
 // flight before the first store. Row index arithmetic (cube <-> raster) is
-// done once per row per thread with multiply-shift division.
+// done once per row per thread with multiply-shift division (the index math
+// itself is in cube_geom.cuh). A batch of problems of one grid is one launch:
+// output row rr belongs to problem rr / (T*H*W) and is permuted inside it.
 #include <cuda_bf16.h>
 
 #include <algorithm>
