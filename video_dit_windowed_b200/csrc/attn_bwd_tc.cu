@@ -16,6 +16,10 @@
 //           of the queries that may see those keys (for a detail key, its
 //           window's queries; for a global key, the detail queries that see
 //           it and every global query); accumulates dV and dK.
+// The DQ form keeps its resident Q and dO rows in tensor memory (written by
+// the compute threads), so its S and dP MMAs read only the streamed half
+// from shared memory (TS form); DKDV has no tensor memory to spare for K and
+// V and reads them from shared memory (SS form).
 // Either way a streamed tile of 128 rows is taken in two halves of 64, each
 // loaded into its own stage of the shared-memory ring (so three halves can
 // be in flight while one is used; the streamed queries' LSE and delta ride in
@@ -33,10 +37,10 @@
 // the other. Two compute warpgroups share the work: thread r of warpgroup g
 // takes resident row r and columns 32g .. 32g+31 of each half (and, in the
 // epilogue, half of the accumulator columns). Tensor memory:
-// S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc (DQ: dQ, then dS packed;
-// DKDV: dV, dK). In DKDV the packed P and dS overwrite the first half of
-// S_h and dP_h, which the other warpgroup may still be reading: the two
-// groups meet on an mbarrier between their loads and their stores.
+// S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc (DQ: dQ, then the
+// resident Q and dO; DKDV: dV, dK). The packed P and dS overwrite the first
+// half of S_h and dP_h, which the other warpgroup may still be reading: the
+// two groups meet on an mbarrier between their loads and their stores.
 // Every wait is bounded, as in the forward kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -88,6 +92,7 @@ struct Params {
     CUtensorMap tm_q[2], tm_k[2], tm_v[2], tm_do[2];   // 128-row boxes; [0] detail, [1] global
     CUtensorMap hm_q[2], hm_k[2], hm_v[2], hm_do[2];   // the same with 64-row boxes
     __nv_bfloat16 *out0[2], *out1[2];   // DQ: dq (out0); DKDV: dv (out0), dk (out1)
+    const __nv_bfloat16 *res_x[2], *res_y[2];   // DQ: Q and dO rows (resident in TMEM)
     const float *lse, *delta;
     uint32_t *err_word;
     int32_t N, L, G, heads, batch;      // N, G: rows of ONE problem
@@ -279,14 +284,15 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
     for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
         const Unit U = decode_unit<FORM>(p, u);
         // Every lane waits and the warp agrees, so the lanes never diverge
-        // around the warp-wide steps below.
-        if (unit_iter > 0 &&
+        // around the warp-wide steps below. (DQ: the compute warps put the
+        // resident Q and dO rows in tensor memory themselves.)
+        if (FORM == kDKDV && unit_iter > 0 &&
             !(ok = __all_sync(kAll, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
                                                kErrTimeoutProducer))))
             break;
         const int side = U.detail ? 0 : 1;
         const int32_t rbase = U.b * (U.detail ? p.N : p.G);
-        if (lane == 0) {
+        if (FORM == kDKDV && lane == 0) {
             const uint32_t bar = ptx::smem_addr(&sm.x_full);
             ptx::mbar_arrive_expect_tx(bar, 2 * kTile);
             tile(sm.x, FORM == kDQ ? &p.tm_q[side] : &p.tm_k[side], bar, U.head, rbase + U.r0,
@@ -294,7 +300,7 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
             tile(sm.y, FORM == kDQ ? &p.tm_do[side] : &p.tm_v[side], bar, U.head, rbase + U.r0,
                  kRows * 128);
         }
-        x_armed = unit_iter + 1;
+        if (FORM == kDKDV) x_armed = unit_iter + 1;
         const int32_t n = 2 * (U.n_a + U.n_b);   // half tiles
         for (int32_t jh = 0; jh < n && ok; ++jh, ++it) {
             const uint32_t s = it % kStages, round = it / kStages;
@@ -369,16 +375,26 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     uint32_t it = 0, unit_iter = 0, p_cnt = 0;
     bool ok = true;
 
+    const uint32_t t_x = t_acc + HD, t_y = t_x + HD / 2;   // DQ: resident Q, dO (packed)
     // S_h = X X'^T and dP_h = Y Y'^T from the half tile in stage s; commit.
+    // DKDV reads X, Y from shared memory (SS); DQ from tensor memory (TS), so
+    // only the streamed half is read from shared memory.
     auto issue_sdp = [&](int h, uint32_t s) {
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
             const uint32_t a_off = ((ks / 4) * (kRows * 128) + (ks % 4) * 32) >> 4;
             const uint32_t b_off = ((ks / 4) * (kHalf * 128) + (ks % 4) * 32) >> 4;
-            ptx::mma_ss(t_s + h * kHalf, ptx::desc_join(x_lo + a_off, kHi),
-                        ptx::desc_join(xs_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
-            ptx::mma_ss(t_dp + h * kHalf, ptx::desc_join(y_lo + a_off, kHi),
-                        ptx::desc_join(ys_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
+            if (FORM == kDQ) {
+                ptx::mma_ts(t_s + h * kHalf, t_x + ks * 8,
+                            ptx::desc_join(xs_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
+                ptx::mma_ts(t_dp + h * kHalf, t_y + ks * 8,
+                            ptx::desc_join(ys_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
+            } else {
+                ptx::mma_ss(t_s + h * kHalf, ptx::desc_join(x_lo + a_off, kHi),
+                            ptx::desc_join(xs_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
+                ptx::mma_ss(t_dp + h * kHalf, ptx::desc_join(y_lo + a_off, kHi),
+                            ptx::desc_join(ys_lo + s * kH16 + b_off, kHi), kIdS, ks > 0);
+            }
         }
         ptx::mma_commit(ptx::smem_addr(&sm.s_full[h]));
     };
@@ -420,7 +436,7 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                 ptx::tc_fence_after();
                 const bool first = j == 0 && h == 0;
                 if (FORM == kDQ) {
-                    issue_acc(t_acc, t_acc + HD + h * (kHalf / 2), xs_mn, st[h], first);
+                    issue_acc(t_acc, t_dp + h * kHalf, xs_mn, st[h], first);        // dQ
                 } else {
                     issue_acc(t_acc, t_s + h * kHalf, ys_mn, st[h], first);       // dV
                     issue_acc(t_acc + HD, t_dp + h * kHalf, xs_mn, st[h], first);  // dK
@@ -455,7 +471,7 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     const uint32_t lane_sel = ((warp & 3) * 32u) << 16;
     const uint32_t t_s = tmem + lane_sel, t_dp = tmem + 2 * kHalf + lane_sel;
     const uint32_t t_acc = tmem + 4 * kHalf + lane_sel;
-    const uint32_t t_ds = t_acc + HD;                 // DQ: packed dS_0 | dS_1
+    const uint32_t t_res = t_acc + HD + part * (HD / 2);   // DQ: this group's resident Q or dO
     const float c2 = p.scale_log2;
     uint32_t cnt = 0, unit_iter = 0;
 
@@ -496,6 +512,38 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         } else if (FORM == kDQ) {
             lse2_own = __builtin_huge_valf();
         }
+        if (FORM == kDQ) {
+            // Resident rows into tensor memory: warpgroup 0 the Q row,
+            // warpgroup 1 the dO row (bf16 pairs, element 2c in the low half
+            // of column c: the A-operand layout of the TS MMAs). Rows past
+            // the problem are zeros. The previous unit's MMAs must be done.
+            if (unit_iter > 0 &&
+                !__all_sync(kAll, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
+                                             kErrTimeoutSoftmax)))
+                return;
+            uint32_t rv[HD / 2];
+            if (valid) {
+                const int64_t abs_row = static_cast<int64_t>(U.b) * (U.detail ? p.N : p.G) + row;
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    (part == 0 ? p.res_x : p.res_y)[U.detail ? 0 : 1] +
+                    (abs_row * p.heads + U.head) * HD);
+#pragma unroll
+                for (int i = 0; i < HD / 8; ++i) {
+                    const uint4 w4 = __ldg(src + i);
+                    rv[4 * i] = w4.x;
+                    rv[4 * i + 1] = w4.y;
+                    rv[4 * i + 2] = w4.z;
+                    rv[4 * i + 3] = w4.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < HD / 2; ++i) rv[i] = 0u;
+            }
+            if constexpr (HD == 128) ptx::tmem_st64(t_res, rv);
+            else ptx::tmem_st32(t_res, rv);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&sm.x_full));
+        }
         const int32_t n = U.n_a + U.n_b;
         for (int32_t j = 0; j < n; ++j, ++cnt) {
             const bool det = streamed_detail(U, j);
@@ -515,7 +563,7 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                 uint32_t sv[kCols], dv[kCols];
                 ptx::tmem_ld32(t_s + h * kHalf + part * kCols, sv);
                 ptx::tmem_ld32(t_dp + h * kHalf + part * kCols, dv);
-                if (FORM == kDKDV) ptx::mbar_arrive(ptx::smem_addr(&sm.ld_done[h]));
+                ptx::mbar_arrive(ptx::smem_addr(&sm.ld_done[h]));
                 const int32_t c0 = base + h * kHalf + part * kCols;   // row of column 0
                 const bool partial = c0 < lo || c0 + kCols > hi;
                 uint32_t pk_p[kCols / 2], pk_ds[kCols / 2];
@@ -542,15 +590,12 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                     pk_ds[e] = ptx::pack_bf16x2(dsv[0], dsv[1]);
                 }
                 // packed pairs: this warpgroup's 32 values are columns 16g .. 16g+15
-                if (FORM == kDKDV) {
-                    if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], cnt & 1,
-                                                     kErrTimeoutSoftmax)))
-                        return;
-                    ptx::tmem_st16_nowait(t_s + h * kHalf + part * 16, pk_p);
-                    ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 16, pk_ds);
-                } else {
-                    ptx::tmem_st16_nowait(t_ds + h * (kHalf / 2) + part * 16, pk_ds);
-                }
+                // of the half's first 32, which the other group may still be
+                // reading: both groups' loads finish first.
+                if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], cnt & 1, kErrTimeoutSoftmax)))
+                    return;
+                if (FORM == kDKDV) ptx::tmem_st16_nowait(t_s + h * kHalf + part * 16, pk_p);
+                ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 16, pk_ds);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[h]));
@@ -606,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t warp = threadIdx.x / 32, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        ptx::mbar_init(ptx::smem_addr(&sm.x_full), 1);
+        ptx::mbar_init(ptx::smem_addr(&sm.x_full), FORM == kDQ ? kCompute : 1);
         ptx::mbar_init(ptx::smem_addr(&sm.x_empty), 1);
         for (int s = 0; s < Smem<HD>::kStages; ++s) {
             ptx::mbar_init(ptx::smem_addr(&sm.st_full[s]), 1);
@@ -720,6 +765,10 @@ atlas_status launch_hd(const AttnBwdArgs &b, const DeviceInfo &dev, cudaStream_t
     Params pq = p;
     pq.out0[0] = static_cast<__nv_bfloat16 *>(b.dq_d);
     pq.out0[1] = static_cast<__nv_bfloat16 *>(b.dq_g);
+    pq.res_x[0] = static_cast<const __nv_bfloat16 *>(a.q_d);
+    pq.res_x[1] = static_cast<const __nv_bfloat16 *>(a.q_g);
+    pq.res_y[0] = static_cast<const __nv_bfloat16 *>(b.do_d);
+    pq.res_y[1] = static_cast<const __nv_bfloat16 *>(b.do_g);
     atlas_status st = launch_form<HD, kDQ>(pq, dev, stream);
     if (st != ATLAS_OK) return st;
     Params pk = p;
