@@ -49,6 +49,7 @@ SMALL = [
     (1536, 768, 129, 1, 128, "bf16"),   # G one past a tile
     (1024, 128, 200, 3, 128, "bf16"),   # windows of exactly one tile
     (960, 48, 77, 2, 128, "bf16"),      # windows not aligned to tiles
+    (512, 1, 64, 2, 128, "bf16"),       # 1x1x1 cubes: each row sees itself and the globals
     (2048, 512, 300, 2, 64, "bf16"),    # head_dim 64
     (3072, 1536, 500, 1, 128, "bf16"),  # long windows
     (768, 768, 0, 2, 128, "bf16"),      # no global tokens (pure window attention)
