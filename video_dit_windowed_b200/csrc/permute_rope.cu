@@ -7,10 +7,11 @@
 //
 // The pass is HBM-bound: every destination row (heads*head_dim elements,
 // 10 KB for 40 heads x 128 bf16) is one contiguous read of its source row and
-// one contiguous write. Each 128-thread group owns one row at a time; a
+// one contiguous write. Each group of threads (32, 64 or 128 by row size)
+// owns one row at a time; a
 // thread owns a fixed 16-byte slot of the head (so its RoPE pairs, and hence
 // its cos/sin table entries, are the same for every head of the row) and
-// moves that slot for heads hg, hg + 128/vph, ... with all loads of a row in
+// moves that slot for heads hg, hg + G/vph, ... with all loads of a row in
 // flight before the first store. Row index arithmetic (cube <-> raster) is
 // done once per row per thread with multiply-shift division (the index math
 // itself is in cube_geom.cuh). A batch of problems of one grid is one launch:
@@ -54,8 +55,7 @@ struct Params {
     uint32_t half[3];       // d_axis / 2 for t, h, w
 };
 
-constexpr int kThreads = 256;     // two 128-thread row groups per block
-constexpr int kGroup = 128;
+constexpr int kThreads = 256;     // row groups of G threads per block (G = 128 or 32)
 constexpr int kMaxInFlight = 8;   // 16-byte loads in flight per thread per row
 
 __device__ __forceinline__ uint4 ld_stream(const uint8_t *p) {
@@ -119,8 +119,10 @@ __device__ __forceinline__ uint4 rotate<4>(uint4 v, const float2 *cs) {
 // row is rotated for the grid position (t, h, w) of its token, in every mode
 // (unorder + rotation with negated scales is the transpose of reorder +
 // rotation, i.e. its gradient).
-template <int EB, bool ROPE, int MODE>
+template <int EB, bool ROPE, int MODE, int G>
 __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) {
+    constexpr int kGroup = G;
+    constexpr uint32_t kGroups = kThreads / G;    // rows in flight per block
     constexpr int kPairs = 16 / EB / 2;  // RoPE pairs in one 16-byte vector
     const uint32_t tid = threadIdx.x & (kGroup - 1);
     const uint32_t group = threadIdx.x / kGroup;
@@ -143,7 +145,8 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) 
         }
     }
 
-    for (uint32_t rr = blockIdx.x * 2 + group; rr < p.total_rows; rr += gridDim.x * 2) {
+    for (uint32_t rr = blockIdx.x * kGroups + group; rr < p.total_rows;
+         rr += gridDim.x * kGroups) {
         // Problem b of the batch, and the row within it.
         const uint32_t b = p.by_rows.div(rr);
         const uint32_t row = rr - b * p.rows;
@@ -262,13 +265,25 @@ atlas_status rope_table(int device, int64_t T, int64_t H, int64_t W, const atlas
     return ATLAS_OK;
 }
 
-template <int EB, bool ROPE, int MODE>
-atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream) {
-    uint32_t blocks_needed = (p.total_rows + 1) / 2;
+template <int EB, bool ROPE, int MODE, int G>
+atlas_status launch_g(const Params &p, const DeviceInfo &dev, cudaStream_t stream) {
+    constexpr uint32_t kGroups = kThreads / G;
+    uint32_t blocks_needed = (p.total_rows + kGroups - 1) / kGroups;
     uint32_t grid = std::min<uint32_t>(blocks_needed, static_cast<uint32_t>(dev.sm_count) * 8u);
     if (grid == 0) return ATLAS_OK;
-    permute_rope_kernel<EB, ROPE, MODE><<<grid, kThreads, 0, stream>>>(p);
+    permute_rope_kernel<EB, ROPE, MODE, G><<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
+}
+
+// Group width by row size, so that a thread keeps several 16-byte loads in
+// flight: 128-thread groups for rows above 8 KB (5 loads per thread at 40
+// heads x 128 bf16), 64 threads up to 8 KB, 32 up to 4 KB (8 rows per block).
+// RoPE needs a head's vectors to fit the group.
+template <int EB, bool ROPE, int MODE>
+atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream) {
+    if (p.row_vecs <= 256 && p.vph <= 32) return launch_g<EB, ROPE, MODE, 32>(p, dev, stream);
+    if (p.row_vecs <= 512 && p.vph <= 64) return launch_g<EB, ROPE, MODE, 64>(p, dev, stream);
+    return launch_g<EB, ROPE, MODE, 128>(p, dev, stream);
 }
 
 // mode: 0 reorder, 1 unorder, 2 raster RoPE; `general` selects the
