@@ -6,6 +6,8 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "atlas_internal.cuh"
 
@@ -51,6 +53,20 @@ bool current_device(DeviceInfo *out) {
     }
     *out = c;
     return c.major == 10 && c.minor == 0;
+}
+
+bool set_smem_limit(const void *func, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void *>> done;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({dev, func})) return true;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    done.insert({dev, func});
+    return true;
 }
 
 namespace {

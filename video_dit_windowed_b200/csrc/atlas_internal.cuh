@@ -53,6 +53,11 @@ struct DeviceInfo {
 // usable device or not compute capability 10.0.
 bool current_device(DeviceInfo *out);
 
+// Raise `func`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (device, function): the attribute belongs to the device's
+// context, so a process driving several GPUs sets it on each.
+bool set_smem_limit(const void *func, int bytes);
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {

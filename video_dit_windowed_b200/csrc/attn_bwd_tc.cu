@@ -709,14 +709,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
 template <int HD, int FORM>
 atlas_status launch_form(Params p, const DeviceInfo &dev, cudaStream_t stream) {
     const size_t smem = sizeof(Smem<HD>) + 1024;
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [&] {
-        attr = cudaFuncSetAttribute(attn_bwd_tc_kernel<HD, FORM>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem));
-    });
-    if (attr != cudaSuccess) return ATLAS_ERR_CUDA;
+    if (!set_smem_limit(reinterpret_cast<const void *>(attn_bwd_tc_kernel<HD, FORM>),
+                        static_cast<int>(smem)))
+        return ATLAS_ERR_CUDA;
     const int64_t per_prob = p.tiles_d + p.tiles_g;
     const int64_t units = per_prob * p.batch * p.heads;
     if (units == 0) return ATLAS_OK;

@@ -709,14 +709,9 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.gwin_off = a.gwin_off;
     p.n_win = static_cast<int32_t>(a.win_off ? a.n_win : a.n_gwin);
     const size_t smem = sizeof(Smem<HD>) + 1024;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(attn_tc_kernel<HD>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(smem));
-    });
-    if (attr_err != cudaSuccess) return ATLAS_ERR_CUDA;
+    if (!set_smem_limit(reinterpret_cast<const void *>(attn_tc_kernel<HD>),
+                        static_cast<int>(smem)))
+        return ATLAS_ERR_CUDA;
     const int grid = std::min(p.n_units, dev.sm_count);
     attn_tc_kernel<HD><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;

@@ -342,13 +342,9 @@ atlas_status launch(Params &p, const void *a, const void *b, const DeviceInfo &d
     if (total > INT32_MAX) return ATLAS_ERR_SHAPE;
     p.n_tile_total = static_cast<int32_t>(total);
     const size_t smem = sizeof(Smem) + 1024;
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [&] {
-        attr = cudaFuncSetAttribute(gemm_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem));
-    });
-    if (attr != cudaSuccess) return ATLAS_ERR_CUDA;
+    if (!set_smem_limit(reinterpret_cast<const void *>(gemm_proj_kernel),
+                        static_cast<int>(smem)))
+        return ATLAS_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(total, dev.sm_count));
     gemm_proj_kernel<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
