@@ -126,8 +126,9 @@ class Path:
       of global Q and K; attention (own window + every global key of the
       problem); unorder O_d.
     "aligned": the aligned-proxy-tokens variant. As "all", but global Q, K
-      (+RoPE) and V are reordered by the aligned global cube, each window sees
-      only its aligned global keys, and O_g is unordered too.
+      (+RoPE) and V are put in the aligned order (cube by cube of the detail
+      grid, any grid ratios), each window sees only its aligned global keys,
+      and O_g is unordered too.
     "raster": naive block attention for comparison. RoPE of detail Q and K
       in raster order, no reorder; windows of window_len consecutive raster
       rows (+ every global key); no unorder.
@@ -147,7 +148,6 @@ class Path:
             raise ValueError(f"--mask {mask} needs a cube that divides the grid")
         self.atlas, self.w, self.dev, self.stream = atlas, w, device, stream
         self.mask, self.B = mask, batch
-        self.gcube = None
         self.rd = atlas.make_rope(w.theta, w.split, w.detail_scales)
         self.rg = atlas.make_rope(w.theta, w.split, w.global_scales)
         e = lambda t: torch.empty_like(t)
@@ -173,10 +173,9 @@ class Path:
         self.o_raster = e(x["q_d"])
         self.win = (atlas.cube_window_offsets(w.grid, w.cube).to(device)
                     if w.partial or mask == "aligned" else None)
-        self.gwin = self.gcube = None
+        self.gwin = None
         if mask == "aligned":
-            self.gcube = atlas.aligned_global_cube(w.grid, w.cube, w.global_grid)
-            self.gwin = atlas.cube_window_offsets(w.global_grid, self.gcube).to(device)
+            self.gwin = atlas.aligned_global_offsets(w.grid, w.cube, w.global_grid).to(device)
             self.v_g = e(x["v_g"])
             self.o_graster = e(x["q_g"])
         self.lse = None
@@ -228,10 +227,10 @@ class Path:
         v_g = x["v_g"]
         if G:
             if self.mask == "aligned":
-                gg, gc = w.global_grid, self.gcube
-                a.cube_reorder_batched(x["q_g"], self.q_g, B, gg, gc, self.rg, stream=s)
-                a.cube_reorder_batched(x["k_g"], self.k_g, B, gg, gc, self.rg, stream=s)
-                a.cube_reorder_batched(x["v_g"], self.v_g, B, gg, gc, None, stream=s)
+                args = (w.grid, w.cube, w.global_grid)
+                a.aligned_global_reorder(x["q_g"], self.q_g, *args, self.rg, B, stream=s)
+                a.aligned_global_reorder(x["k_g"], self.k_g, *args, self.rg, B, stream=s)
+                a.aligned_global_reorder(x["v_g"], self.v_g, *args, None, B, stream=s)
                 v_g = self.v_g
             else:
                 a.rope3d_batched(x["q_g"], self.q_g, B, w.global_grid, self.rg, stream=s)
@@ -250,8 +249,8 @@ class Path:
         if N and self.mask != "raster":
             a.cube_unorder_batched(self.o_d, self.o_raster, B, w.grid, w.cube, stream=s)
         if self.mask == "aligned" and G:
-            a.cube_unorder_batched(self.o_g, self.o_graster, B, w.global_grid, self.gcube,
-                                   stream=s)
+            a.aligned_global_unorder(self.o_g, self.o_graster, w.grid, w.cube, w.global_grid,
+                                     batch=B, stream=s)
         rec(4)
         if self.backward:
             self.step_backward(v_d, v_g, ev)
@@ -263,13 +262,13 @@ class Path:
         a, w, s, B = self.atlas, self.w, self.stream, self.B
         rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
         N, G, m = w.n_detail, w.n_global, self.mask
-        gg, gc = w.global_grid, self.gcube
+        gg, args = w.global_grid, (w.grid, w.cube, w.global_grid)
         do_d, do_g = self.do["d"], self.do["g"]
         if N and m != "raster":
             a.cube_reorder_batched(do_d, self.do_att["d"], B, w.grid, w.cube, stream=s)
             do_d = self.do_att["d"]
         if G and m == "aligned":
-            a.cube_reorder_batched(do_g, self.do_att["g"], B, gg, gc, stream=s)
+            a.aligned_global_reorder(do_g, self.do_att["g"], *args, batch=B, stream=s)
             do_g = self.do_att["g"]
         rec(5)
         g = self.grad
@@ -289,9 +288,9 @@ class Path:
                 a.cube_unorder_batched(g[2], r[2], B, w.grid, w.cube, stream=s)
         if G:
             if m == "aligned":
-                a.cube_unorder_rope(g[3], r[3], gg, gc, self.rg_t, B, stream=s)
-                a.cube_unorder_rope(g[4], r[4], gg, gc, self.rg_t, B, stream=s)
-                a.cube_unorder_batched(g[5], r[5], B, gg, gc, stream=s)
+                a.aligned_global_unorder(g[3], r[3], *args, self.rg_t, B, stream=s)
+                a.aligned_global_unorder(g[4], r[4], *args, self.rg_t, B, stream=s)
+                a.aligned_global_unorder(g[5], r[5], *args, batch=B, stream=s)
             else:
                 a.rope3d_batched(g[3], r[3], B, gg, self.rg_t, stream=s)
                 a.rope3d_batched(g[4], r[4], B, gg, self.rg_t, stream=s)
@@ -336,7 +335,7 @@ class Path:
         return self.flops() * 14 // 4
 
     def flops(self):
-        return self.B * self.w.unmasked_flops(self.mask, self.gcube)
+        return self.B * self.w.unmasked_flops(self.mask)
 
     def prep_bytes(self):
         """Algorithmic bytes of the reorder/RoPE phase: one read and one

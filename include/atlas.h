@@ -338,6 +338,51 @@ atlas_status atlas_local_global_attn_bwd(
     atlas_stream_t stream);
 
 /*
+ * atlas_aligned_global_reorder / atlas_aligned_global_unorder -- the global
+ * proxy's tokens to and from the aligned order, for any grid ratios.
+ *
+ * Passage: Methodologie 2, position alignment. Reading: global index x of an
+ * axis of e tokens sits at detail position x*E/e of the detail axis (E
+ * tokens) and is aligned with the detail cube (c tokens) holding that point,
+ * box(x) = floor(x*E / (c*e)); box b spans global indices [ceil(b*c*e/E),
+ * ceil((b+1)*c*e/E)) (possibly empty), and the box triples partition the
+ * global grid by the detail cube each token is aligned with. The aligned
+ * order lists the tokens box by box in the cube grid's raster order (raster
+ * order inside a box), so the aligned keys of detail window w are one range
+ * [offsets[w], offsets[w+1]) (atlas_aligned_global_offsets): pass it as
+ * atlas_attn_layout.global_window_offsets. When the ratios are integers
+ * dividing the cube this is the cube order of atlas_aligned_global_cube.
+ *
+ * src, dst: [batch * t*h*w, heads, head_dim] of the global grid (raster order
+ * for the reorder's input and the unorder's output); grid and cube are the
+ * detail grid and its cube. rope: rotation at each token's global raster
+ * position (NULL: none; for the unorder, the transpose with negated scales
+ * maps gradients back). Errors as atlas_cube_reorder_batched.
+ */
+atlas_status atlas_aligned_global_reorder(const void *src, void *dst, int64_t batch,
+                                          atlas_grid3 grid, atlas_cube3 cube,
+                                          atlas_grid3 global_grid, int32_t heads,
+                                          int32_t head_dim, atlas_dtype dtype,
+                                          const atlas_rope *rope, atlas_stream_t stream);
+atlas_status atlas_aligned_global_unorder(const void *src, void *dst, int64_t batch,
+                                          atlas_grid3 grid, atlas_cube3 cube,
+                                          atlas_grid3 global_grid, int32_t heads,
+                                          int32_t head_dim, atlas_dtype dtype,
+                                          const atlas_rope *rope, atlas_stream_t stream);
+
+/*
+ * atlas_aligned_global_offsets -- the global key range of every detail window
+ * in the aligned order (host). offsets: host array of `capacity` int32, or
+ * NULL to query the count; *n_windows receives the number of detail cubes
+ * (windows, raster order over the cube grid); offsets[n_windows] = t*h*w.
+ * Errors: NULL n_windows (NULL), non-positive extents or too many tokens
+ * (SHAPE), capacity < n_windows+1 (CAPACITY). No device work.
+ */
+atlas_status atlas_aligned_global_offsets(atlas_grid3 grid, atlas_cube3 cube,
+                                          atlas_grid3 global_grid, int32_t *offsets,
+                                          int64_t capacity, int64_t *n_windows);
+
+/*
  * atlas_aligned_global_cube -- the global-grid cube whose cubes are the
  * aligned sets of the detail cubes (host).
  *

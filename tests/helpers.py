@@ -41,6 +41,24 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+def aligned_positions(grid, cube, gg):
+    """pos[g] = place of global raster token g in the aligned order, from the
+    reading of position alignment: global index x of an axis of e tokens sits
+    at detail position x*E/e, in detail cube floor(x*E/(c*e)); tokens are
+    listed cube by cube (raster order of the cube grid), raster order inside."""
+    nh = -(-grid[1] // cube[1])
+    nw = -(-grid[2] // cube[2])
+    keys = []
+    for g in range(gg[0] * gg[1] * gg[2]):
+        x = (g // (gg[1] * gg[2]), (g // gg[2]) % gg[1], g % gg[2])
+        b = [x[a] * grid[a] // (cube[a] * gg[a]) for a in range(3)]
+        keys.append(((b[0] * nh + b[1]) * nw + b[2], g))
+    order = [g for _, g in sorted(keys)]
+    pos = np.empty(len(order), dtype=np.int64)
+    pos[np.array(order, dtype=np.int64)] = np.arange(len(order))
+    return pos
+
+
 def ulp(v: np.ndarray, dtype: str) -> np.ndarray:
     _, e = np.frexp(np.abs(v))
     bits = 8 if dtype == "bf16" else 24

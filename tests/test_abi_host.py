@@ -305,3 +305,70 @@ def test_projection_validation(lib):
     if not torch.cuda.is_available():
         assert qkv() == atlas.ERR_DEVICE
         assert out() == atlas.ERR_DEVICE
+
+
+def test_aligned_global_offsets_host(lib):
+    """Window ranges of the aligned order: validation, and for ratios that
+    are not integers the range of window w holds exactly the global tokens
+    the oracle's aligned predicate gives detail cube w (probe as above, with
+    the aligned order's positions from their definition)."""
+    import numpy as np
+    import oracle
+    from helpers import aligned_positions
+    G3, C3 = atlas.Grid3, atlas.Cube3
+    n = ctypes.c_int64(0)
+    assert lib.atlas_aligned_global_offsets(G3(4, 8, 8), C3(2, 4, 4), G3(2, 4, 4), None, 0,
+                                            None) == atlas.ERR_NULL
+    assert lib.atlas_aligned_global_offsets(G3(4, 8, 8), C3(2, 4, 4), G3(2, 0, 4), None, 0,
+                                            ctypes.byref(n)) == atlas.ERR_SHAPE
+    assert lib.atlas_aligned_global_offsets(G3(4, 8, 8), C3(0, 4, 4), G3(2, 4, 4), None, 0,
+                                            ctypes.byref(n)) == atlas.ERR_SHAPE
+    assert lib.atlas_aligned_global_offsets(G3(4, 8, 8), C3(2, 4, 4), G3(2, 4, 4), None, 0,
+                                            ctypes.byref(n)) == atlas.OK
+    assert n.value == 8
+    buf = (ctypes.c_int32 * 8)()
+    assert lib.atlas_aligned_global_offsets(G3(4, 8, 8), C3(2, 4, 4), G3(2, 4, 4), buf, 8,
+                                            ctypes.byref(n)) == atlas.ERR_CAPACITY
+    orc = oracle.Oracle()
+    for grid, cube, gg in (((5, 7, 9), (2, 3, 4), (2, 3, 4)), ((6, 20, 30), (3, 8, 8), (4, 6, 7)),
+                           ((4, 8, 8), (2, 4, 4), (3, 10, 5))):
+        goff = atlas.aligned_global_offsets(grid, cube, gg).numpy()
+        doff = atlas.cube_window_offsets(grid, cube).numpy()
+        G = gg[0] * gg[1] * gg[2]
+        assert goff.size == doff.size and goff[0] == 0 and goff[-1] == G
+        assert np.all(np.diff(goff) >= 0)
+        pos = aligned_positions(grid, cube, gg)
+        assert sorted(pos.tolist()) == list(range(G))
+        D = 8
+        for w in range(doff.size - 1):
+            lo, hi = int(doff[w]), int(doff[w + 1])
+            vg = np.zeros((G, D))
+            inside = (pos >= goff[w]) & (pos < goff[w + 1])
+            vg[inside, 0] = 1.0
+            vg[~inside, 1] = 1.0
+            kd = np.zeros((hi - lo, D))
+            o, _ = orc.attention_head_aligned(grid, cube, gg, 1.0, kd, kd, lo, np.zeros((G, D)),
+                                              vg, np.arange(lo, hi), np.zeros((hi - lo, D)))
+            assert np.all(o[:, 1] == 0.0), (grid, w)
+            n_in = int(inside.sum())
+            assert np.allclose(o[:, 0], n_in / (hi - lo + n_in)), (grid, w)
+        if grid == (5, 7, 9):
+            assert int(np.sum(np.diff(goff) == 0)) > 0   # windows with no aligned token
+
+
+def test_aligned_global_permute_validation(lib):
+    big = FAKE + (1 << 30)
+    G3, C3 = atlas.Grid3, atlas.Cube3
+    for fn in (lib.atlas_aligned_global_reorder, lib.atlas_aligned_global_unorder):
+        call = lambda src=FAKE, dst=big, b=1, grid=G3(4, 8, 8), cube=C3(2, 4, 4), \
+            gg=G3(2, 4, 4), hd=64, dt=atlas.FP32: fn(src, dst, b, grid, cube, gg, 2, hd, dt,
+                                                      None, None)
+        assert call(src=None) == atlas.ERR_NULL
+        assert call(dst=None) == atlas.ERR_NULL
+        assert call(gg=G3(2, 0, 4)) == atlas.ERR_SHAPE
+        assert call(cube=C3(2, 4, 0)) == atlas.ERR_SHAPE
+        assert call(grid=G3(-1, 8, 8)) == atlas.ERR_SHAPE
+        assert call(b=-1) == atlas.ERR_SHAPE
+        assert call(src=FAKE + 8) == atlas.ERR_ALIGN
+        assert call(dst=FAKE + 64) == atlas.ERR_ALIAS
+        assert call(dt=7) == atlas.ERR_UNSUPPORTED

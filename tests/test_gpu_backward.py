@@ -140,6 +140,45 @@ def test_backward_aligned(dtype, B):
         assert_grads_close(part, ref, dtype, f"aligned problem {b}")
 
 
+@pytest.mark.parametrize("dtype,B", [("bf16", 1), ("fp32", 2)])
+def test_backward_aligned_order_general(dtype, B):
+    """Aligned variant at ratios that are not integers (detail 6x20x30 with
+    cubes 3x8x8 and partial cubes, global 4x6x7): global tokens in the
+    aligned order on the GPU, raster order in the oracle."""
+    grid, cube, gg, heads, hd = (6, 20, 30), (3, 8, 8), (4, 6, 7), 2, 128
+    N, G = 3600, 168
+    win = atlas.cube_window_offsets(grid, cube)
+    gwin = atlas.aligned_global_offsets(grid, cube, gg)
+    t = inputs(B, N, G, heads, hd, dtype, seed=24)
+    tg = dict(t)
+    for s in ("q_d", "k_d", "v_d", "do_d"):
+        tg[s] = torch.empty_like(t[s])
+        atlas.cube_reorder_batched(t[s], tg[s], B, grid, cube)
+    for s in ("q_g", "k_g", "v_g", "do_g"):
+        tg[s] = torch.empty_like(t[s])
+        atlas.aligned_global_reorder(t[s], tg[s], grid, cube, gg, batch=B)
+    got = run_gpu(tg, B, heads, N, G, window_offsets=win.to(DEV),
+                  global_window_offsets=gwin.to(DEV))
+    for i in range(6):
+        r = torch.empty_like(got[i])
+        if i < 3:
+            atlas.cube_unorder_batched(got[i], r, B, grid, cube)
+        else:
+            atlas.aligned_global_unorder(got[i], r, grid, cube, gg, batch=B)
+        got[i] = r
+    torch.cuda.synchronize()
+    o = orc()
+    for b in range(B):
+        sd, sg = slice(b * N, (b + 1) * N), slice(b * G, (b + 1) * G)
+        cu = lambda s: o.cube_reorder(f64(t[s][sd]), grid, cube)
+        ref = o.attention_bwd_full_aligned(
+            cu("q_d"), cu("k_d"), cu("v_d"), grid, cube, f64(t["q_g"][sg]), f64(t["k_g"][sg]),
+            f64(t["v_g"][sg]), gg, cu("do_d"), f64(t["do_g"][sg]), hd ** -0.5, n_threads())
+        ref = [o.cube_unorder(r, grid, cube) if i < 3 else r for i, r in enumerate(ref)]
+        part = [f64(g[sd if i < 3 else sg]) for i, g in enumerate(got)]
+        assert_grads_close(part, ref, dtype, f"aligned order problem {b}")
+
+
 def test_backward_dv_of_constant_do():
     """dO = 1 on every row: dV_j = sum_i P_ij, so the detail and global dV
     columns sum, over all keys, to the number of query rows (each row's P

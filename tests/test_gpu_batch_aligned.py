@@ -7,10 +7,10 @@
   AtlasVid", Methodologie 2: a detail query sees the aligned global tokens;
   position alignment scales global coordinates by the resolution ratios).
   Reading: global token (tg, hg, wg) sits at (tg*T/t, hg*H/h, wg*W/w) of the
-  detail grid and is aligned with the cube holding that point. With integer
-  ratios dividing the cube, the aligned tokens of cube c are cube c of the
-  global grid cut into the cube / ratio, so the GPU path reorders the global
-  tokens by that cube and passes per-window global offsets.
+  detail grid and is aligned with the cube holding that point. The GPU path
+  lists the global tokens in the aligned order (cube by cube of the detail
+  grid) and passes per-window global offsets; with integer ratios dividing
+  the cube that order is the global grid's own cube order.
 
 The oracle takes the global tokens in raster order and decides alignment
 from coordinates; the GPU results are mapped back to raster order.
@@ -19,8 +19,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (assert_attn_close, assert_rope_close, check_no_device_error, f64, n_threads,
-                     orc)
+from helpers import (aligned_positions, assert_attn_close, assert_rope_close,
+                     check_no_device_error, f64, n_threads, orc)
 from video_dit_windowed_b200 import atlas
 from video_dit_windowed_b200.workloads import normal
 
@@ -277,4 +277,159 @@ def test_aligned_720p_sampled():
             grid, cube, gg, hd ** -0.5, None, None, 0, kg, vg, N + g_rows,
             f64(xg["q_g"][torch.as_tensor(g_rows, device=DEV), head]), n_threads())
         got = f64(o_g[torch.as_tensor(gpos[g_rows], device=DEV), head])
+        assert_attn_close(got, ref, "bf16", f"global rows head {head}")
+
+
+# ---------------------------------------------------------------------------
+# The aligned order: any grid ratios
+# ---------------------------------------------------------------------------
+
+def general_aligned_chain(x, grid, cube, gg, B, hd, global_scales):
+    """Raster inputs -> detail cube reorder (+RoPE) and global aligned-order
+    reorder (+RoPE at global raster coordinates) -> attention with per-window
+    global ranges -> back to raster order."""
+    rd = atlas.make_rope(10000.0, split_for(hd), (1.0, 1.0, 1.0))
+    rg = atlas.make_rope(10000.0, split_for(hd), global_scales)
+    y = {s: torch.empty_like(x[s]) for s in x}
+    for s in ("q_d", "k_d", "v_d"):
+        atlas.cube_reorder_batched(x[s], y[s], B, grid, cube, rd if s != "v_d" else None)
+    for s in ("q_g", "k_g", "v_g"):
+        atlas.aligned_global_reorder(x[s], y[s], grid, cube, gg, rg if s != "v_g" else None,
+                                     batch=B)
+    win = atlas.cube_window_offsets(grid, cube).to(DEV)
+    gwin = atlas.aligned_global_offsets(grid, cube, gg).to(DEV)
+    assert win.numel() == gwin.numel()
+    N, G = grid[0] * grid[1] * grid[2], gg[0] * gg[1] * gg[2]
+    heads = x["q_d"].shape[1]
+    o_d, o_g = torch.empty_like(y["q_d"]), torch.empty_like(y["q_g"])
+    lse = torch.empty(B, heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_ex(y["q_d"], y["k_d"], y["v_d"], y["q_g"], y["k_g"], y["v_g"], o_d,
+                               o_g, lse, batch=B, window_offsets=win,
+                               global_window_offsets=gwin)
+    r_d, r_g = torch.empty_like(o_d), torch.empty_like(o_g)
+    atlas.cube_unorder_batched(o_d, r_d, B, grid, cube)
+    atlas.aligned_global_unorder(o_g, r_g, grid, cube, gg, batch=B)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    return r_d, r_g, lse, y
+
+
+# detail grid, cube, global grid, batch, heads, hd, dtype. Ratios that are
+# not integers, ratios below one, windows with no aligned global token
+# (5/2 tokens per global step in t with cubes of 2: cube 2 of t gets none).
+GENERAL_CASES = [
+    ((5, 7, 9), (2, 3, 4), (2, 3, 4), 1, 2, 128, "bf16"),
+    ((5, 7, 9), (2, 3, 4), (2, 3, 4), 2, 2, 64, "fp32"),
+    ((6, 20, 30), (3, 8, 8), (4, 6, 7), 1, 2, 128, "bf16"),
+    ((6, 20, 30), (3, 8, 8), (4, 6, 7), 2, 1, 64, "fp32"),
+    ((4, 8, 8), (2, 4, 4), (3, 10, 5), 1, 2, 128, "bf16"),
+    ((9, 36, 44), (3, 16, 16), (5, 7, 11), 1, 2, 128, "bf16"),
+]
+
+
+@pytest.mark.parametrize("grid,cube,gg,B,heads,hd,dtype", GENERAL_CASES)
+def test_aligned_order_chain(grid, cube, gg, B, heads, hd, dtype):
+    N, G = grid[0] * grid[1] * grid[2], gg[0] * gg[1] * gg[2]
+    ratios = tuple(a / b for a, b in zip(grid, gg))
+    x = {s: mk(B * (N if s.endswith("_d") else G), heads, hd, s, dtype, seed=14)
+         for s in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")}
+    r_d, r_g, lse, y = general_aligned_chain(x, grid, cube, gg, B, hd, ratios)
+    o = orc()
+    pos = aligned_positions(grid, cube, gg)
+    for b in range(B):
+        sd, sg = slice(b * N, (b + 1) * N), slice(b * G, (b + 1) * G)
+        # the permutation alone: bit-exact against the order's definition
+        raw = x["v_g"][sg].cpu().view(torch.uint8).numpy().reshape(G, -1)
+        want = np.empty_like(raw)
+        want[pos] = raw
+        assert y["v_g"][sg].cpu().view(torch.uint8).numpy().reshape(G, -1).tobytes() == \
+            want.tobytes()
+        rot = lambda s, g, sc: o.rope3d_grid(f64(x[s][sd if s.endswith("_d") else sg]), g,
+                                             10000.0, split_for(hd), sc)
+        qd = o.cube_reorder(rot("q_d", grid, (1, 1, 1)), grid, cube)
+        kd = o.cube_reorder(rot("k_d", grid, (1, 1, 1)), grid, cube)
+        vd = o.cube_reorder(f64(x["v_d"][sd]), grid, cube)
+        ref_d, ref_g, ref_l = o.attention_full_aligned(
+            qd, kd, vd, grid, cube, rot("q_g", gg, ratios), rot("k_g", gg, ratios),
+            f64(x["v_g"][sg]), gg, hd ** -0.5, n_threads())
+        got = np.concatenate([f64(r_d[sd]), f64(r_g[sg])])
+        ref = np.concatenate([o.cube_unorder(ref_d, grid, cube), ref_g])
+        assert_attn_close(got, ref, dtype, f"{grid} {gg} problem {b}")
+        l_gpu = f64(lse[b])
+        assert np.max(np.abs(l_gpu[:, :N] - ref_l[:, :N])) <= LSE_TOL[dtype]
+        assert np.max(np.abs(l_gpu[:, N + pos] - ref_l[:, N:])) <= LSE_TOL[dtype]
+
+
+@pytest.mark.parametrize("grid,cube,gg", [((6, 16, 16), (3, 8, 8), (6, 4, 4)),
+                                          ((21, 48, 80), (3, 16, 16), (21, 12, 20)),
+                                          ((4, 8, 8), (2, 4, 4), (2, 4, 4))])
+def test_aligned_order_is_cube_order_for_integral_ratios(grid, cube, gg):
+    """With integer ratios dividing the cube the aligned order is the global
+    grid's cube order: same bits, same window ranges."""
+    gcube = atlas.aligned_global_cube(grid, cube, gg)
+    G = gg[0] * gg[1] * gg[2]
+    x = mk(2 * G, 3, 128, "k_g", "bf16", seed=15)
+    rg = atlas.make_rope(10000.0, split_for(128), tuple(a / b for a, b in zip(grid, gg)))
+    a, b = torch.empty_like(x), torch.empty_like(x)
+    atlas.aligned_global_reorder(x, a, grid, cube, gg, rg, batch=2)
+    atlas.cube_reorder_batched(x, b, 2, gg, gcube, rg)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert torch.equal(atlas.aligned_global_offsets(grid, cube, gg),
+                       atlas.cube_window_offsets(gg, gcube))
+    # the inverse: of the rotated order, the rotated raster tokens; of the
+    # plain order, the input bits
+    z, xr, p = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    atlas.aligned_global_unorder(a, z, grid, cube, gg, batch=2)
+    atlas.rope3d_batched(x, xr, 2, gg, rg)
+    torch.cuda.synchronize()
+    assert torch.equal(z.view(torch.uint8), xr.view(torch.uint8))
+    atlas.aligned_global_reorder(x, p, grid, cube, gg, batch=2)
+    atlas.aligned_global_unorder(p, z, grid, cube, gg, batch=2)
+    torch.cuda.synchronize()
+    assert torch.equal(z.view(torch.uint8), x.view(torch.uint8))
+
+
+def test_aligned_order_8k_sampled():
+    """8K geometry with partial cubes (detail 8x270x480, cubes 3x16x16,
+    global 8x27x48: ratios 1, 10, 10, which do not divide the 16-token cube
+    sides), 4 heads: sampled windows and global rows against the oracle."""
+    grid, cube, gg, heads, hd = (8, 270, 480), (3, 16, 16), (8, 27, 48), 4, 128
+    N, G = 8 * 270 * 480, 8 * 27 * 48
+    x = {s: mk(N if s.endswith("_d") else G, heads, hd, s, "bf16", seed=16)
+         for s in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")}
+    y = {s: torch.empty_like(x[s]) for s in x}
+    for s in ("q_d", "k_d", "v_d"):
+        atlas.cube_reorder(x[s], y[s], grid, cube)
+    for s in ("q_g", "k_g", "v_g"):
+        atlas.aligned_global_reorder(x[s], y[s], grid, cube, gg)
+    win = atlas.cube_window_offsets(grid, cube)
+    gwin = atlas.aligned_global_offsets(grid, cube, gg)
+    o_d, o_g = torch.empty_like(y["q_d"]), torch.empty_like(y["q_g"])
+    lse = torch.empty(1, heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_ex(y["q_d"], y["k_d"], y["v_d"], y["q_g"], y["k_g"], y["v_g"], o_d,
+                               o_g, lse, window_offsets=win.to(DEV),
+                               global_window_offsets=gwin.to(DEV))
+    r_g = torch.empty_like(o_g)
+    atlas.aligned_global_unorder(o_g, r_g, grid, cube, gg)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    wo = win.numpy().astype(np.int64)
+    nwin = wo.size - 1
+    for head in (0, heads - 1):
+        kg, vg = f64(x["k_g"][:, head]), f64(x["v_g"][:, head])
+        for w in (0, 31, nwin // 2 + 7, nwin - 1):
+            lo, hi = int(wo[w]), int(wo[w + 1])
+            rows = np.arange(lo, hi)
+            ref, ref_l = orc().attention_head_aligned(
+                grid, cube, gg, hd ** -0.5, f64(y["k_d"][lo:hi, head]),
+                f64(y["v_d"][lo:hi, head]), lo, kg, vg, rows, f64(y["q_d"][lo:hi, head]),
+                n_threads())
+            assert_attn_close(f64(o_d[lo:hi, head]), ref, "bf16", f"window {w} head {head}")
+            assert np.max(np.abs(f64(lse[0, head, lo:hi]) - ref_l)) <= LSE_TOL["bf16"]
+        g_rows = np.array([0, 5, 1234, G - 1])
+        ref, _ = orc().attention_head_aligned(
+            grid, cube, gg, hd ** -0.5, None, None, 0, kg, vg, N + g_rows,
+            f64(x["q_g"][torch.as_tensor(g_rows, device=DEV), head]), n_threads())
+        got = f64(r_g[torch.as_tensor(g_rows, device=DEV), head])
         assert_attn_close(got, ref, "bf16", f"global rows head {head}")

@@ -99,6 +99,14 @@ def _declare(lib):
     lib.atlas_out_proj_unorder.restype = ctypes.c_int
     lib.atlas_out_proj_unorder.argtypes = [_vp, _vp, _i64, Grid3, Cube3, _i32, _i32,
                                            ctypes.c_int, _vp, _vp]
+    for name in ("atlas_aligned_global_reorder", "atlas_aligned_global_unorder"):
+        fn = getattr(lib, name)
+        fn.restype = ctypes.c_int
+        fn.argtypes = [_vp, _vp, _i64, Grid3, Cube3, Grid3, _i32, _i32, ctypes.c_int,
+                       ctypes.POINTER(Rope), _vp]
+    lib.atlas_aligned_global_offsets.restype = ctypes.c_int
+    lib.atlas_aligned_global_offsets.argtypes = [Grid3, Cube3, Grid3, _vp, _i64,
+                                                 ctypes.POINTER(_i64)]
     lib.atlas_aligned_global_cube.restype = ctypes.c_int
     lib.atlas_aligned_global_cube.argtypes = [Grid3, Cube3, Grid3, ctypes.POINTER(Cube3)]
     lib.atlas_cube_reorder_batched.restype = ctypes.c_int
@@ -362,6 +370,47 @@ def out_proj_unorder(o, w, grid, cube, y, batch=1, stream=None):
                                       _stream(o, stream))
     _check(st, "atlas_out_proj_unorder")
     return y
+
+
+def aligned_global_reorder(src, dst, grid, cube, global_grid, rope: Rope | None = None,
+                           batch=1, stream=None):
+    """Global-proxy tokens (raster order of ``global_grid``) into the aligned
+    order of ``grid`` cut into ``cube``; any grid ratios."""
+    n, heads, hd = src.shape
+    st = lib().atlas_aligned_global_reorder(
+        _ptr(src), _ptr(dst), int(batch), Grid3(*grid), Cube3(*cube), Grid3(*global_grid), heads,
+        hd, _dtype_code(src), ctypes.byref(rope) if rope is not None else None,
+        _stream(src, stream))
+    _check(st, "atlas_aligned_global_reorder")
+    return dst
+
+
+def aligned_global_unorder(src, dst, grid, cube, global_grid, rope: Rope | None = None,
+                           batch=1, stream=None):
+    """Inverse of ``aligned_global_reorder`` (optionally rotating, e.g. by the
+    transposed RoPE for gradients)."""
+    n, heads, hd = src.shape
+    st = lib().atlas_aligned_global_unorder(
+        _ptr(src), _ptr(dst), int(batch), Grid3(*grid), Cube3(*cube), Grid3(*global_grid), heads,
+        hd, _dtype_code(src), ctypes.byref(rope) if rope is not None else None,
+        _stream(src, stream))
+    _check(st, "atlas_aligned_global_unorder")
+    return dst
+
+
+def aligned_global_offsets(grid, cube, global_grid):
+    """Global key range of every detail window in the aligned order, as a
+    host int32 tensor [n_windows + 1]."""
+    import torch
+    n = _i64(0)
+    args = (Grid3(*grid), Cube3(*cube), Grid3(*global_grid))
+    _check(lib().atlas_aligned_global_offsets(*args, None, 0, ctypes.byref(n)),
+           "atlas_aligned_global_offsets")
+    out = torch.empty(n.value + 1, dtype=torch.int32)
+    _check(lib().atlas_aligned_global_offsets(*args, ctypes.c_void_p(out.data_ptr()),
+                                              out.numel(), ctypes.byref(n)),
+           "atlas_aligned_global_offsets")
+    return out
 
 
 def aligned_global_cube(grid, cube, global_grid):

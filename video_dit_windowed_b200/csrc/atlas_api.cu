@@ -10,6 +10,7 @@
 #include <utility>
 
 #include "atlas_internal.cuh"
+#include "cube_geom.cuh"
 
 namespace atlas {
 
@@ -224,6 +225,87 @@ ATLAS_API atlas_status atlas_cube_unorder_batched(const void *src, void *dst, in
                                                   int32_t heads, int32_t head_dim,
                                                   atlas_dtype dtype, atlas_stream_t stream) {
     return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, nullptr, stream);
+}
+
+namespace atlas {
+namespace {
+
+// Reorder to (mode 5) or from (mode 6) the aligned order of global tokens.
+atlas_status aligned_perm(const void *src, void *dst, int64_t batch, atlas_grid3 grid,
+                          atlas_cube3 cube, atlas_grid3 gg, int32_t heads, int32_t head_dim,
+                          atlas_dtype dtype, const atlas_rope *rope, atlas_stream_t stream,
+                          int mode) {
+    size_t bytes = 0;
+    atlas_status st = check_permute(src, dst, batch, gg, heads, head_dim, dtype, &bytes);
+    if (st != ATLAS_OK) return st;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1 || grid.T > kMaxRows || grid.H > kMaxRows ||
+        grid.W > kMaxRows)
+        return ATLAS_ERR_SHAPE;
+    if ((st = check_cube(grid, cube)) != ATLAS_OK) return st;
+    if (rope && (st = check_rope(*rope, head_dim, dtype)) != ATLAS_OK) return st;
+    if (ranges_overlap(src, bytes, dst, bytes)) return ATLAS_ERR_ALIAS;
+    PermuteArgs a{src, dst, gg.T, gg.H, gg.W, cube.ct, cube.ch, cube.cw,
+                  heads, head_dim, elem_bytes(dtype), mode, rope, batch,
+                  grid.T, grid.H, grid.W};
+    return launch_permute_rope(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace atlas
+
+ATLAS_API atlas_status atlas_aligned_global_reorder(const void *src, void *dst, int64_t batch,
+                                                    atlas_grid3 grid, atlas_cube3 cube,
+                                                    atlas_grid3 global_grid, int32_t heads,
+                                                    int32_t head_dim, atlas_dtype dtype,
+                                                    const atlas_rope *rope,
+                                                    atlas_stream_t stream) {
+    return atlas::aligned_perm(src, dst, batch, grid, cube, global_grid, heads, head_dim, dtype,
+                               rope, stream, 5);
+}
+
+ATLAS_API atlas_status atlas_aligned_global_unorder(const void *src, void *dst, int64_t batch,
+                                                    atlas_grid3 grid, atlas_cube3 cube,
+                                                    atlas_grid3 global_grid, int32_t heads,
+                                                    int32_t head_dim, atlas_dtype dtype,
+                                                    const atlas_rope *rope,
+                                                    atlas_stream_t stream) {
+    return atlas::aligned_perm(src, dst, batch, grid, cube, global_grid, heads, head_dim, dtype,
+                               rope, stream, 6);
+}
+
+ATLAS_API atlas_status atlas_aligned_global_offsets(atlas_grid3 grid, atlas_cube3 cube,
+                                                    atlas_grid3 global_grid, int32_t *offsets,
+                                                    int64_t capacity, int64_t *n_windows) {
+    if (!n_windows) return ATLAS_ERR_NULL;
+    if (grid.T < 1 || grid.H < 1 || grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1 ||
+        global_grid.T < 1 || global_grid.H < 1 || global_grid.W < 1)
+        return ATLAS_ERR_SHAPE;
+    if (grid.T > kMaxRows || grid.H > kMaxRows || grid.W > kMaxRows ||
+        global_grid.T * global_grid.H * global_grid.W > kMaxRows)
+        return ATLAS_ERR_SHAPE;
+    auto n_along = [](int64_t e, int64_t c) { return (e + c - 1) / c; };
+    const int64_t nt = n_along(grid.T, cube.ct), nh = n_along(grid.H, cube.ch),
+                  nw = n_along(grid.W, cube.cw);
+    *n_windows = nt * nh * nw;
+    if (!offsets) return ATLAS_OK;   // size query
+    if (capacity < *n_windows + 1) return ATLAS_ERR_CAPACITY;
+    using atlas::geom::box_start;
+    const uint32_t T = static_cast<uint32_t>(global_grid.T), H = static_cast<uint32_t>(global_grid.H),
+                   W = static_cast<uint32_t>(global_grid.W);
+    const uint32_t DT = static_cast<uint32_t>(grid.T), DH = static_cast<uint32_t>(grid.H),
+                   DW = static_cast<uint32_t>(grid.W);
+    int64_t n = 0;
+    for (uint32_t bt = 0; bt < nt; ++bt)
+        for (uint32_t bh = 0; bh < nh; ++bh)
+            for (uint32_t bw = 0; bw < nw; ++bw) {
+                const uint32_t st = box_start(bt, T, DT, cube.ct), sh = box_start(bh, H, DH, cube.ch),
+                               sw = box_start(bw, W, DW, cube.cw);
+                const uint32_t et = box_start(bt + 1, T, DT, cube.ct) - st;
+                const uint32_t eh = box_start(bh + 1, H, DH, cube.ch) - sh;
+                offsets[n++] = static_cast<int32_t>(st * H * W + et * sh * W + et * eh * sw);
+            }
+    offsets[n] = static_cast<int32_t>(static_cast<int64_t>(T) * H * W);
+    return ATLAS_OK;
 }
 
 ATLAS_API atlas_status atlas_cube_unorder_rope(const void *src, void *dst, int64_t batch,

@@ -73,9 +73,11 @@ struct PermuteArgs {
     int64_t T, H, W;
     int32_t ct, ch, cw;
     int32_t heads, head_dim, elem_bytes;
-    int mode;               // 0 reorder (raster -> cube), 1 unorder, 2 raster RoPE
+    int mode;               // 0 reorder (raster -> cube), 1 unorder, 2 raster RoPE,
+                            // 5 / 6 to / from the aligned order of global tokens
     const atlas_rope *rope; // may be NULL (pure permutation)
     int64_t batch = 1;      // problems of this grid stacked along the rows
+    int64_t DT = 0, DH = 0, DW = 0;   // modes 5 / 6: the detail grid (T, H, W: the global)
 };
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
 atlas_status release_rope_tables();

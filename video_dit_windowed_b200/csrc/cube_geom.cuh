@@ -38,6 +38,9 @@ struct FastDiv {
 struct Geom {
     uint32_t T, H, W, ct, ch, cw, cubes_h, cubes_w, L;
     FastDiv by_W, by_H, by_ct, by_ch, by_cw, by_cubes_w, by_cubes_h, by_L;
+    // aligned order of a global grid (T x H x W here) against a detail grid
+    // DT x DH x DW cut into ct x ch x cw cubes; 0 when unused
+    uint32_t DT, DH, DW;
 };
 
 // Raster coordinates of a raster row.
@@ -117,6 +120,67 @@ __device__ __forceinline__ void cube_coords_general(const Geom &g, uint32_t j, u
     w = bw * g.cw + (rem - lh * ew);
 }
 
+// ---------------------------------------------------------------------------
+// Aligned order of the global-proxy tokens ("Technische Samenvatting:
+// AtlasVid", Methodologie 2, position alignment): global index x of an axis
+// of e tokens sits at detail position x*E/e of the detail axis of E tokens,
+// and belongs to the detail cube (of c tokens) holding that point:
+// box(x) = floor(x*E / (c*e)). Box b spans global indices
+// [ceil(b*c*e/E), ceil((b+1)*c*e/E)) clamped to e (it may be empty), the boxes
+// of an axis partition it, and a global token's box triple is the detail
+// cube it is aligned with. The aligned order lists the tokens box by box in
+// the cube grid's raster order, raster order inside a box: the cube order of
+// the partial-cube case with these boundaries.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint32_t box_of(uint32_t x, uint32_t e, uint32_t E,
+                                                   uint32_t c) {
+    return static_cast<uint32_t>(static_cast<uint64_t>(x) * E / (static_cast<uint64_t>(c) * e));
+}
+__host__ __device__ __forceinline__ uint32_t box_start(uint32_t b, uint32_t e, uint32_t E,
+                                                      uint32_t c) {
+    const uint64_t v = (static_cast<uint64_t>(b) * c * e + E - 1) / E;
+    return static_cast<uint32_t>(v < e ? v : e);
+}
+
+__device__ __forceinline__ uint32_t aligned_position(const Geom &g, uint32_t t, uint32_t h,
+                                                     uint32_t w) {
+    const uint32_t bt = box_of(t, g.T, g.DT, g.ct), bh = box_of(h, g.H, g.DH, g.ch),
+                   bw = box_of(w, g.W, g.DW, g.cw);
+    const uint32_t st = box_start(bt, g.T, g.DT, g.ct), sh = box_start(bh, g.H, g.DH, g.ch),
+                   sw = box_start(bw, g.W, g.DW, g.cw);
+    const uint32_t et = box_start(bt + 1, g.T, g.DT, g.ct) - st;
+    const uint32_t eh = box_start(bh + 1, g.H, g.DH, g.ch) - sh;
+    const uint32_t ew = box_start(bw + 1, g.W, g.DW, g.cw) - sw;
+    const uint32_t before = st * g.H * g.W + et * sh * g.W + et * eh * sw;
+    return before + ((t - st) * eh + (h - sh)) * ew + (w - sw);
+}
+
+// Inverse: the raster coordinates of the token at aligned position j. The
+// t-slab of box bt holds positions [st*H*W, (st+et)*H*W), so j / (H*W) is a
+// global t inside it; likewise along h and w within the slab.
+__device__ __forceinline__ void aligned_coords(const Geom &g, uint32_t j, uint32_t &t,
+                                               uint32_t &h, uint32_t &w) {
+    const uint32_t bt = box_of(j / (g.H * g.W), g.T, g.DT, g.ct);
+    const uint32_t st = box_start(bt, g.T, g.DT, g.ct);
+    const uint32_t et = box_start(bt + 1, g.T, g.DT, g.ct) - st;
+    uint32_t rem = j - st * g.H * g.W;
+    const uint32_t bh = box_of(rem / (et * g.W), g.H, g.DH, g.ch);
+    const uint32_t sh = box_start(bh, g.H, g.DH, g.ch);
+    const uint32_t eh = box_start(bh + 1, g.H, g.DH, g.ch) - sh;
+    rem -= et * sh * g.W;
+    const uint32_t bw = box_of(rem / (et * eh), g.W, g.DW, g.cw);
+    const uint32_t sw = box_start(bw, g.W, g.DW, g.cw);
+    const uint32_t ew = box_start(bw + 1, g.W, g.DW, g.cw) - sw;
+    rem -= et * eh * sw;
+    const uint32_t plane = eh * ew;
+    const uint32_t lt = rem / plane;
+    rem -= lt * plane;
+    const uint32_t lh = rem / ew;
+    t = st + lt;
+    h = sh + lh;
+    w = sw + (rem - lh * ew);
+}
+
 // Host: the geometry of a T x H x W grid cut into ct x ch x cw cubes.
 inline Geom make_geom(uint32_t T, uint32_t H, uint32_t W, uint32_t ct, uint32_t ch,
                       uint32_t cw) {
@@ -140,6 +204,7 @@ inline Geom make_geom(uint32_t T, uint32_t H, uint32_t W, uint32_t ct, uint32_t 
     g.by_cubes_w = FastDiv(g.cubes_w);
     g.by_cubes_h = FastDiv(g.cubes_h);
     g.by_L = FastDiv(g.L);
+    g.DT = g.DH = g.DW = 0;
     return g;
 }
 

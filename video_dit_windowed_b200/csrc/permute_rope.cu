@@ -115,7 +115,8 @@ __device__ __forceinline__ uint4 rotate<4>(uint4 v, const float2 *cs) {
 
 // MODE 0: dst in cube order, src raster (reorder). MODE 1: dst raster, src
 // cube order (unorder). MODE 2: dst and src raster (RoPE only). MODE 3 / 4:
-// as 0 / 1 for grids the cube does not divide (partial cubes). With ROPE the
+// as 0 / 1 for grids the cube does not divide (partial cubes). MODE 5 / 6:
+// as 0 / 1 with the aligned order of global-proxy tokens (cube_geom.cuh). With ROPE the
 // row is rotated for the grid position (t, h, w) of its token, in every mode
 // (unorder + rotation with negated scales is the transpose of reorder +
 // rotation, i.e. its gradient).
@@ -163,6 +164,12 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const Params p) 
         } else if (MODE == 4) {
             raster_coords(p.g, row, t, h, w);
             src_row = cube_position_general(p.g, t, h, w);
+        } else if (MODE == 5) {
+            geom::aligned_coords(p.g, row, t, h, w);
+            src_row = (t * p.g.H + h) * p.g.W + w;
+        } else if (MODE == 6) {
+            raster_coords(p.g, row, t, h, w);
+            src_row = geom::aligned_position(p.g, t, h, w);
         } else {
             raster_coords(p.g, row, t, h, w);
             src_row = row;
@@ -291,6 +298,13 @@ atlas_status launch(const Params &p, const DeviceInfo &dev, cudaStream_t stream)
 template <int EB>
 atlas_status dispatch(const Params &p, bool rope, int mode, bool general, const DeviceInfo &dev,
                       cudaStream_t stream) {
+    if (mode == 5 || mode == 6) {   // aligned order of global tokens
+        if (rope)
+            return mode == 5 ? launch<EB, true, 5>(p, dev, stream)
+                             : launch<EB, true, 6>(p, dev, stream);
+        return mode == 5 ? launch<EB, false, 5>(p, dev, stream)
+                         : launch<EB, false, 6>(p, dev, stream);
+    }
     if (rope) {
         if (mode == 2) return launch<EB, true, 2>(p, dev, stream);
         if (mode == 1)
@@ -365,6 +379,9 @@ void fill_geometry(Params &p, const PermuteArgs &a) {
     p.g = geom::make_geom(static_cast<uint32_t>(a.T), static_cast<uint32_t>(a.H),
                           static_cast<uint32_t>(a.W), static_cast<uint32_t>(a.ct),
                           static_cast<uint32_t>(a.ch), static_cast<uint32_t>(a.cw));
+    p.g.DT = static_cast<uint32_t>(a.DT);
+    p.g.DH = static_cast<uint32_t>(a.DH);
+    p.g.DW = static_cast<uint32_t>(a.DW);
 }
 
 }  // namespace

@@ -90,12 +90,21 @@ class Workload:
     def elem_bytes(self) -> int:
         return 2 if self.dtype == "bf16" else 4
 
-    def allowed_pairs(self, mask: str = "all", global_cube=None) -> int:
+    def aligned_boxes(self, axis: int):
+        """Global tokens aligned with each detail cube along one axis: global
+        index x of e tokens sits at detail position x*E/e, in detail cube
+        floor(x*E/(c*e)); cube b holds global indices [ceil(b*c*e/E),
+        ceil((b+1)*c*e/E)) clipped to e."""
+        E, c, e = self.grid[axis], self.cube[axis], self.global_grid[axis]
+        start = lambda b: min(-(-(b * c * e) // E), e)
+        return [start(b + 1) - start(b) for b in range(-(-E // c))]
+
+    def allowed_pairs(self, mask: str = "all") -> int:
         """Allowed (query, key) pairs of one problem and one head. mask:
         "all" (detail: own cube + every global key), "aligned" (own cube +
-        the global cube of ``global_cube`` with the same index), "raster"
-        (windows of window_len consecutive raster rows + every global key),
-        "dense" (every token sees every token)."""
+        the global tokens aligned with it), "raster" (windows of window_len
+        consecutive raster rows + every global key), "dense" (every token
+        sees every token)."""
         N, G = self.n_detail, self.n_global
         if mask == "dense":
             return (N + G) ** 2
@@ -108,13 +117,12 @@ class Workload:
             return win + N * G + G * G
         cross = 1
         for a in range(3):
-            cross *= sum(e * g for e, g in zip(self.extents(a),
-                                               self.extents(a, global_cube, self.global_grid)))
+            cross *= sum(e * g for e, g in zip(self.extents(a), self.aligned_boxes(a))) if N else 0
         return win + cross + G * G
 
-    def unmasked_flops(self, mask: str = "all", global_cube=None) -> int:
+    def unmasked_flops(self, mask: str = "all") -> int:
         """2*D FLOPs for q.k plus 2*D for p*v, per allowed (query, key) pair."""
-        return 4 * self.head_dim * self.heads * self.allowed_pairs(mask, global_cube)
+        return 4 * self.head_dim * self.heads * self.allowed_pairs(mask)
 
     def reorder_rope_bytes(self) -> int:
         """One read and one write of detail Q, K, V plus global Q, K."""
