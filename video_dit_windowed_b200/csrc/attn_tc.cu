@@ -8,17 +8,23 @@
 //
 // One softmax per query row over its allowed keys, flash style:
 //   * a work unit is one head of one problem (a batch stacks problems along
-//     the rows) and 256 consecutive query rows (two 128-row Q tiles), either
-//     detail rows (cube order) or global rows;
-//   * its key list is the detail rows of the windows its queries belong to
-//     (128-key tiles from the first window's start), then the global keys of
-//     its problem: all of them, or in the aligned variant the union of its
-//     windows' global ranges; per-row masks cut tiles that straddle a range
-//     edge, so units of windows that are multiples of 256 rows see exactly
-//     their own window;
+//     the rows) and up to 256 query rows (two 128-row Q tiles), either detail
+//     rows (cube order) or global rows;
+//   * windows of at least 128 rows get units of their own ("window units"):
+//     a fixed number of 256-row slots per window, the last one partly filled,
+//     slots past a shorter window's end skipped, so a unit never reads keys
+//     of a neighbouring window even when windows are not multiples of 256
+//     rows (partial cubes shift every later window off the 256-row grid);
+//     shorter windows pack 256 consecutive rows per unit, and the key list
+//     is then the union of their windows, cut by per-row masks;
+//   * a unit's key list is its window's detail rows (128-key tiles from the
+//     window's start), then the global keys of its problem: all of them, or
+//     in the aligned variant its window's range (the union of its windows'
+//     ranges for packed units);
 //   * windows are L rows or the ranges of an offsets array (partial cubes);
 //     ranges from offsets are clamped so that any offsets keep every access
-//     in bounds;
+//     in bounds; with offsets the kernel finds the longest window itself
+//     (every CTA scans the offsets once) and chooses the unit form;
 //   * persistent CTAs (one per SM) walk the units head-major, so the CTAs in
 //     flight share one head's global K/V in L2.
 // Warp roles per CTA (384 threads):
@@ -44,6 +50,7 @@
 #include <cuda_bf16.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "atlas_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -119,6 +126,7 @@ struct Smem {
     uint64_t o_final[kQTiles];   // every MMA of the unit done           (commit)
     uint64_t drain;
     uint32_t tmem_base;
+    int32_t max_len;     // longest window, from the offsets
     volatile int abort;
     uint32_t *err_word;
 };
@@ -130,8 +138,9 @@ struct Params {
     uint32_t *err_word;
     int32_t N, L, G, heads;  // N, G: detail and global rows of ONE problem
     float scale_log2;
-    int32_t n_dunits, n_gunits;          // units of one problem
-    int32_t units_per_prob, units_per_head, n_units, n_gtiles;
+    int32_t n_dunits, n_gunits;          // packed-form units of one problem
+    int32_t batch, n_gtiles;
+    int32_t upw;          // window units per window; 0: packed units; -1: from the offsets
     int32_t stall_unit;   // test hook: this unit's first K tile is never loaded (-1: off)
     const int32_t *win_off;   // window offsets [n_win + 1] of one problem (NULL: L rows)
     const int32_t *gwin_off;  // global key offsets [n_win + 1] per window (NULL: all keys)
@@ -166,39 +175,97 @@ __device__ __forceinline__ int32_t global_end(const Params &p, int32_t w, int32_
     return p.gwin_off == nullptr ? p.G : min(max(__ldg(p.gwin_off + w + 1), start), p.G);
 }
 
-// Work unit: one head, one problem of the batch, kUnitRows query rows.
-// Rows are per problem (q0, rows); row0 is the problem's first row in the
-// stacked tensors; kw0 / kg0 are absolute first key rows.
-struct Unit {
-    int32_t head, detail, b, q0, rows, row0, kw0, n_wtiles, kg0, n_tiles;
+// The unit form and counts, the same in every thread of every CTA.
+struct Sched {
+    int32_t upw, n_dunits, units_per_prob, units_per_head, n_units;
 };
 
-__device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
+// max_len: the longest window (clamped ranges of the offsets), when p.upw < 0.
+__device__ __forceinline__ Sched make_sched(const Params &p, int32_t max_len) {
+    Sched S;
+    S.upw = p.upw;
+    if (S.upw < 0) {
+        // Window units when windows are long enough, and their slots stay
+        // within three times the packed count (offsets mixing a long window
+        // with many short ones would otherwise make mostly empty units).
+        const int64_t upw = (max_len + kUnitRows - 1) / kUnitRows;
+        const int64_t n = static_cast<int64_t>(p.n_win) * upw;
+        const bool ok = max_len >= kBM && n <= 3 * static_cast<int64_t>(p.n_dunits) &&
+                        (n + p.n_gunits) * p.batch * p.heads <= INT32_MAX;
+        S.upw = ok ? static_cast<int32_t>(upw) : 0;
+    }
+    const int32_t n_win = p.win_off != nullptr ? p.n_win : (p.L > 0 ? p.N / p.L : 0);
+    S.n_dunits = S.upw > 0 ? n_win * S.upw : p.n_dunits;
+    S.units_per_prob = S.n_dunits + p.n_gunits;
+    S.units_per_head = S.units_per_prob * p.batch;
+    S.n_units = S.units_per_head * p.heads;
+    return S;
+}
+
+// Work unit: one head, one problem of the batch, up to kUnitRows query rows.
+// Rows are per problem: rows q0 .. qend-1 are the unit's; row0 is the
+// problem's first row in the stacked tensors; kw0 / kg0 are absolute first
+// key rows. A window unit (win >= 0) has one key range for all its rows:
+// detail [kw0, whi), global [kg0, ghi). n_tiles == 0: an empty slot.
+struct Unit {
+    int32_t head, detail, b, q0, qend, row0, kw0, n_wtiles, kg0, n_tiles, win, whi, ghi;
+};
+
+__device__ __forceinline__ Unit decode_unit(const Params &p, const Sched &S, int32_t u) {
     Unit U;
-    U.head = u / p.units_per_head;
-    int32_t lu = u - U.head * p.units_per_head;
-    U.b = lu / p.units_per_prob;
-    lu -= U.b * p.units_per_prob;
-    U.detail = lu < p.n_dunits;
+    U.head = u / S.units_per_head;
+    int32_t lu = u - U.head * S.units_per_head;
+    U.b = lu / S.units_per_prob;
+    lu -= U.b * S.units_per_prob;
+    U.detail = lu < S.n_dunits;
     int32_t n_gtiles = p.n_gtiles;
     U.kg0 = U.b * p.G;
-    if (U.detail) {
+    U.ghi = U.kg0 + p.G;
+    U.win = -1;
+    U.whi = 0;
+    if (U.detail && S.upw > 0) {
+        const int32_t w = lu / S.upw, sub = lu - w * S.upw;
+        int32_t s, e;
+        if (p.win_off != nullptr) {
+            s = min(max(__ldg(p.win_off + w), 0), p.N);
+            e = min(max(__ldg(p.win_off + w + 1), s), p.N);
+        } else {
+            s = w * p.L;
+            e = min(p.N, s + p.L);
+        }
+        U.row0 = U.b * p.N;
+        U.q0 = s + sub * kUnitRows;
+        U.qend = min(U.q0 + kUnitRows, e);
+        U.kw0 = U.row0 + s;
+        U.whi = U.row0 + e;
+        U.n_wtiles = (e - s + kBN - 1) / kBN;
+        U.win = w;
+        if (p.gwin_off != nullptr) {
+            const int32_t g0 = global_start(p, w), g1 = global_end(p, w, g0);
+            U.kg0 += g0;
+            U.ghi = U.b * p.G + g1;
+            n_gtiles = (g1 - g0 + kBN - 1) / kBN;
+        }
+        if (U.qend <= U.q0) U.n_wtiles = n_gtiles = 0;
+    } else if (U.detail) {
         U.q0 = lu * kUnitRows;
-        U.rows = p.N;
+        U.qend = min(U.q0 + kUnitRows, p.N);
         U.row0 = U.b * p.N;
         const int32_t q_last = min(U.q0 + kUnitRows, p.N) - 1;
         const int32_t w0 = window_of(p, U.q0), w1 = window_of(p, q_last);
         U.kw0 = U.row0 + window_start(p, w0, U.q0);
         const int32_t kw1 = U.row0 + window_end(p, w1, q_last);
         U.n_wtiles = (kw1 - U.kw0 + kBN - 1) / kBN;
+        U.whi = kw1;
         if (p.gwin_off != nullptr) {
             const int32_t g0 = global_start(p, w0), g1 = global_end(p, w1, g0);
             U.kg0 += g0;
+            U.ghi = U.b * p.G + g1;
             n_gtiles = (g1 - g0 + kBN - 1) / kBN;
         }
     } else {
-        U.q0 = (lu - p.n_dunits) * kUnitRows;
-        U.rows = p.G;
+        U.q0 = (lu - S.n_dunits) * kUnitRows;
+        U.qend = min(U.q0 + kUnitRows, p.G);
         U.row0 = U.b * p.G;
         U.kw0 = 0;
         U.n_wtiles = 0;
@@ -232,13 +299,22 @@ __device__ __forceinline__ bool wait_phase(Smem<HD> &sm, uint64_t &bar, uint32_t
 __device__ __forceinline__ int32_t key_row(const Unit &U, int32_t j) {
     return j < U.n_wtiles ? U.kw0 + j * kBN : U.kg0 + (j - U.n_wtiles) * kBN;
 }
+// Columns of key tile j that can hold a key allowed to some row of the unit:
+// 32, 64 or all kBN. A narrow tile's S = Q K^T is computed for those columns
+// only and its P*V reads only them; the S columns beyond are stale and never
+// read.
+__device__ __forceinline__ int32_t tile_cols(const Unit &U, int32_t j) {
+    const int32_t n = j < U.n_wtiles ? U.whi - (U.kw0 + j * kBN)
+                                      : U.ghi - (U.kg0 + (j - U.n_wtiles) * kBN);
+    return n <= 32 ? 32 : (n <= 64 ? 64 : kBN);
+}
 
 // ---------------------------------------------------------------------------
 // Producer: Q tiles once per unit, then K(0), V(0), K(1), V(1), ... in the
 // order the MMAs consume them.
 // ---------------------------------------------------------------------------
 template <int HD>
-__device__ void producer(const Params &p, Smem<HD> &sm) {
+__device__ void producer(const Params &p, const Sched &S, Smem<HD> &sm) {
     constexpr uint32_t kBytes = Smem<HD>::kTileBytes;
     constexpr int kSlots = Smem<HD>::kSlots;
     uint32_t it = 0, unit_iter = 0;
@@ -266,8 +342,9 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
         return true;
     };
 
-    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, S, u);
+        if (U.n_tiles == 0) continue;
         if (unit_iter > 0 && !(ok = wait_phase(sm, sm.q_empty, (unit_iter - 1) & 1,
                                                kErrTimeoutProducer)))
             break;
@@ -295,6 +372,7 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
             ok = load(win ? &p.tm_kd : &p.tm_kg, U.head, row) &&
                  load(win ? &p.tm_vd : &p.tm_vg, U.head, row);
         }
+        ++unit_iter;
     }
     if (!ok) {
         // Let every copy already issued land before the CTA can exit.
@@ -312,9 +390,11 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 // O0 += P0(j)V(j), S0(j+1), O1 += P1(j)V(j), S1(j+1).
 // ---------------------------------------------------------------------------
 template <int HD>
-__device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+__device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t tmem) {
     constexpr int kSlots = Smem<HD>::kSlots;
     constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(kBM, kBN, 0);
+    constexpr uint32_t kIdescQK64 = ptx::idesc_bf16_f32(kBM, 64, 0);
+    constexpr uint32_t kIdescQK32 = ptx::idesc_bf16_f32(kBM, 32, 0);
     constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, HD, 1);
     uint32_t it = 0, unit_iter = 0;
     uint32_t p_cnt = 0;   // P tiles consumed per Q tile (both tiles move together)
@@ -334,62 +414,72 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     const uint32_t k_lo0 = ptx::desc_sw128_lo(ptx::smem_addr(sm.kv[0]), 16);
     const uint32_t v_lo0 = ptx::desc_sw128_lo(ptx::smem_addr(sm.kv[0]), kBN * 128);
     constexpr uint32_t kTile16 = Smem<HD>::kTileBytes >> 4;
-    // S_i = Q_i K^T from the K tile in `slot`.
-    auto issue_s = [&](int i, uint32_t k_slot) {
+    // S_i = Q_i K^T from the K tile in `slot`, for the tile's first nc keys
+    // (the K-major operand's first nc rows: the same descriptors).
+    auto issue_s = [&](int i, uint32_t k_slot, int32_t nc) {
         const uint32_t q_lo = q_lo0 + i * kTile16, k_lo = k_lo0 + k_slot * kTile16;
         const uint32_t d_s = tmem + i * kBN;
+        const uint32_t idesc = nc == kBN ? kIdescQK : (nc == 64 ? kIdescQK64 : kIdescQK32);
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
             const uint32_t off = ((ks / 4) * (kBM * 128) + (ks % 4) * 32) >> 4;
             ptx::mma_ss(d_s, ptx::desc_join(q_lo + off, kHi), ptx::desc_join(k_lo + off, kHi),
-                        kIdescQK, ks > 0);
+                        idesc, ks > 0);
         }
         ptx::mma_commit(ptx::smem_addr(&sm.s_full[i]));
     };
-    // O_i += P_i V, P_i from tensor memory, from the V tile in `slot`.
-    auto issue_pv = [&](int i, uint32_t v_slot, bool first) -> bool {
+    // O_i += P_i V, P_i from tensor memory, from the V tile in `slot`; the
+    // first nc keys only (nc / 16 steps of K = 16).
+    auto issue_pv = [&](int i, uint32_t v_slot, bool first, int32_t nc) -> bool {
         if (!wait_phase(sm, sm.p_full[i], p_cnt & 1, kErrTimeoutMma)) return false;
         ptx::tc_fence_after();
         const uint32_t v_lo = v_lo0 + v_slot * kTile16;
         const uint32_t d_o = tmem + 2 * kBN + i * HD, a_p = tmem + i * kBN;
         ptx::mma_ts(d_o, a_p, ptx::desc_join(v_lo, kHi), kIdescPV, first ? 0u : 1u);
 #pragma unroll
-        for (int ks = 1; ks < kBN / 16; ++ks)
+        for (int ks = 1; ks < kBN / 16; ++ks) {
+            if (ks * 16 >= nc) break;
             ptx::mma_ts(d_o, a_p + ks * 8, ptx::desc_join(v_lo + ((ks * 16 * 128) >> 4), kHi),
                         kIdescPV, 1u);
+        }
         return true;
     };
 
-    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, S, u);
+        if (U.n_tiles == 0) continue;
         for (int i = 0; i < kQTiles && ok; ++i)
             ok = wait_phase(sm, sm.q_full[i], unit_iter & 1, kErrTimeoutMma);
         if (!ok) break;
         ptx::tc_fence_after();
         uint32_t k_slot, v_slot;
         if (!(ok = next_slot(k_slot))) break;
-        issue_s(0, k_slot);
-        issue_s(1, k_slot);
+        int32_t nc = tile_cols(U, 0);
+        issue_s(0, k_slot, nc);
+        issue_s(1, k_slot, nc);
         ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
             const bool more = j + 1 < U.n_tiles;
+            const int32_t nc_next = more ? tile_cols(U, j + 1) : 0;
             // ring order: V(j) was loaded before K(j+1)
-            if (!(ok = next_slot(v_slot)) || !(ok = issue_pv(0, v_slot, j == 0))) break;
+            if (!(ok = next_slot(v_slot)) || !(ok = issue_pv(0, v_slot, j == 0, nc))) break;
             if (more) {
                 if (!(ok = next_slot(k_slot))) break;
-                issue_s(0, k_slot);
+                issue_s(0, k_slot, nc_next);
             }
-            if (!(ok = issue_pv(1, v_slot, j == 0))) break;
+            if (!(ok = issue_pv(1, v_slot, j == 0, nc))) break;
             if (more) {
-                issue_s(1, k_slot);
+                issue_s(1, k_slot, nc_next);
                 ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
             }
+            nc = nc_next;
             ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[v_slot]));
             ++p_cnt;
         }
         if (!ok) break;
         for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
         ptx::mma_commit(ptx::smem_addr(&sm.q_empty));
+        ++unit_iter;
     }
     // Drain: every MMA issued must finish before tensor memory is freed.
     ptx::mma_commit(ptx::smem_addr(&sm.drain));
@@ -400,7 +490,8 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
 // Softmax + epilogue of Q tile `qt`; 128 threads, thread = row = TMEM lane.
 // ---------------------------------------------------------------------------
 template <int HD>
-__device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, int qt) {
+__device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t tmem,
+                                 int qt) {
     const uint32_t warp = (threadIdx.x / 32) & 3;
     const uint32_t r = threadIdx.x & 127;                 // row within the tile
     const uint32_t lane_sel = (warp * 32u) << 16;         // TMEM lane field
@@ -410,34 +501,14 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
     const float sc = p.scale_log2;
     constexpr uint32_t kAll = 0xffffffffu;
 
-    // P = exp2(S*scale*log2e - m) as bf16 pairs into tensor memory (two
-    // stores of 32 columns); returns the row sum of the fp32 P.
-    auto exp_store = [&](const uint32_t (&sr)[kBN], float m) -> float {
-        float sum8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int c = half * 64 + 2 * e;
-                const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c]), sc, -m));
-                const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c + 1]), sc, -m));
-                sum8[e & 7] += p0 + p1;
-                pk[e] = ptx::pack_bf16x2(p0, p1);
-            }
-            ptx::tmem_st32_nowait(t_s + half * 32, pk);
-        }
-        ptx::tmem_wait_st();
-#pragma unroll
-        for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-            for (int k = 0; k < w; ++k) sum8[k] += sum8[k + w];
-        return sum8[0];
-    };
-    // The same, with the row maximum of the raw S taken in the same pass.
-    auto exp_store_max = [&](const uint32_t (&sr)[kBN], float m, float &mx) -> float {
+    // P = exp2(S*scale*log2e - m) of the NC columns in `sr`, as bf16 pairs
+    // into tensor memory (stores of 32 packed columns; one of 16 for a
+    // 32-column tile); returns the row sum of the fp32 P. WithMax: the row
+    // maximum of the raw S is taken in the same pass, into mx.
+    auto exp_store = [&](auto with_max, const auto &sr, float m, float &mx) -> float {
+        constexpr bool kWithMax = decltype(with_max)::value;
+        constexpr int NC = static_cast<int>(sizeof(sr) / sizeof(uint32_t));
+        constexpr int kPer = NC >= 64 ? 32 : 16;
         float sum8[8], m8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -445,19 +516,22 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
             m8[k] = kNegInf;
         }
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t pk[32];
+        for (int g = 0; g < NC / (2 * kPer); ++g) {
+            uint32_t pk[kPer];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int c = half * 64 + 2 * e;
+            for (int e = 0; e < kPer; ++e) {
+                const int c = g * 2 * kPer + 2 * e;
                 const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
-                m8[e & 7] = ptx::max3(m8[e & 7], s0, s1);
+                if constexpr (kWithMax) m8[e & 7] = ptx::max3(m8[e & 7], s0, s1);
                 const float p0 = ptx::ex2(fmaf(s0, sc, -m));
                 const float p1 = ptx::ex2(fmaf(s1, sc, -m));
                 sum8[e & 7] += p0 + p1;
                 pk[e] = ptx::pack_bf16x2(p0, p1);
             }
-            ptx::tmem_st32_nowait(t_s + half * 32, pk);
+            if constexpr (kPer == 32)
+                ptx::tmem_st32_nowait(t_s + g * 32, pk);
+            else
+                ptx::tmem_st16_nowait(t_s + g * 16, pk);
         }
         ptx::tmem_wait_st();
 #pragma unroll
@@ -465,20 +539,24 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
 #pragma unroll
             for (int k = 0; k < w; ++k) {
                 sum8[k] += sum8[k + w];
-                m8[k] = fmaxf(m8[k], m8[k + w]);
+                if constexpr (kWithMax) m8[k] = fmaxf(m8[k], m8[k + w]);
             }
-        mx = m8[0];
+        if constexpr (kWithMax) mx = m8[0];
         return sum8[0];
     };
-    auto row_max = [&](const uint32_t (&sr)[kBN]) -> float {
+    // Row maximum of the NC columns in `sr` (NC a multiple of 16).
+    auto row_max = [&](const auto &sr) -> float {
+        constexpr int NC = static_cast<int>(sizeof(sr) / sizeof(uint32_t));
         float m8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(sr[k]);
 #pragma unroll
-        for (int c = 8; c < kBN; c += 16)
+        for (int c = 8; c + 16 <= NC; c += 16)
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 m8[k] = ptx::max3(m8[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], __uint_as_float(sr[NC - 8 + k]));
         return ptx::max3(ptx::max3(m8[0], m8[1], m8[2]), ptx::max3(m8[3], m8[4], m8[5]),
                          fmaxf(m8[6], m8[7]));
     };
@@ -498,13 +576,16 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
     };
 
     uint32_t cnt = 0, unit_iter = 0;   // key tiles processed (all units)
-    for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units; u += gridDim.x) {
+        const Unit U = decode_unit(p, S, u);
+        if (U.n_tiles == 0) continue;
         const int32_t q = U.q0 + qt * kBM + static_cast<int32_t>(r);
-        const bool row_valid = q < U.rows;
+        const bool row_valid = q < U.qend;
         // Allowed keys (absolute rows): detail [lo, hi), global [glo, ghi).
-        int32_t lo = 0, hi = 0, glo = U.b * p.G, ghi = glo + p.G;
-        if (U.detail) {
+        int32_t lo = U.kw0, hi = U.whi, glo = U.kg0, ghi = U.ghi;
+        if (U.detail && U.win < 0) {
+            glo = U.b * p.G;
+            ghi = glo + p.G;
             const int32_t qc = min(q, p.N - 1);
             const int32_t w = window_of(p, qc);
             lo = U.row0 + window_start(p, w, qc);
@@ -519,50 +600,65 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
         for (int32_t j = 0; j < U.n_tiles; ++j, ++cnt) {
             if (!__all_sync(kAll, wait_phase(sm, sm.s_full[qt], cnt & 1, err))) return;
             ptx::tc_fence_after();
-            uint32_t sr[kBN];
-            ptx::tmem_ld128(t_s, sr);
             // Mask keys outside this row's allowed range.
             const int32_t k0 = key_row(U, j);
             const int32_t klo = j < U.n_wtiles ? lo : glo;
             const int32_t khi = j < U.n_wtiles ? hi : ghi;
             const bool row_masked = k0 < klo || k0 + kBN > khi;
-            if (row_masked) {
+            // One key tile of NC columns (all 128, or the first 64 or 32 of a
+            // narrow tile: the others hold no allowed key of any row).
+            auto tile = [&](auto ncw) -> float {
+                constexpr int NC = decltype(ncw)::value;
+                uint32_t sr[NC];
+                if constexpr (NC == 128)
+                    ptx::tmem_ld128(t_s, sr);
+                else if constexpr (NC == 64)
+                    ptx::tmem_ld64(t_s, sr);
+                else
+                    ptx::tmem_ld32(t_s, sr);
+                if (row_masked) {
 #pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
-            }
-            float sum;
-            if (__any_sync(kAll, m_run == kNegInf || row_masked)) {
-                // No reference yet, or masked keys: row max first. The
-                // reference moves only when the tile's max exceeds it by more
-                // than the threshold (exact either way: O and l share it).
-                const float mx2 = row_max(sr) * sc;
-                const bool need = (m_run == kNegInf) ? (mx2 != kNegInf)
-                                                     : (mx2 > m_run + kRescaleThreshold);
-                float alpha = 1.f;
-                if (need) {
-                    alpha = (m_run == kNegInf) ? 0.f : ptx::ex2(m_run - mx2);
-                    m_run = mx2;
+                    for (int c = 0; c < NC; ++c)
+                        if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
                 }
-                l_run *= alpha;
-                if (j > 0) rescale_o(need, alpha);
-                sum = exp_store(sr, m_run == kNegInf ? 0.f : m_run);
-            } else {
-                // Exponentials against the running reference right away, the
-                // tile max in the same pass; redo the (rare) rows whose max
-                // moved past the threshold.
-                float mx;
-                sum = exp_store_max(sr, m_run, mx);
-                const float mx2 = mx * sc;
-                const bool need = mx2 > m_run + kRescaleThreshold;
-                if (__any_sync(kAll, need)) {
-                    const float alpha = need ? ptx::ex2(m_run - mx2) : 1.f;
-                    if (need) m_run = mx2;
+                float sum, mx;
+                if (__any_sync(kAll, m_run == kNegInf || row_masked)) {
+                    // No reference yet, or masked keys: row max first. The
+                    // reference moves only when the tile's max exceeds it by
+                    // more than the threshold (exact either way: O and l
+                    // share it).
+                    const float mx2 = row_max(sr) * sc;
+                    const bool need = (m_run == kNegInf) ? (mx2 != kNegInf)
+                                                         : (mx2 > m_run + kRescaleThreshold);
+                    float alpha = 1.f;
+                    if (need) {
+                        alpha = (m_run == kNegInf) ? 0.f : ptx::ex2(m_run - mx2);
+                        m_run = mx2;
+                    }
                     l_run *= alpha;
-                    rescale_o(need, alpha);
-                    sum = exp_store(sr, m_run);
+                    if (j > 0) rescale_o(need, alpha);
+                    sum = exp_store(std::false_type{}, sr, m_run == kNegInf ? 0.f : m_run, mx);
+                } else {
+                    // Exponentials against the running reference right away,
+                    // the tile max in the same pass; redo the (rare) rows
+                    // whose max moved past the threshold.
+                    sum = exp_store(std::true_type{}, sr, m_run, mx);
+                    const float mx2 = mx * sc;
+                    const bool need = mx2 > m_run + kRescaleThreshold;
+                    if (__any_sync(kAll, need)) {
+                        const float alpha = need ? ptx::ex2(m_run - mx2) : 1.f;
+                        if (need) m_run = mx2;
+                        l_run *= alpha;
+                        rescale_o(need, alpha);
+                        sum = exp_store(std::false_type{}, sr, m_run, mx);
+                    }
                 }
-            }
+                return sum;
+            };
+            const int32_t nc = tile_cols(U, j);
+            const float sum = nc == kBN ? tile(std::integral_constant<int, kBN>{})
+                              : nc == 64 ? tile(std::integral_constant<int, 64>{})
+                                         : tile(std::integral_constant<int, 32>{});
             l_run += sum;
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
@@ -601,6 +697,7 @@ __device__ void softmax_epilogue(const Params &p, Smem<HD> &sm, uint32_t tmem, i
                 (m_run + __log2f(l_run)) * 0.69314718055994531f;
         }
         ptx::tc_fence_before();
+        ++unit_iter;
     }
 }
 
@@ -625,6 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         ptx::mbar_init(ptx::smem_addr(&sm.drain), 1);
         sm.abort = 0;
+        sm.max_len = 0;
         sm.err_word = p.err_word;
         ptx::fence_mbar_init();
     }
@@ -643,6 +741,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
+    if (p.upw < 0) {
+        // The longest window: one pass over the offsets per CTA.
+        int32_t m = 0;
+        for (int32_t w = threadIdx.x; w < p.n_win; w += kThreads) {
+            const int32_t s = min(max(__ldg(p.win_off + w), 0), p.N);
+            m = max(m, min(max(__ldg(p.win_off + w + 1), s), p.N) - s);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) atomicMax(&sm.max_len, m);
+        __syncthreads();
+    }
+    const Sched S = make_sched(p, sm.max_len);
     const uint32_t tmem = sm.tmem_base;
     // A 512-column allocation always starts at column 0 of lane 0.
     const bool tmem_ok = tmem == 0;
@@ -652,12 +763,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        if (tmem_ok) softmax_epilogue<HD>(p, sm, tmem, warp / 4);
+        if (tmem_ok) softmax_epilogue<HD>(p, S, sm, tmem, warp / 4);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (tmem_ok && lane == 0) {
-            if (warp == kProducerWarp) producer<HD>(p, sm);
-            if (warp == kMmaWarp) mma_issuer<HD>(p, sm, tmem);
+            if (warp == kProducerWarp) producer<HD>(p, S, sm);
+            if (warp == kMmaWarp) mma_issuer<HD>(p, S, sm, tmem);
         }
     }
     __syncwarp();
@@ -697,22 +808,35 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.n_dunits = static_cast<int32_t>((a.n_detail + kUnitRows - 1) / kUnitRows);
     p.n_gunits = static_cast<int32_t>((a.n_global + kUnitRows - 1) / kUnitRows);
-    p.units_per_prob = p.n_dunits + p.n_gunits;
-    if (p.units_per_prob == 0) return ATLAS_OK;
-    if (static_cast<int64_t>(p.units_per_prob) * a.batch * a.heads > INT32_MAX)
-        return ATLAS_ERR_SHAPE;
-    p.units_per_head = p.units_per_prob * static_cast<int32_t>(a.batch);
-    p.n_units = p.units_per_head * a.heads;
+    const int64_t packed_units = static_cast<int64_t>(p.n_dunits) + p.n_gunits;
+    if (packed_units == 0) return ATLAS_OK;
+    if (packed_units * a.batch * a.heads > INT32_MAX) return ATLAS_ERR_SHAPE;
+    p.batch = static_cast<int32_t>(a.batch);
     p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
     p.stall_unit = take_stall_request() ? 0 : -1;
     p.win_off = a.win_off;
     p.gwin_off = a.gwin_off;
     p.n_win = static_cast<int32_t>(a.win_off ? a.n_win : a.n_gwin);
+    // Unit form: window units for windows of at least one Q tile. Fixed
+    // windows decide here (their slots never exceed three times the packed
+    // count); offsets are read by the kernel only.
+    int64_t n_units = packed_units * a.batch * a.heads;
+    if (!has_d) {
+        p.upw = 0;
+    } else if (a.win_off != nullptr) {
+        p.upw = -1;
+        n_units = std::max<int64_t>(n_units, dev.sm_count);
+    } else {
+        p.upw = p.L >= kBM ? (p.L + kUnitRows - 1) / kUnitRows : 0;
+        if (p.upw > 0)
+            n_units = (static_cast<int64_t>(p.N / p.L) * p.upw + p.n_gunits) * a.batch * a.heads;
+        if (n_units > INT32_MAX) return ATLAS_ERR_SHAPE;
+    }
     const size_t smem = sizeof(Smem<HD>) + 1024;
     if (!set_smem_limit(reinterpret_cast<const void *>(attn_tc_kernel<HD>),
                         static_cast<int>(smem)))
         return ATLAS_ERR_CUDA;
-    const int grid = std::min(p.n_units, dev.sm_count);
+    const int grid = static_cast<int>(std::min<int64_t>(n_units, dev.sm_count));
     attn_tc_kernel<HD><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
