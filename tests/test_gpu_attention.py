@@ -52,6 +52,9 @@ SMALL = [
     (512, 1, 64, 2, 128, "bf16"),       # 1x1x1 cubes: each row sees itself and the globals
     (2048, 512, 300, 2, 64, "bf16"),    # head_dim 64
     (3072, 1536, 500, 1, 128, "bf16"),  # long windows
+    (1920, 384, 65, 2, 128, "bf16"),    # 1.5 units per window: a half-empty second unit
+    (2560, 640, 33, 2, 128, "bf16"),    # 2.5 units per window; a 64-key global tile
+    (1280, 640, 20, 1, 64, "bf16"),     # a 32-key global tile at head_dim 64
     (768, 768, 0, 2, 128, "bf16"),      # no global tokens (pure window attention)
     (0, 1, 1000, 2, 128, "bf16"),       # global tokens only
     (600, 100, 50, 2, 128, "fp32"),

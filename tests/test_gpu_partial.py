@@ -194,3 +194,70 @@ def test_long_shapes_full_size_sampled(name):
         assert float((t.float() - 1).abs().max()) <= 8e-3
     del q_d, k_d, v_d, q_g, k_g, v_g, o_d, o_g
     torch.cuda.empty_cache()
+
+
+# Window offsets that exercise both unit forms of the tensor-core forward:
+# long windows of unequal lengths (own units, empty trailing slots, a
+# 100-row window and a one-row window inside a long-window layout), and a
+# layout whose slots would exceed three times the packed count (one long
+# window among many short ones: packed units over the union of windows).
+OFFSET_CASES = [
+    [0, 700, 1212, 1213, 1313, 2081, 2336, 2592],
+    [0, 1000] + list(range(1001, 1501)),
+    [0, 128, 256, 384, 640, 900],
+    [0, 384, 768, 1152],
+]
+
+
+@pytest.mark.parametrize("offsets", OFFSET_CASES)
+@pytest.mark.parametrize("aligned", [False, True])
+def test_window_units_match_oracle(offsets, aligned):
+    """Variable windows against the oracle, all keys or per-window global
+    ranges (some empty), bf16 on the tensor-core path."""
+    off = torch.tensor(offsets, dtype=torch.int32)
+    N, G, heads, hd = offsets[-1], 333, 2, 128
+    nw = len(offsets) - 1
+    t = {s: normal((N if s.endswith("_d") else G, heads, hd), s, torch.bfloat16, seed=31,
+                   device=DEV) for s in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")}
+    gwin = None
+    if aligned:
+        rng = np.random.default_rng(5)
+        cuts = np.sort(rng.integers(0, G + 1, size=nw - 1))
+        cuts[nw // 2 - 1:nw // 2 + 1] = cuts[nw // 2 - 1]       # an empty range
+        gwin = np.concatenate([[0], cuts, [G]]).astype(np.int32)
+    o_d, o_g = torch.empty_like(t["q_d"]), torch.empty_like(t["q_g"])
+    lse = torch.empty(1, heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_ex(
+        t["q_d"], t["k_d"], t["v_d"], t["q_g"], t["k_g"], t["v_g"], o_d, o_g, lse,
+        window_offsets=off.to(DEV),
+        global_window_offsets=torch.from_numpy(gwin).to(DEV) if aligned else None)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    woff = np.asarray(offsets, dtype=np.int64)
+    for h in range(heads):
+        kd, vd = f64(t["k_d"][:, h]), f64(t["v_d"][:, h])
+        kg, vg = f64(t["k_g"][:, h]), f64(t["v_g"][:, h])
+        q = np.concatenate([f64(t["q_d"][:, h]), f64(t["q_g"][:, h])])
+        if aligned:
+            # window w alone, with its global range as the whole global set
+            parts, lparts = [], []
+            for w in range(nw):
+                s0, e0, g0, g1 = int(woff[w]), int(woff[w + 1]), int(gwin[w]), int(gwin[w + 1])
+                o_w, l_w = orc().attention_head(e0 - s0, e0 - s0, g1 - g0, hd ** -0.5,
+                                                kd[s0:e0], vd[s0:e0], 0, kg[g0:g1], vg[g0:g1],
+                                                np.arange(e0 - s0, dtype=np.int64), q[s0:e0],
+                                                n_threads())
+                parts.append(o_w)
+                lparts.append(l_w)
+            o_g_ref, l_g_ref = orc().attention_head(0, 1, G, hd ** -0.5, None, None, 0, kg, vg,
+                                                    np.arange(G, dtype=np.int64), q[N:],
+                                                    n_threads())
+            ref = np.concatenate(parts + [o_g_ref])
+            ref_l = np.concatenate(lparts + [l_g_ref])
+        else:
+            ref, ref_l = orc().attention_head(N, 1, G, hd ** -0.5, kd, vd, 0, kg, vg,
+                                              np.arange(N + G, dtype=np.int64), q, n_threads(),
+                                              woff)
+        got = np.concatenate([f64(o_d[:, h]), f64(o_g[:, h])])
+        assert_attn_close(got, ref, "bf16", f"{offsets[:4]} head {h}")
+        assert np.max(np.abs(f64(lse[0, h]) - ref_l)) <= 5e-3
