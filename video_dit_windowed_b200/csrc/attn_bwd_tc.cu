@@ -20,6 +20,12 @@
 // the compute threads), so its S and dP MMAs read only the streamed half
 // from shared memory (TS form); DKDV has no tensor memory to spare for K and
 // V and reads them from shared memory (SS form).
+// Resident tiles of detail rows follow the forward's unit forms: windows of
+// at least 128 rows get tiles of their own (a fixed number of slots per
+// window, the last one partly filled, slots past a shorter window's end
+// skipped), so a tile never streams a neighbouring window's rows; shorter
+// windows pack 128 consecutive rows. With window offsets the kernel finds the
+// longest window itself.
 // Either way a streamed tile of 128 rows is taken in two halves of 64, each
 // loaded into its own stage of the shared-memory ring (so three halves can
 // be in flight while one is used; the streamed queries' LSE and delta ride in
@@ -84,6 +90,7 @@ struct Smem {
     uint64_t acc_full, acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
+    int32_t max_len;     // longest window, from the offsets
     volatile int abort;
     uint32_t *err_word;
 };
@@ -101,8 +108,32 @@ struct Params {
     int32_t n_win;
     int32_t tiles_d, tiles_g;           // 128-row tiles of one problem's detail / global rows
     int32_t n_long;                     // DKDV: units over global keys (scheduled first)
-    int32_t n_units;
+    int32_t upw;   // detail tiles per window; 0: packed tiles; -1: from the offsets
 };
+
+// The unit form and counts, the same in every thread of every CTA.
+struct Sched {
+    int32_t upw, n_dunits, n_units;
+};
+
+// max_len: the longest window (clamped ranges of the offsets), when p.upw < 0.
+__device__ __forceinline__ Sched make_sched(const Params &p, int32_t max_len) {
+    Sched S;
+    S.upw = p.upw;
+    if (S.upw < 0) {
+        // Tiles of their own when windows are long enough, and their slots
+        // stay within three times the packed count.
+        const int64_t upw = (max_len + kRows - 1) / kRows;
+        const int64_t n = static_cast<int64_t>(p.n_win) * upw;
+        const bool ok = max_len >= kRows && n <= 3 * static_cast<int64_t>(p.tiles_d) &&
+                        (n + p.tiles_g) * p.batch * p.heads <= INT32_MAX;
+        S.upw = ok ? static_cast<int32_t>(upw) : 0;
+    }
+    const int32_t n_win = p.win_off != nullptr ? p.n_win : (p.L > 0 ? p.N / p.L : 0);
+    S.n_dunits = S.upw > 0 ? n_win * S.upw : p.tiles_d;
+    S.n_units = (S.n_dunits + p.tiles_g) * p.batch * p.heads;
+    return S;
+}
 
 // ---- window geometry (per problem; as the forward) --------------------------
 __device__ __forceinline__ int32_t window_of(const Params &p, int32_t x) {
@@ -150,58 +181,96 @@ __device__ __forceinline__ int32_t window_of_global(const Params &p, int32_t g) 
     return (s <= g && g < global_end(p, lo, s)) ? lo : -1;
 }
 
-// A work unit: one head, one problem, 128 resident rows, and the streamed
-// tiles: n_a tiles of detail rows from row a0, then n_b tiles of global rows
-// from row b0 (rows within the problem).
+// A work unit: one head, one problem, resident rows r0 .. rend-1, and the
+// streamed tiles: n_a tiles of detail rows from row a0 (rows up to a_end),
+// then n_b tiles of global rows from row b0 (up to b_end); rows within the
+// problem. win >= 0: a window tile, whose rows all see the same ranges.
+// n_a + n_b == 0: an empty slot.
 struct Unit {
-    int32_t head, b, detail, r0, rows, a0, n_a, b0, n_b;
+    int32_t head, b, detail, r0, rend, a0, n_a, a_end, b0, n_b, b_end, win;
 };
 
+// Resident tile `lu` of one problem's detail rows in window form: the
+// window's rows are streamed (and, for DQ, its global range).
 template <int FORM>
-__device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
+__device__ __forceinline__ void window_tile(const Params &p, const Sched &S, int32_t lu,
+                                            Unit &U) {
+    const int32_t w = lu / S.upw, sub = lu - w * S.upw;
+    int32_t s, e;
+    window_rows(p, w, s, e);
+    U.win = w;
+    U.r0 = s + sub * kRows;
+    U.rend = min(U.r0 + kRows, e);
+    U.a0 = s;
+    U.a_end = e;
+    U.n_a = (e - s + kRows - 1) / kRows;
+    U.b0 = U.n_b = U.b_end = 0;
+    if (FORM == kDQ) {
+        const int32_t g0 = global_start(p, w), g1 = global_end(p, w, g0);
+        U.b0 = g0;
+        U.b_end = g1;
+        U.n_b = (g1 - g0 + kRows - 1) / kRows;
+    }
+    if (U.rend <= U.r0) U.n_a = U.n_b = 0;
+}
+
+template <int FORM>
+__device__ __forceinline__ Unit decode_unit(const Params &p, const Sched &S, int32_t u) {
     Unit U;
-    const int32_t per_prob = p.tiles_d + p.tiles_g;
+    U.win = -1;
+    const int32_t per_prob = S.n_dunits + p.tiles_g;
     if (FORM == kDQ) {
         U.head = u / (per_prob * p.batch);
         int32_t lu = u - U.head * per_prob * p.batch;
         U.b = lu / per_prob;
         lu -= U.b * per_prob;
-        U.detail = lu < p.tiles_d;
-        U.r0 = (U.detail ? lu : lu - p.tiles_d) * kRows;
-        U.rows = U.detail ? p.N : p.G;
+        U.detail = lu < S.n_dunits;
+        if (U.detail && S.upw > 0) {
+            window_tile<FORM>(p, S, lu, U);
+            return U;
+        }
+        U.r0 = (U.detail ? lu : lu - S.n_dunits) * kRows;
+        U.rend = min(U.r0 + kRows, U.detail ? p.N : p.G);
         U.n_a = 0;
-        U.a0 = 0;
+        U.a0 = U.a_end = 0;
         int32_t g0 = 0, g1 = p.G;
         if (U.detail) {
-            const int32_t last = min(U.r0 + kRows, p.N) - 1;
+            const int32_t last = U.rend - 1;
             const int32_t w0 = window_of(p, U.r0), w1 = window_of(p, last);
             U.a0 = window_start(p, w0, U.r0);
-            U.n_a = (window_end(p, w1, last) - U.a0 + kRows - 1) / kRows;
+            U.a_end = window_end(p, w1, last);
+            U.n_a = (U.a_end - U.a0 + kRows - 1) / kRows;
             if (p.gwin_off != nullptr) {
                 g0 = global_start(p, w0);
                 g1 = max(global_end(p, w1, g0), g0);
             }
         }
         U.b0 = g0;
+        U.b_end = g1;
         U.n_b = (g1 - g0 + kRows - 1) / kRows;
     } else {
         // global-key units first (they stream every query that sees them)
         const bool long_unit = u < p.n_long;
-        const int32_t span = long_unit ? p.tiles_g : p.tiles_d;
+        const int32_t span = long_unit ? p.tiles_g : S.n_dunits;
         const int32_t v = long_unit ? u : u - p.n_long;
         U.head = v / (span * p.batch);
         int32_t lv = v - U.head * span * p.batch;
         U.b = lv / span;
         lv -= U.b * span;
         U.detail = !long_unit;
+        if (U.detail && S.upw > 0) {
+            window_tile<FORM>(p, S, lv, U);
+            return U;
+        }
         U.r0 = lv * kRows;
-        U.rows = U.detail ? p.N : p.G;
-        const int32_t last = min(U.r0 + kRows, U.rows) - 1;
+        U.rend = min(U.r0 + kRows, U.detail ? p.N : p.G);
+        const int32_t last = U.rend - 1;
         if (U.detail) {
             const int32_t w0 = window_of(p, U.r0), w1 = window_of(p, last);
             U.a0 = window_start(p, w0, U.r0);
-            U.n_a = (window_end(p, w1, last) - U.a0 + kRows - 1) / kRows;
-            U.b0 = 0;
+            U.a_end = window_end(p, w1, last);
+            U.n_a = (U.a_end - U.a0 + kRows - 1) / kRows;
+            U.b0 = U.b_end = 0;
             U.n_b = 0;
         } else {
             int32_t q0 = 0, q1 = p.N;
@@ -220,8 +289,10 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, int32_t u) {
                 }
             }
             U.a0 = q0;
+            U.a_end = q1;
             U.n_a = (q1 - q0 + kRows - 1) / kRows;
             U.b0 = 0;
+            U.b_end = p.G;
             U.n_b = p.tiles_g;
         }
     }
@@ -263,7 +334,7 @@ __device__ __forceinline__ int32_t streamed_row(const Unit &U, int32_t j) {
 // barrier.
 // ---------------------------------------------------------------------------
 template <int HD, int FORM>
-__device__ void producer(const Params &p, Smem<HD> &sm) {
+__device__ void producer(const Params &p, const Sched &S, Smem<HD> &sm) {
     constexpr int kStages = Smem<HD>::kStages;
     constexpr uint32_t kTile = Smem<HD>::kTile, kHalfTile = Smem<HD>::kHalfTile;
     constexpr uint32_t kAll = 0xffffffffu;
@@ -281,8 +352,9 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
             ptx::tma_load_3d(ptx::smem_addr(dst + db * box_bytes), map, bar, db * 64, head,
                              row);
     };
-    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit<FORM>(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit<FORM>(p, S, u);
+        if (U.n_a + U.n_b == 0) continue;
         // Every lane waits and the warp agrees, so the lanes never diverge
         // around the warp-wide steps below. (DQ: the compute warps put the
         // resident Q and dO rows in tensor memory themselves.)
@@ -341,6 +413,7 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
             for (int t = 0; t < kStages; ++t)
                 if (t == static_cast<int>(s)) armed[t] = round + 1;
         }
+        ++unit_iter;
     }
     if (!ok && lane == 0) {
         // Let every copy already issued land before the CTA can exit.
@@ -357,7 +430,7 @@ __device__ void producer(const Params &p, Smem<HD> &sm) {
 // S_h, dP_h of tile j+1.
 // ---------------------------------------------------------------------------
 template <int HD, int FORM>
-__device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+__device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t tmem) {
     constexpr int kStages = Smem<HD>::kStages;
     constexpr uint32_t kH16 = Smem<HD>::kHalfTile >> 4;
     constexpr uint32_t kIdS = ptx::idesc_bf16_f32(kRows, kHalf, 0);   // S_h, dP_h
@@ -372,7 +445,8 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     const uint32_t xs_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.xs[0]), kHalf * 128);
     const uint32_t ys_mn = ptx::desc_sw128_lo(ptx::smem_addr(sm.ys[0]), kHalf * 128);
     const uint32_t t_s = tmem, t_dp = tmem + 2 * kHalf, t_acc = tmem + 4 * kHalf;
-    uint32_t it = 0, unit_iter = 0, p_cnt = 0;
+    uint32_t it = 0, unit_iter = 0;
+    uint32_t p_cnt = 0;
     bool ok = true;
 
     const uint32_t t_x = t_acc + HD, t_y = t_x + HD / 2;   // DQ: resident Q, dO (packed)
@@ -416,9 +490,10 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         return r;
     };
 
-    for (int32_t u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit<FORM>(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit<FORM>(p, S, u);
         const int32_t n = U.n_a + U.n_b;
+        if (n == 0) continue;
         if (!(ok = wait_phase(sm, sm.x_full, unit_iter & 1, kErrTimeoutMma))) break;
         ptx::tc_fence_after();
         uint32_t st[2];   // stages of the current tile's halves
@@ -452,6 +527,7 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&sm.acc_full));
         ptx::mma_commit(ptx::smem_addr(&sm.x_empty));
+        ++unit_iter;
     }
     // Drain: every MMA issued must finish before tensor memory is freed.
     ptx::mma_commit(ptx::smem_addr(&sm.drain));
@@ -462,7 +538,7 @@ __device__ void mma_issuer(const Params &p, Smem<HD> &sm, uint32_t tmem) {
 // Compute warps: thread = resident row = tensor-memory lane.
 // ---------------------------------------------------------------------------
 template <int HD, int FORM>
-__device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
+__device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t tmem) {
     constexpr int kStages = Smem<HD>::kStages;
     constexpr int kCols = kHalf / 2;                 // columns of a half per warpgroup
     constexpr uint32_t kAll = 0xffffffffu;
@@ -475,10 +551,11 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
     const float c2 = p.scale_log2;
     uint32_t cnt = 0, unit_iter = 0;
 
-    for (int32_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++unit_iter) {
-        const Unit U = decode_unit<FORM>(p, u);
+    for (int32_t u = blockIdx.x; u < S.n_units; u += gridDim.x) {
+        const Unit U = decode_unit<FORM>(p, S, u);
+        if (U.n_a + U.n_b == 0) continue;
         const int32_t row = U.r0 + static_cast<int32_t>(r);   // resident row (in problem)
-        const bool valid = row < U.rows;
+        const bool valid = row < U.rend;
         // Allowed streamed rows: [da, db) of detail tiles, [ga, gb) of global tiles.
         int32_t da = 0, db = 0, ga = 0, gb = 0;
         float lse2_own = 0.f, delta_own = 0.f;
@@ -486,7 +563,12 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
             if (FORM == kDQ) {
                 ga = 0;
                 gb = p.G;
-                if (U.detail) {
+                if (U.detail && U.win >= 0) {
+                    da = U.a0;
+                    db = U.a_end;
+                    ga = U.b0;
+                    gb = U.b_end;
+                } else if (U.detail) {
                     const int32_t w = window_of(p, row);
                     da = window_start(p, w, row);
                     db = window_end(p, w, row);
@@ -497,6 +579,9 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                                         (p.N + p.G) + (U.detail ? row : p.N + row);
                 lse2_own = __ldg(p.lse + col) * kLog2e;
                 delta_own = __ldg(p.delta + col);
+            } else if (U.detail && U.win >= 0) {
+                da = U.a0;
+                db = U.a_end;
             } else if (U.detail) {
                 const int32_t w = window_of(p, row);
                 da = window_start(p, w, row);
@@ -552,12 +637,12 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
 #pragma unroll 1
             for (int h = 0; h < 2; ++h) {
                 // ring stage of this half tile (the producer's order)
-                const uint32_t hc = 2 * cnt + h, stage = hc % kStages;
+                const uint32_t hc = 2 * cnt + h, stage = hc % kStages, ch = cnt;
                 if (FORM == kDKDV &&
                     !__all_sync(kAll, wait_phase(sm, sm.st_full[stage], (hc / kStages) & 1,
                                                  kErrTimeoutSoftmax)))
                     return;
-                if (!__all_sync(kAll, wait_phase(sm, sm.s_full[h], cnt & 1, kErrTimeoutSoftmax)))
+                if (!__all_sync(kAll, wait_phase(sm, sm.s_full[h], ch & 1, kErrTimeoutSoftmax)))
                     return;
                 ptx::tc_fence_after();
                 uint32_t sv[kCols], dv[kCols];
@@ -592,7 +677,7 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
                 // packed pairs: this warpgroup's 32 values are columns 16g .. 16g+15
                 // of the half's first 32, which the other group may still be
                 // reading: both groups' loads finish first.
-                if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], cnt & 1, kErrTimeoutSoftmax)))
+                if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], ch & 1, kErrTimeoutSoftmax)))
                     return;
                 if (FORM == kDKDV) ptx::tmem_st16_nowait(t_s + h * kHalf + part * 16, pk_p);
                 ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 16, pk_ds);
@@ -641,6 +726,7 @@ __device__ void compute(const Params &p, Smem<HD> &sm, uint32_t tmem) {
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(ptx::smem_addr(&sm.acc_empty));
+        ++unit_iter;
     }
 }
 
@@ -666,6 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         ptx::mbar_init(ptx::smem_addr(&sm.acc_empty), kCompute);
         ptx::mbar_init(ptx::smem_addr(&sm.drain), 1);
         sm.abort = 0;
+        sm.max_len = 0;
         sm.err_word = p.err_word;
         ptx::fence_mbar_init();
     }
@@ -688,13 +775,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
+    if (p.upw < 0) {
+        // The longest window: one pass over the offsets per CTA.
+        int32_t m = 0;
+        for (int32_t w = threadIdx.x; w < p.n_win; w += kThreads) {
+            int32_t s, e;
+            window_rows(p, w, s, e);
+            m = max(m, e - s);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) atomicMax(&sm.max_len, m);
+        __syncthreads();
+    }
+    const Sched S = make_sched(p, sm.max_len);
     const uint32_t tmem = sm.tmem_base;
     const bool tmem_ok = tmem == 0;   // a 512-column allocation starts at column 0
     if (!tmem_ok && threadIdx.x == 0) atomicOr(p.err_word, kErrTmemAlloc);
     if (tmem_ok) {
-        if (warp < 8) compute<HD, FORM>(p, sm, tmem);
-        else if (warp == kProducerWarp) producer<HD, FORM>(p, sm);
-        else if (lane == 0) mma_issuer<HD, FORM>(p, sm, tmem);
+        if (warp < 8) compute<HD, FORM>(p, S, sm, tmem);
+        else if (warp == kProducerWarp) producer<HD, FORM>(p, S, sm);
+        else if (lane == 0) mma_issuer<HD, FORM>(p, S, sm, tmem);
     }
     __syncwarp();
     ptx::tc_fence_before();
@@ -712,11 +813,24 @@ atlas_status launch_form(Params p, const DeviceInfo &dev, cudaStream_t stream) {
     if (!set_smem_limit(reinterpret_cast<const void *>(attn_bwd_tc_kernel<HD, FORM>),
                         static_cast<int>(smem)))
         return ATLAS_ERR_CUDA;
-    const int64_t per_prob = p.tiles_d + p.tiles_g;
-    const int64_t units = per_prob * p.batch * p.heads;
+    const int64_t per_prob = static_cast<int64_t>(p.tiles_d) + p.tiles_g;
+    int64_t units = per_prob * p.batch * p.heads;
     if (units == 0) return ATLAS_OK;
     if (units > INT32_MAX) return ATLAS_ERR_SHAPE;
-    p.n_units = static_cast<int32_t>(units);
+    // Unit form: tiles of their own for windows of at least 128 rows. Fixed
+    // windows decide here (their slots never exceed three times the packed
+    // count); offsets are read by the kernel only.
+    if (p.N == 0) {
+        p.upw = 0;
+    } else if (p.win_off != nullptr) {
+        p.upw = -1;
+        units = std::max<int64_t>(units, dev.sm_count);
+    } else {
+        p.upw = p.L >= kRows ? (p.L + kRows - 1) / kRows : 0;
+        if (p.upw > 0)
+            units = (static_cast<int64_t>(p.N / p.L) * p.upw + p.tiles_g) * p.batch * p.heads;
+        if (units > INT32_MAX) return ATLAS_ERR_SHAPE;
+    }
     p.n_long = FORM == kDKDV ? p.tiles_g * p.batch * p.heads : 0;
     const int grid = static_cast<int>(std::min<int64_t>(units, dev.sm_count));
     attn_bwd_tc_kernel<HD, FORM><<<grid, kThreads, smem, stream>>>(p);
