@@ -501,6 +501,9 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
         issue_sdp(0, st[0]);
         if (!(ok = next_stage(st[1]))) break;
         issue_sdp(1, st[1]);
+        // The resident rows are read by S and dP only: once the unit's last
+        // S/dP are issued, a commit frees them for the next unit's rows.
+        if (n == 1) ptx::mma_commit(ptx::smem_addr(&sm.x_empty));
         for (int32_t j = 0; j < n && ok; ++j) {
             const bool more = j + 1 < n;
             for (int h = 0; h < 2 && ok; ++h) {
@@ -520,13 +523,13 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
                 if (more) {
                     if (!(ok = next_stage(st[h]))) break;
                     issue_sdp(h, st[h]);
+                    if (h == 1 && j + 2 == n) ptx::mma_commit(ptx::smem_addr(&sm.x_empty));
                 }
             }
             ++p_cnt;
         }
         if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&sm.acc_full));
-        ptx::mma_commit(ptx::smem_addr(&sm.x_empty));
         ++unit_iter;
     }
     // Drain: every MMA issued must finish before tensor memory is freed.
@@ -550,6 +553,37 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
     const uint32_t t_res = t_acc + HD + part * (HD / 2);   // DQ: this group's resident Q or dO
     const float c2 = p.scale_log2;
     uint32_t cnt = 0, unit_iter = 0;
+
+    // DQ: the resident rows of unit V into tensor memory: warpgroup 0 the Q
+    // row, warpgroup 1 the dO row (bf16 pairs, element 2c in the low half of
+    // column c: the A-operand layout of the TS MMAs). Rows past the unit are
+    // zeros. The previous unit's S/dP MMAs must be done (x_empty).
+    auto write_resident = [&](const Unit &V) {
+        const int32_t vrow = V.r0 + static_cast<int32_t>(r);
+        uint32_t rv[HD / 2];
+        if (vrow < V.rend) {
+            const int64_t abs_row = static_cast<int64_t>(V.b) * (V.detail ? p.N : p.G) + vrow;
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                (part == 0 ? p.res_x : p.res_y)[V.detail ? 0 : 1] +
+                (abs_row * p.heads + V.head) * HD);
+#pragma unroll
+            for (int i = 0; i < HD / 8; ++i) {
+                const uint4 w4 = __ldg(src + i);
+                rv[4 * i] = w4.x;
+                rv[4 * i + 1] = w4.y;
+                rv[4 * i + 2] = w4.z;
+                rv[4 * i + 3] = w4.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < HD / 2; ++i) rv[i] = 0u;
+        }
+        if constexpr (HD == 128) ptx::tmem_st64(t_res, rv);
+        else ptx::tmem_st32(t_res, rv);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(ptx::smem_addr(&sm.x_full));
+    };
+    bool resident_ready = false;   // DQ: this unit's rows were written ahead
 
     for (int32_t u = blockIdx.x; u < S.n_units; u += gridDim.x) {
         const Unit U = decode_unit<FORM>(p, S, u);
@@ -597,38 +631,14 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
         } else if (FORM == kDQ) {
             lse2_own = __builtin_huge_valf();
         }
-        if (FORM == kDQ) {
-            // Resident rows into tensor memory: warpgroup 0 the Q row,
-            // warpgroup 1 the dO row (bf16 pairs, element 2c in the low half
-            // of column c: the A-operand layout of the TS MMAs). Rows past
-            // the problem are zeros. The previous unit's MMAs must be done.
+        if (FORM == kDQ && !resident_ready) {
             if (unit_iter > 0 &&
                 !__all_sync(kAll, wait_phase(sm, sm.x_empty, (unit_iter - 1) & 1,
                                              kErrTimeoutSoftmax)))
                 return;
-            uint32_t rv[HD / 2];
-            if (valid) {
-                const int64_t abs_row = static_cast<int64_t>(U.b) * (U.detail ? p.N : p.G) + row;
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    (part == 0 ? p.res_x : p.res_y)[U.detail ? 0 : 1] +
-                    (abs_row * p.heads + U.head) * HD);
-#pragma unroll
-                for (int i = 0; i < HD / 8; ++i) {
-                    const uint4 w4 = __ldg(src + i);
-                    rv[4 * i] = w4.x;
-                    rv[4 * i + 1] = w4.y;
-                    rv[4 * i + 2] = w4.z;
-                    rv[4 * i + 3] = w4.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < HD / 2; ++i) rv[i] = 0u;
-            }
-            if constexpr (HD == 128) ptx::tmem_st64(t_res, rv);
-            else ptx::tmem_st32(t_res, rv);
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(ptx::smem_addr(&sm.x_full));
+            write_resident(U);
         }
+        resident_ready = false;
         const int32_t n = U.n_a + U.n_b;
         for (int32_t j = 0; j < n; ++j, ++cnt) {
             const bool det = streamed_detail(U, j);
@@ -684,6 +694,23 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[h]));
+            }
+        }
+        if (FORM == kDQ) {
+            // The next unit's resident rows go in as soon as this unit's
+            // S/dP are done, so its first S/dP run during this epilogue.
+            int32_t u2 = u + gridDim.x;
+            Unit V;
+            for (; u2 < S.n_units; u2 += gridDim.x) {
+                V = decode_unit<FORM>(p, S, u2);
+                if (V.n_a + V.n_b != 0) break;
+            }
+            if (u2 < S.n_units) {
+                if (!__all_sync(kAll, wait_phase(sm, sm.x_empty, unit_iter & 1,
+                                                 kErrTimeoutSoftmax)))
+                    return;
+                write_resident(V);
+                resident_ready = true;
             }
         }
         // Epilogue: accumulators -> bf16 rows.
