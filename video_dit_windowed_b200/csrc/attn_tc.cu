@@ -458,6 +458,10 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
         issue_s(0, k_slot, nc);
         issue_s(1, k_slot, nc);
         ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
+        // Q is read by the S MMAs only: once the unit's last S is issued, a
+        // commit frees it, and the next unit's Q loads during the last P*V
+        // and this unit's epilogue.
+        if (U.n_tiles == 1) ptx::mma_commit(ptx::smem_addr(&sm.q_empty));
         for (int32_t j = 0; j < U.n_tiles && ok; ++j) {
             const bool more = j + 1 < U.n_tiles;
             const int32_t nc_next = more ? tile_cols(U, j + 1) : 0;
@@ -471,6 +475,7 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
             if (more) {
                 issue_s(1, k_slot, nc_next);
                 ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[k_slot]));
+                if (j + 2 == U.n_tiles) ptx::mma_commit(ptx::smem_addr(&sm.q_empty));
             }
             nc = nc_next;
             ptx::mma_commit(ptx::smem_addr(&sm.kv_empty[v_slot]));
@@ -478,7 +483,6 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
         }
         if (!ok) break;
         for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
-        ptx::mma_commit(ptx::smem_addr(&sm.q_empty));
         ++unit_iter;
     }
     // Drain: every MMA issued must finish before tensor memory is freed.
