@@ -372,3 +372,28 @@ def test_aligned_global_permute_validation(lib):
         assert call(src=FAKE + 8) == atlas.ERR_ALIGN
         assert call(dst=FAKE + 64) == atlas.ERR_ALIAS
         assert call(dt=7) == atlas.ERR_UNSUPPORTED
+
+
+def test_aligned_global_offsets_property(lib):
+    """Many random shapes: the range lengths of the aligned order equal the
+    number of global tokens whose alignment point floor(x*E/(c*e)) falls in
+    each detail cube, counted token by token; the ranges are the prefix sums
+    of those counts in the cube grid's raster order."""
+    import numpy as np
+    rng = np.random.default_rng(2026)
+    for _ in range(300):
+        grid = tuple(int(v) for v in rng.integers(1, 40, size=3))
+        cube = tuple(int(min(g, v)) for g, v in zip(grid, rng.integers(1, 17, size=3)))
+        gg = tuple(int(v) for v in rng.integers(1, 25, size=3))
+        nb = [-(-E // c) for E, c in zip(grid, cube)]
+        counts = np.zeros(nb[0] * nb[1] * nb[2], dtype=np.int64)
+        bt = [x * grid[0] // (cube[0] * gg[0]) for x in range(gg[0])]
+        bh = [x * grid[1] // (cube[1] * gg[1]) for x in range(gg[1])]
+        bw = [x * grid[2] // (cube[2] * gg[2]) for x in range(gg[2])]
+        for a in bt:
+            for b in bh:
+                for c in bw:
+                    counts[(a * nb[1] + b) * nb[2] + c] += 1
+        want = np.concatenate([[0], np.cumsum(counts)])
+        got = atlas.aligned_global_offsets(grid, cube, gg).numpy()
+        assert np.array_equal(got, want), (grid, cube, gg)
