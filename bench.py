@@ -580,7 +580,9 @@ def max_over_ranks(v, world):
     return float(t.item())
 
 
-def config_of(w, world, mask="all", batch=1, backward=False, graph=False):
+def config_of(w, world, mask="all", batch=1, backward=False, graph=False, shard="replicas"):
+    """The line's config. ``w`` is one rank's workload; with head sharding
+    its heads are the rank's share of the problem's."""
     c = {"workload": w.name, "mask": mask, "pass": "forward+backward" if backward else "forward",
          "launch": "cuda graph" if graph else "stream", "detail_grid": list(w.grid), "cube": list(w.cube),
          "global_grid": list(w.global_grid), "n_detail": w.n_detail, "window_len": w.window_len,
@@ -588,6 +590,10 @@ def config_of(w, world, mask="all", batch=1, backward=False, graph=False):
          "rope_split": list(w.split), "detail_scales": list(w.detail_scales),
          "global_scales": list(w.global_scales), "batch_per_gpu": batch,
          "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"}
+    if shard == "heads" and world > 1:
+        c["heads"] = w.heads * world
+        c["heads_per_gpu"] = w.heads
+        c["parallelism"] = f"head-parallel over {world} GPUs (no collective)"
     per_tensor = max(w.n_detail, w.n_global) * w.heads * w.head_dim * w.elem_bytes
     c["l2"] = (f"inputs larger than L2 ({per_tensor / 1e6:.0f} MB per tensor)"
                if per_tensor > 126e6 else "inputs smaller than L2; no flush")
@@ -600,7 +606,7 @@ def run_reference(args, world, rank):
     if args.mask != "all" or args.batch != 1 or args.backward:
         raise SystemExit("the oracle arm times the method's own mask, one problem per step "
                          "(--mask all --batch 1)")
-    w = workload(args)
+    w = workload(args, world)
     times = []
     # each step a bounded sample: the whole --steps/--warmup run stays near a minute
     budget = max(0.5, min(args.cpu_budget, 60.0 / max(1, args.steps + args.warmup)))
@@ -611,8 +617,9 @@ def run_reference(args, world, rank):
     value = statistics.mean(times)
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "impl": "reference", "config": config_of(w, world),
+           "scaling": scaling_of(args), "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": config_of(w, world, shard=args.shard),
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                             "sample": sample + " per step"},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -621,19 +628,31 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
-def workload(args):
+def workload(args, world=1):
+    """One rank's workload: the named one (with --heads, that many heads);
+    with --shard heads, this rank's share of the heads of one problem (heads
+    are independent end to end, so the shards need no collective)."""
+    import dataclasses
     w = WORKLOADS[args.workload]
     if args.heads:
-        import dataclasses
         w = dataclasses.replace(w, heads=args.heads)
+    if getattr(args, "shard", "replicas") == "heads" and world > 1:
+        if w.heads % world:
+            raise SystemExit(f"--shard heads: {w.heads} heads do not split over {world} GPUs")
+        w = dataclasses.replace(w, heads=w.heads // world)
     return w
+
+
+def scaling_of(args):
+    """Weak: every rank adds a problem. Strong: the ranks share one problem."""
+    return "strong" if getattr(args, "shard", "replicas") == "heads" else "weak"
 
 
 def run_atlas(args, world, rank, local):
     from video_dit_windowed_b200 import atlas, build
     if not os.path.exists(atlas.LIB_PATH):
         build.build()
-    w = workload(args)
+    w = workload(args, world)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
@@ -734,9 +753,10 @@ def run_atlas(args, world, rank, local):
     peak_tf = pk["bf16_tflops_sustained"]
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w, world, args.mask, args.batch, args.backward, args.graph),
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": scaling_of(args), "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, world, args.mask, args.batch, args.backward, args.graph,
+                            args.shard),
         "attn_tflops": attn_tf, "attn_ms": attn_ms,
         "attn_frac_of_bf16_peak": {"sustained": attn_tf / pk["bf16_tflops_sustained"],
                                    "burst": attn_tf / pk["bf16_tflops"], "peaks": pk_kind},
@@ -929,10 +949,17 @@ def main():
                     help="time a training step: the forward path plus its backward (gradients "
                          "w.r.t. the raster inputs); value counts the backward as 2.5x the "
                          "forward FLOPs")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with --gpus N: replicas (every rank runs its own problem, weak "
+                         "scaling) or heads (the ranks split one problem's heads, strong "
+                         "scaling)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of its own "
                          "(smaller cases for profiler captures; reported in config)")
     args = ap.parse_args()
+    if args.shard == "heads" and args.proj:
+        raise SystemExit("--proj runs replicas only: with the heads split, the output "
+                         "projection would need a sum over the ranks")
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

@@ -221,3 +221,32 @@ def test_full_size_sampled_rows(name):
             assert float((t.float() - 1).abs().max()) <= 8e-3
     del q_d, k_d, v_d, q_g, k_g, v_g, o_d, o_g
     torch.cuda.empty_cache()
+
+
+def test_head_shards_equal_the_full_call():
+    """Head-parallel sharding: heads are independent end to end, so the
+    reorder+RoPE and the attention of a slice of the heads (as one rank of a
+    head-parallel run holds them) give the full call's bits for those heads."""
+    grid, cube, gg, heads, hd = (6, 16, 16), (3, 8, 8), (6, 4, 4), 4, 128
+    N, G, L = 1536, 96, 192
+    rope = atlas.make_rope(10000.0, (44, 42, 42), (1.0, 1.0, 1.0))
+    x = {s: normal((N if s.endswith("_d") else G, heads, hd), s, torch.bfloat16, seed=41,
+                   device="cuda") for s in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")}
+
+    def run(t, nh):
+        q, k = torch.empty_like(t["q_d"]), torch.empty_like(t["k_d"])
+        atlas.cube_reorder(t["q_d"], q, grid, cube, rope)
+        atlas.cube_reorder(t["k_d"], k, grid, cube, rope)
+        o_d, o_g = torch.empty_like(q), torch.empty_like(t["q_g"])
+        lse = torch.empty(nh, N + G, dtype=torch.float32, device="cuda")
+        atlas.local_global_attn(q, k, t["v_d"], L, t["q_g"], t["k_g"], t["v_g"], o_d, o_g, lse)
+        return q, o_d, o_g, lse
+
+    full = run(x, heads)
+    for h0, h1 in ((0, 2), (2, 4), (1, 2)):
+        part = run({s: v[:, h0:h1].contiguous() for s, v in x.items()}, h1 - h0)
+        torch.cuda.synchronize()
+        check_no_device_error()
+        for a, b in zip(full[:3], part[:3]):
+            assert torch.equal(a[:, h0:h1].contiguous().view(torch.int16), b.view(torch.int16))
+        assert torch.equal(full[3][h0:h1], part[3])

@@ -63,3 +63,42 @@ def test_reference_arm_two_ranks_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_head_shards_cover_the_problem():
+    """--shard heads: each rank's workload holds heads/N heads, the line
+    reports the problem's heads and strong scaling; a head count that does
+    not split is refused."""
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    args = argparse.Namespace(workload="720p", heads=0, shard="heads")
+    for world in (1, 2, 4, 8):
+        w = bench.workload(args, world)
+        assert w.heads * world == 40
+        c = bench.config_of(w, world, shard="heads")
+        assert c["heads"] == 40
+        if world > 1:
+            assert c["heads_per_gpu"] == 40 // world and "head-parallel" in c["parallelism"]
+    assert bench.scaling_of(args) == "strong"
+    assert bench.scaling_of(argparse.Namespace(shard="replicas")) == "weak"
+    with pytest.raises(SystemExit):
+        bench.workload(args, 3)
+    # FLOPs: the shards' FLOPs add up to the problem's
+    full = bench.workload(argparse.Namespace(workload="720p", heads=0, shard="replicas"), 4)
+    assert 4 * bench.workload(args, 4).unmasked_flops() == full.unmasked_flops()
+
+
+def test_reference_arm_head_shards_two_ranks():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+           "--workload", "tiny", "--cpu-budget", "1", "--shard", "heads"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["scaling"] == "strong" and lines[0]["config"]["heads"] == 2
+    assert lines[0]["config"]["heads_per_gpu"] == 1
