@@ -273,3 +273,25 @@ def test_backward_full_size_sampled():
         assert_grads_close([g_q, g_k, g_v], [dq, dk, dv], "bf16", f"720p head {head}")
     del got, t
     torch.cuda.empty_cache()
+
+
+# Window offsets for both unit forms of the backward (as the forward's
+# parity cases): unequal long windows with empty slots and a one-row window,
+# and one long window among many short ones (packed tiles).
+BWD_OFFSETS = [
+    [0, 700, 1212, 1213, 1313, 2081, 2336, 2592],
+    [0, 1000] + list(range(1001, 1501)),
+]
+
+
+@pytest.mark.parametrize("offsets", BWD_OFFSETS)
+def test_backward_window_forms(offsets):
+    N, G, heads, hd = offsets[-1], 150, 2, 128
+    off = torch.tensor(offsets, dtype=torch.int32)
+    t = inputs(1, N, G, heads, hd, "bf16", seed=25)
+    got = run_gpu(t, 1, heads, N, G, window_offsets=off.to(DEV))
+    ref = orc().attention_bwd_full(f64(t["q_d"]), f64(t["k_d"]), f64(t["v_d"]), 1,
+                                   f64(t["q_g"]), f64(t["k_g"]), f64(t["v_g"]), f64(t["do_d"]),
+                                   f64(t["do_g"]), hd ** -0.5, n_threads(),
+                                   win_off=np.asarray(offsets, dtype=np.int64))
+    assert_grads_close([f64(g) for g in got], ref, "bf16", f"offsets {offsets[:4]}")
