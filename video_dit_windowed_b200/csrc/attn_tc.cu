@@ -439,11 +439,16 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
         const uint32_t v_lo = v_lo0 + v_slot * kTile16;
         const uint32_t d_o = tmem + 2 * kBN + i * HD, a_p = tmem + i * kBN;
         ptx::mma_ts(d_o, a_p, ptx::desc_join(v_lo, kHi), kIdescPV, first ? 0u : 1u);
+        if (nc == kBN) {
 #pragma unroll
-        for (int ks = 1; ks < kBN / 16; ++ks) {
-            if (ks * 16 >= nc) break;
-            ptx::mma_ts(d_o, a_p + ks * 8, ptx::desc_join(v_lo + ((ks * 16 * 128) >> 4), kHi),
-                        kIdescPV, 1u);
+            for (int ks = 1; ks < kBN / 16; ++ks)
+                ptx::mma_ts(d_o, a_p + ks * 8,
+                            ptx::desc_join(v_lo + ((ks * 16 * 128) >> 4), kHi), kIdescPV, 1u);
+        } else {
+#pragma unroll 1
+            for (int ks = 1; ks * 16 < nc; ++ks)
+                ptx::mma_ts(d_o, a_p + ks * 8,
+                            ptx::desc_join(v_lo + ((ks * 16 * 128) >> 4), kHi), kIdescPV, 1u);
         }
         return true;
     };
