@@ -763,7 +763,7 @@ def run_atlas(args, world, rank, local):
         "reorder_rope_gbs": rr_gbs, "reorder_rope_ms": rr_ms,
         "reorder_rope_frac_of_hbm": (rr_gbs / pk["hbm_gbs"]) if rr_gbs else None,
         "unorder_gbs": un_bytes / (un_ms * 1e-3) / 1e9 if un_ms > 0 and un_bytes else None,
-        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>", "achieved": attn_tf,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128, false>", "achieved": attn_tf,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
                      "peak_kind": f"{pk_kind} bf16 sustained",
                      "traffic": traffic,

@@ -501,7 +501,11 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
 // ---------------------------------------------------------------------------
 // Softmax + epilogue of Q tile `qt`; 128 threads, thread = row = TMEM lane.
 // ---------------------------------------------------------------------------
-template <int HD>
+// NARROW: the softmax has 64- and 32-column forms for narrow tiles (their
+// exponentials skipped); without it a narrow tile's softmax takes all 128
+// columns (the masked ones give P = 0) and only its MMAs are narrow. The
+// extra forms cost about 1 % on layouts whose narrow tiles are rare.
+template <int HD, bool NARROW>
 __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t tmem,
                                  int qt) {
     const uint32_t warp = (threadIdx.x / 32) & 3;
@@ -667,10 +671,15 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
                 }
                 return sum;
             };
-            const int32_t nc = tile_cols(U, j);
-            const float sum = nc == kBN ? tile(std::integral_constant<int, kBN>{})
-                              : nc == 64 ? tile(std::integral_constant<int, 64>{})
-                                         : tile(std::integral_constant<int, 32>{});
+            float sum;
+            if constexpr (NARROW) {
+                const int32_t nc = tile_cols(U, j);
+                sum = nc == kBN ? tile(std::integral_constant<int, kBN>{})
+                      : nc == 64 ? tile(std::integral_constant<int, 64>{})
+                                 : tile(std::integral_constant<int, 32>{});
+            } else {
+                sum = tile(std::integral_constant<int, kBN>{});
+            }
             l_run += sum;
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
@@ -713,7 +722,7 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
     }
 }
 
-template <int HD>
+template <int HD, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem<HD> &sm = *reinterpret_cast<Smem<HD> *>(
@@ -775,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     if (warp < 8) {
         ptx::setmaxnreg_inc<kRegsSoftmax>();
-        if (tmem_ok) softmax_epilogue<HD>(p, S, sm, tmem, warp / 4);
+        if (tmem_ok) softmax_epilogue<HD, NARROW>(p, S, sm, tmem, warp / 4);
     } else {
         ptx::setmaxnreg_dec<kRegsOther>();
         if (tmem_ok && lane == 0) {
@@ -844,12 +853,18 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
             n_units = (static_cast<int64_t>(p.N / p.L) * p.upw + p.n_gunits) * a.batch * a.heads;
         if (n_units > INT32_MAX) return ATLAS_ERR_SHAPE;
     }
+    // Narrow softmax forms where narrow tiles are frequent: per-window global
+    // ranges (aligned proxy tokens) or variable windows (partial cubes).
+    const bool narrow = a.win_off != nullptr || a.gwin_off != nullptr;
+    const void *fn = narrow ? reinterpret_cast<const void *>(attn_tc_kernel<HD, true>)
+                            : reinterpret_cast<const void *>(attn_tc_kernel<HD, false>);
     const size_t smem = sizeof(Smem<HD>) + 1024;
-    if (!set_smem_limit(reinterpret_cast<const void *>(attn_tc_kernel<HD>),
-                        static_cast<int>(smem)))
-        return ATLAS_ERR_CUDA;
+    if (!set_smem_limit(fn, static_cast<int>(smem))) return ATLAS_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(n_units, dev.sm_count));
-    attn_tc_kernel<HD><<<grid, kThreads, smem, stream>>>(p);
+    if (narrow)
+        attn_tc_kernel<HD, true><<<grid, kThreads, smem, stream>>>(p);
+    else
+        attn_tc_kernel<HD, false><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
 
