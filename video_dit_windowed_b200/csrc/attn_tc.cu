@@ -44,7 +44,7 @@
 // covers O_i += P_i(j) V(j). Each softmax therefore has the time of the other
 // tile's two MMAs to produce its P. A key tile whose keys end within its first
 // 32 or 64 columns for every row of the unit gets S and P*V MMAs of that width
-// only. The Q tiles are released right after the unit's last S MMA, so the
+// only (and, in the NARROW form of the kernel, a softmax of that width). The Q tiles are released right after the unit's last S MMA, so the
 // next unit's Q loads during the last P*V and the epilogue.
 // Every wait is bounded: on expiry a bit is set in the device error word,
 // the CTA drains its in-flight copies and MMAs, frees TMEM and returns.
