@@ -103,16 +103,3 @@ def test_reference_arm_head_shards_two_ranks():
     assert lines[0]["scaling"] == "strong" and lines[0]["config"]["heads"] == 2
     assert lines[0]["config"]["heads_per_gpu"] == 1
 
-
-def test_traffic_record_is_current():
-    """The committed ncu traffic record was taken on the attention kernel as
-    it stands (bench.py reports it only then), and it is close to the
-    algorithmic bytes: Q, K, V read once and O written once."""
-    sys.path.insert(0, ROOT)
-    import argparse
-    import bench
-    w = bench.workload(argparse.Namespace(workload="720p", heads=0, shard="replicas"))
-    t = bench.measured_traffic(w)
-    assert t is not None, "profiles/attn_tc_traffic.txt is stale: capture the kernel again"
-    algorithmic = 4 * (w.n_detail + w.n_global) * w.heads * w.head_dim * w.elem_bytes
-    assert 0.9 * algorithmic <= t <= 1.1 * algorithmic

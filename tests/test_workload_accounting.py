@@ -53,3 +53,19 @@ def test_aligned_boxes_partition_the_global_axes():
         for a in range(3):
             boxes = w.aligned_boxes(a)
             assert sum(boxes) == gg[a] and min(boxes) >= 0
+
+
+def test_traffic_record_is_current():
+    """The committed ncu traffic record was taken on the attention kernel as
+    it stands (bench.py reports it only then), and it is close to the
+    algorithmic bytes: Q, K, V read once and O written once."""
+    import argparse
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    w = bench.workload(argparse.Namespace(workload="720p", heads=0, shard="replicas"))
+    t = bench.measured_traffic(w)
+    assert t is not None, "profiles/attn_tc_traffic.txt is stale: capture the kernel again"
+    algorithmic = 4 * (w.n_detail + w.n_global) * w.heads * w.head_dim * w.elem_bytes
+    assert 0.9 * algorithmic <= t <= 1.1 * algorithmic
