@@ -1,5 +1,6 @@
 """The work counts behind every bench figure, checked on CPU against the
-oracle's own mask: allowed (query, key) pairs per mask and problem.
+oracle's own mask: allowed (query, key) pairs per mask and problem; and the
+committed DRAM-traffic record the roofline line reports.
 
 With Q = K = 0 every allowed logit is 0, so the oracle's log-sum-exp of a
 row is log(number of keys that row may see); summing exp(lse) over all rows
