@@ -44,9 +44,10 @@
 // takes resident row r and columns 32g .. 32g+31 of each half (and, in the
 // epilogue, half of the accumulator columns). Tensor memory:
 // S_0 | S_1 | dP_0 | dP_1 (64 columns each) | acc (DQ: dQ, then the
-// resident Q and dO; DKDV: dV, dK). The packed P and dS overwrite the first
-// half of S_h and dP_h, which the other warpgroup may still be reading: the
-// two groups meet on an mbarrier between their loads and their stores.
+// resident Q and dO; DKDV: dV, dK). Each warpgroup writes its packed P and
+// dS over columns of S_h and dP_h that only it reads (group 0: columns 0-15,
+// group 1: columns 48-63), so the two groups never wait for each other; the
+// accumulating MMAs take their A operand from those two column ranges.
 // Every wait is bounded, as in the forward kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -86,7 +87,6 @@ struct Smem {
     uint64_t x_full, x_empty;
     uint64_t st_full[kStages], st_empty[kStages];
     uint64_t s_full[2], p_full[2];
-    uint64_t ld_done[2];          // DKDV: both warpgroups have read S_h and dP_h
     uint64_t acc_full, acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
@@ -474,11 +474,14 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
     };
     // acc += A (tensor memory, 64 streamed rows packed in 32 columns) times
     // the half tile in stage s as an MN-major B operand.
+    // The packed rows sit in columns 0-15 (keys 0-31, compute group 0) and
+    // 48-63 (keys 32-63, group 1) of the half's 64.
     auto issue_acc = [&](uint32_t d, uint32_t a, uint32_t b_lo, uint32_t s, bool first) {
 #pragma unroll
         for (int ks = 0; ks < kHalf / 16; ++ks) {
             const uint32_t off = s * kH16 + ((ks * 16 * 128) >> 4);
-            ptx::mma_ts(d, a + ks * 8, ptx::desc_join(b_lo + off, kHi), kIdAcc,
+            const uint32_t col = ks < 2 ? ks * 8 : 32 + ks * 8;
+            ptx::mma_ts(d, a + col, ptx::desc_join(b_lo + off, kHi), kIdAcc,
                         (first && ks == 0) ? 0u : 1u);
         }
     };
@@ -658,7 +661,6 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
                 uint32_t sv[kCols], dv[kCols];
                 ptx::tmem_ld32(t_s + h * kHalf + part * kCols, sv);
                 ptx::tmem_ld32(t_dp + h * kHalf + part * kCols, dv);
-                ptx::mbar_arrive(ptx::smem_addr(&sm.ld_done[h]));
                 const int32_t c0 = base + h * kHalf + part * kCols;   // row of column 0
                 const bool partial = c0 < lo || c0 + kCols > hi;
                 uint32_t pk_p[kCols / 2], pk_ds[kCols / 2];
@@ -684,13 +686,11 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
                     pk_p[e] = ptx::pack_bf16x2(pv[0], pv[1]);
                     pk_ds[e] = ptx::pack_bf16x2(dsv[0], dsv[1]);
                 }
-                // packed pairs: this warpgroup's 32 values are columns 16g .. 16g+15
-                // of the half's first 32, which the other group may still be
-                // reading: both groups' loads finish first.
-                if (!__all_sync(kAll, wait_phase(sm, sm.ld_done[h], ch & 1, kErrTimeoutSoftmax)))
-                    return;
-                if (FORM == kDKDV) ptx::tmem_st16_nowait(t_s + h * kHalf + part * 16, pk_p);
-                ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 16, pk_ds);
+                // Packed pairs go into this warpgroup's own columns (the first
+                // 16 of group 0's 32, the last 16 of group 1's), which the
+                // other group never reads: no meeting between the groups.
+                if (FORM == kDKDV) ptx::tmem_st16_nowait(t_s + h * kHalf + part * 48, pk_p);
+                ptx::tmem_st16_nowait(t_dp + h * kHalf + part * 48, pk_ds);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[h]));
@@ -773,7 +773,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         for (int h = 0; h < 2; ++h) {
             ptx::mbar_init(ptx::smem_addr(&sm.s_full[h]), 1);
             ptx::mbar_init(ptx::smem_addr(&sm.p_full[h]), kCompute);
-            ptx::mbar_init(ptx::smem_addr(&sm.ld_done[h]), kCompute);
         }
         ptx::mbar_init(ptx::smem_addr(&sm.acc_full), 1);
         ptx::mbar_init(ptx::smem_addr(&sm.acc_empty), kCompute);
