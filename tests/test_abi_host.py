@@ -397,3 +397,19 @@ def test_aligned_global_offsets_property(lib):
         want = np.concatenate([[0], np.cumsum(counts)])
         got = atlas.aligned_global_offsets(grid, cube, gg).numpy()
         assert np.array_equal(got, want), (grid, cube, gg)
+
+
+def test_plain_c_program_against_the_header(lib, tmp_path):
+    """The boundary from C: tests/c_abi/host_calls.c, compiled with gcc
+    against include/atlas.h and linked to libatlas.so, runs its host-only
+    checks (window offsets of the cube and aligned orders against counts from
+    the definitions, status names, an argument error) and prints ok."""
+    src = os.path.join(ROOT, "tests", "c_abi", "host_calls.c")
+    exe = str(tmp_path / "host_calls")
+    libdir = os.path.dirname(atlas.LIB_PATH)
+    cmd = ["gcc", "-std=c11", "-Wall", "-Werror", "-O1", src, "-I", os.path.join(ROOT, "include"),
+           "-L", libdir, "-l:libatlas.so", f"-Wl,-rpath,{libdir}", "-o", exe]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
