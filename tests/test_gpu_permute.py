@@ -172,3 +172,30 @@ def test_full_size_reorder_rope(name):
     assert_rope_close(got, exact, xs, w.dtype)
     del x, y
     torch.cuda.empty_cache()
+
+
+def test_plain_c_program_on_the_gpu(tmp_path):
+    """The boundary from C on the GPU: tests/c_abi/gpu_chain.c allocates with
+    the CUDA runtime, reorders arbitrary bytes through libatlas.so, and
+    compares them bit for bit with the oracle's permutation (linked only in
+    this test), then checks that the unorder restores the input."""
+    import os
+    import subprocess
+    import oracle
+    from video_dit_windowed_b200 import atlas as _atlas
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = os.path.join(root, "tests", "c_abi", "gpu_chain.c")
+    exe = str(tmp_path / "gpu_chain")
+    libdir = os.path.dirname(_atlas.LIB_PATH)
+    odir = os.path.dirname(oracle.LIB_PATH)
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    cmd = ["gcc", "-std=c11", "-Wall", "-Werror", "-O1", src,
+           "-I", os.path.join(root, "include"), "-I", os.path.join(cuda, "include"),
+           "-L", libdir, "-l:libatlas.so", f"-Wl,-rpath,{libdir}",
+           "-L", odir, "-l:liboracle_atlas.so", f"-Wl,-rpath,{odir}",
+           "-L", os.path.join(cuda, "lib64"), "-lcudart", f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}",
+           "-o", exe]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
