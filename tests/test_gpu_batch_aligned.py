@@ -459,3 +459,22 @@ def test_aligned_order_random_shapes():
         assert y.cpu().view(torch.uint8).numpy().reshape(B, G, -1).tobytes() == want.tobytes(), \
             (grid, cube, gg)
         assert torch.equal(z.view(torch.uint8), x.view(torch.uint8))
+
+
+def test_aligned_unorder_with_rope_is_rope_after_unorder():
+    """The unorder with a rotation (used with the transposed RoPE to bring
+    global dQ/dK back to raster order) rotates each token at its global raster
+    position: the same bits as the plain unorder followed by the rotation."""
+    grid, cube, gg = (6, 20, 30), (3, 8, 8), (4, 6, 7)
+    G = gg[0] * gg[1] * gg[2]
+    for dtype in ("bf16", "fp32"):
+        x = mk(2 * G, 3, 128, "q_g", dtype, seed=17)
+        rg = atlas.make_rope(10000.0, split_for(128), tuple(a / b for a, b in zip(grid, gg)))
+        rt = atlas.transpose_rope(rg)
+        a, b, c = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+        atlas.aligned_global_unorder(x, a, grid, cube, gg, rt, batch=2)
+        atlas.aligned_global_unorder(x, b, grid, cube, gg, batch=2)
+        atlas.rope3d_batched(b, c, 2, gg, rt)
+        torch.cuda.synchronize()
+        check_no_device_error()
+        assert torch.equal(a.view(torch.uint8), c.view(torch.uint8)), dtype
