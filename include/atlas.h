@@ -185,15 +185,19 @@ atlas_status atlas_local_global_attn(
  *     pairs (256 KB), held by every GPU that loads the library until the
  *     process exits. A RoPE needs T*(d_t/2) + H*(d_h/2) + W*(d_w/2) pairs;
  *     more than 32768 returns ATLAS_ERR_CAPACITY and launches nothing.
- *   - Each call builds the table on the host and copies it into the array
+ *   - A call whose grid extents or RoPE differ from those the device's
+ *     array was last filled with builds the table on the host, in a host
+ *     staging buffer that every call reuses, and copies it into the array
  *     on `stream` (from pageable memory: the call returns once the copy has
- *     been staged), then launches the kernel on `stream`.
+ *     been staged). A call with the same extents and RoPE as the last fill
+ *     skips both and reads the array as it stands. Then the kernel is
+ *     launched on `stream`.
  *   - Every call on a device shares the array and overwrites it: calls whose
  *     work overlaps on the GPU (for example on two streams) race; issue
  *     them on one stream or otherwise order them.
  *   - The first call on each device resolves the array's device address
  *     (cudaGetSymbolAddress, with that device current) and reads the device
- *     properties; make that first call before any stream capture.
+ *     properties.
  *   - No cudaMalloc, cudaFree or other allocating routine is called.
  * Without rope the call is a pure permutation and touches no table.
  */
@@ -501,6 +505,12 @@ atlas_status atlas_debug_stall_next_attention(void);
 
 /* Free the cached RoPE tables of every device (synchronises the device). */
 atlas_status atlas_release_caches(void);
+
+/* Number of RoPE cos/sin tables the library holds, over all devices, in
+ * device memory it allocated itself (the cache of atlas_cube_reorder and the
+ * other rotating calls; emptied by atlas_release_caches). The fixed array
+ * of atlas_cube_reorder_noalloc is not counted. Host only; never fails. */
+int64_t atlas_cached_rope_tables(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t atlas_version(void);

@@ -13,11 +13,15 @@ This file is collected last on purpose (it is named so): if it fails, a run
 that stops at the first failure has already run every other test.
 """
 import ctypes
+import os
+import subprocess
+import sys
+import textwrap
 
 import pytest
 import torch
 
-from helpers import assert_rope_close, check_no_device_error, f64
+from helpers import assert_rope_close, check_no_device_error, f64, orc
 from video_dit_windowed_b200 import atlas
 from video_dit_windowed_b200.workloads import normal
 
@@ -49,13 +53,23 @@ def _compare(call, seed):
     # existing entry point's output (same table, same kernel: equal in fact)
     assert_rope_close(f64(got), f64(ref), f64(ref), dtype)
     assert torch.equal(got.view(torch.uint8), ref.view(torch.uint8))
+    # and against the fp64 oracle's RoPE then reorder, on the first and last
+    # head (the rotation is the same for every head)
+    heads = [0, call["heads"] - 1]
+    xs = f64(x[:, heads])
+    exact = orc().cube_reorder(orc().rope3d_grid(xs, call["grid"], 10000.0, call["split"],
+                                                 call["scales"]), call["grid"], call["cube"])
+    assert_rope_close(f64(got[:, heads]), exact, orc().cube_reorder(xs, call["grid"],
+                                                                    call["cube"]), dtype)
 
 
 def test_noalloc_matches_reorder_twice():
     for i, call in enumerate(CALLS):
         _compare(call, seed=i)
     # and the first configuration once more, after the second overwrote it
+    # (refilled), then again with the same grid and RoPE (the fill skipped)
     _compare(CALLS[0], seed=7)
+    _compare(CALLS[0], seed=8)
 
 
 def test_noalloc_pure_permutation():
@@ -80,3 +94,32 @@ def test_noalloc_rejects_tables_beyond_capacity():
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == atlas.ERR_CAPACITY
     assert "CAPACITY" in atlas.status_string(st)
+
+
+def test_noalloc_first_call_leaves_the_allocating_cache_empty():
+    """In a fresh process, the no-alloc entry point (with RoPE, two grids)
+    is the library's first call: afterwards the library holds no table in
+    memory it allocated. The allocating entry point then adds one, so the
+    count does see allocations."""
+    script = textwrap.dedent("""
+        import torch
+        from video_dit_windowed_b200 import atlas
+        x = torch.randn(8 * 16 * 16, 2, 128, device="cuda").to(torch.bfloat16)
+        y = torch.empty_like(x)
+        rope = atlas.make_rope(10000.0, (44, 42, 42), (1.0, 1.0, 1.0))
+        atlas.cube_reorder_noalloc(x, y, (8, 16, 16), (2, 8, 8), rope)
+        atlas.cube_reorder_noalloc(x, y, (4, 32, 16), (2, 8, 8), rope)
+        torch.cuda.synchronize()
+        assert atlas.last_device_error() == 0
+        assert atlas.cached_rope_tables() == 0, atlas.cached_rope_tables()
+        atlas.cube_reorder(x, y, (8, 16, 16), (2, 8, 8), rope)
+        torch.cuda.synchronize()
+        assert atlas.cached_rope_tables() == 1, atlas.cached_rope_tables()
+        print("fresh process ok")
+    """)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root + os.pathsep + os.environ.get("PYTHONPATH", ""))
+    res = subprocess.run([sys.executable, "-c", script], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stdout + res.stderr
+    assert "fresh process ok" in res.stdout

@@ -131,6 +131,8 @@ def _declare(lib):
     lib.atlas_debug_stall_next_attention.argtypes = []
     lib.atlas_release_caches.restype = ctypes.c_int
     lib.atlas_release_caches.argtypes = []
+    lib.atlas_cached_rope_tables.restype = ctypes.c_int64
+    lib.atlas_cached_rope_tables.argtypes = []
     lib.atlas_version.restype = ctypes.c_int32
     lib.atlas_version.argtypes = []
     return lib
@@ -485,6 +487,11 @@ def debug_stall_next_attention():
     """Test hook: the next bf16 attention launch leaves one K tile unloaded,
     so its bounded waits expire and it reports ATLAS_ERR_TIMEOUT."""
     _check(lib().atlas_debug_stall_next_attention(), "atlas_debug_stall_next_attention")
+
+
+def cached_rope_tables() -> int:
+    """RoPE tables the library holds in device memory it allocated."""
+    return int(lib().atlas_cached_rope_tables())
 
 
 def release_caches():

@@ -668,6 +668,8 @@ ATLAS_API atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *
 
 ATLAS_API atlas_status atlas_release_caches(void) { return release_rope_tables(); }
 
+ATLAS_API int64_t atlas_cached_rope_tables(void) { return cached_rope_tables(); }
+
 ATLAS_API atlas_status atlas_debug_stall_next_attention(void) {
     g_stall_request.store(1);
     return ATLAS_OK;

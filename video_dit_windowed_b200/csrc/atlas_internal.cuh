@@ -81,6 +81,7 @@ struct PermuteArgs {
 };
 atlas_status launch_permute_rope(const PermuteArgs &a, cudaStream_t stream);
 atlas_status release_rope_tables();
+int64_t cached_rope_tables();
 // The cached cos/sin table of `rope` on a T x H x W grid, current device
 // (layout: axis t [t][k], then h, then w; fp64 angles rounded to fp32).
 atlas_status rope_table_for(int64_t T, int64_t H, int64_t W, const atlas_rope &rope,

@@ -326,9 +326,24 @@ atlas_status dispatch(const Params &p, bool rope, int mode, bool general, const 
 constexpr size_t kStaticRopeEntries = 32768;  // 256 KB of (cos, sin) per device
 static __device__ __align__(256) float2 g_static_rope_table[kStaticRopeEntries];
 
-std::mutex g_static_mutex;                      // guards the two arrays below
+std::mutex g_static_mutex;                      // guards the arrays below
 float2 g_static_host_table[kStaticRopeEntries];  // host staging, reused per call
 float2 *g_static_table_dev[64] = {nullptr};      // device address, per device
+
+// What the array of each device was last filled with (grid extents and
+// RoPE): a call with the same ones skips the host fill and the copy.
+struct StaticTableKey {
+    bool valid = false;
+    int64_t T = 0, H = 0, W = 0;
+    atlas_rope rope{};
+    bool same(int64_t t, int64_t h, int64_t w, const atlas_rope &r) const {
+        return valid && T == t && H == h && W == w && rope.theta == r.theta &&
+               rope.d_t == r.d_t && rope.d_h == r.d_h && rope.d_w == r.d_w &&
+               rope.scale_t == r.scale_t && rope.scale_h == r.scale_h &&
+               rope.scale_w == r.scale_w;
+    }
+};
+StaticTableKey g_static_key[64];
 
 // Device address of the static table on `device` (the current device). The
 // array's name is only a host-side stand-in; its address is resolved once per
@@ -419,6 +434,11 @@ atlas_status rope_table_for(int64_t T, int64_t H, int64_t W, const atlas_rope &r
     return st;
 }
 
+int64_t cached_rope_tables() {
+    std::lock_guard<std::mutex> lock(g_tab_mutex);
+    return static_cast<int64_t>(g_tables.size());
+}
+
 atlas_status release_rope_tables() {
     std::lock_guard<std::mutex> lock(g_tab_mutex);
     atlas_status st = ATLAS_OK;
@@ -451,13 +471,22 @@ atlas_status launch_permute_rope_noalloc(const PermuteArgs &a, cudaStream_t stre
     float2 *tab = nullptr;
     atlas_status st = static_table_address(dev.device, &tab);
     if (st != ATLAS_OK) return st;
-    fill_rope_table(g_static_host_table, a.T, a.H, a.W, r);
-    // From pageable host memory: returns once the staging copy is taken, so
-    // the host buffer may be refilled by the next call; ordered on `stream`
-    // before the kernel.
-    if (n > 0 && cudaMemcpyAsync(tab, g_static_host_table, n * sizeof(float2),
-                                 cudaMemcpyHostToDevice, stream) != cudaSuccess)
-        return ATLAS_ERR_CUDA;
+    StaticTableKey &key = g_static_key[dev.device];
+    if (!key.same(a.T, a.H, a.W, r)) {
+        key.valid = false;
+        fill_rope_table(g_static_host_table, a.T, a.H, a.W, r);
+        // From pageable host memory: returns once the staging copy is taken,
+        // so the host buffer may be refilled by the next call; ordered on
+        // `stream` before the kernel.
+        if (n > 0 && cudaMemcpyAsync(tab, g_static_host_table, n * sizeof(float2),
+                                     cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return ATLAS_ERR_CUDA;
+        key.valid = true;
+        key.T = a.T;
+        key.H = a.H;
+        key.W = a.W;
+        key.rope = r;
+    }
     p.tab = tab;
     p.half[0] = static_cast<uint32_t>(r.d_t / 2);
     p.half[1] = static_cast<uint32_t>(r.d_h / 2);
