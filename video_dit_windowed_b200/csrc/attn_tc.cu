@@ -145,6 +145,7 @@ struct Params {
     int32_t batch, n_gtiles;
     int32_t upw;          // window units per window; 0: packed units; -1: from the offsets
     int32_t stall_unit;   // test hook: this unit's first K tile is never loaded (-1: off)
+    int32_t o_v8;         // both outputs 32-byte aligned: the epilogue stores 32 B at a time
     const int32_t *win_off;   // window offsets [n_win + 1] of one problem (NULL: L rows)
     const int32_t *gwin_off;  // global key offsets [n_win + 1] per window (NULL: all keys)
     int32_t n_win;
@@ -275,6 +276,22 @@ __device__ __forceinline__ Unit decode_unit(const Params &p, const Sched &S, int
     }
     U.n_tiles = U.n_wtiles + n_gtiles;
     return U;
+}
+
+// Window units with offsets: bring the offsets decode_unit(u) reads into L1,
+// so that decoding the next unit after an epilogue costs no trip to L2.
+__device__ __forceinline__ void prefetch_unit(const Params &p, const Sched &S, int32_t u) {
+    if (u >= S.n_units || S.upw <= 0 || p.win_off == nullptr) return;
+    int32_t lu = u - (u / S.units_per_head) * S.units_per_head;
+    lu -= (lu / S.units_per_prob) * S.units_per_prob;
+    if (lu >= S.n_dunits) return;
+    const int32_t w = lu / S.upw;
+    ptx::prefetch_l1(p.win_off + w);
+    ptx::prefetch_l1(p.win_off + w + 1);
+    if (p.gwin_off != nullptr) {
+        ptx::prefetch_l1(p.gwin_off + w);
+        ptx::prefetch_l1(p.gwin_off + w + 1);
+    }
 }
 
 // Bounded wait. Returns false (after flagging `err`) if the phase did not
@@ -490,6 +507,7 @@ __device__ void mma_issuer(const Params &p, const Sched &S, Smem<HD> &sm, uint32
             ++p_cnt;
         }
         if (!ok) break;
+        prefetch_unit(p, S, u + gridDim.x);
         for (int i = 0; i < kQTiles; ++i) ptx::mma_commit(ptx::smem_addr(&sm.o_final[i]));
         ++unit_iter;
     }
@@ -685,6 +703,7 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
             ptx::mbar_arrive(ptx::smem_addr(&sm.p_full[qt]));
         }
         // Epilogue: O / l -> bf16 rows; LSE.
+        if (r == 0) prefetch_unit(p, S, u + gridDim.x);
         if (!__all_sync(0xffffffffu, wait_phase(sm, sm.o_final[qt], unit_iter & 1, err)))
             return;
         ptx::tc_fence_after();
@@ -696,7 +715,18 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
         for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
             ptx::tmem_ld32(t_o + c * 32, o);
-            if (row_valid) {
+            if (row_valid && p.o_v8) {
+                // two 32-byte stores per 32 columns: whole sectors
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                    uint32_t w8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        w8[e] = ptx::pack_bf16x2(__uint_as_float(o[16 * v + 2 * e]) * inv_l,
+                                                 __uint_as_float(o[16 * v + 2 * e + 1]) * inv_l);
+                    ptx::st_global_v8(reinterpret_cast<uint8_t *>(dst) + c * 64 + v * 32, w8);
+                }
+            } else if (row_valid) {
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     uint4 w;
@@ -835,6 +865,7 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     p.batch = static_cast<int32_t>(a.batch);
     p.n_gtiles = static_cast<int32_t>((a.n_global + kBN - 1) / kBN);
     p.stall_unit = take_stall_request() ? 0 : -1;
+    p.o_v8 = ((reinterpret_cast<uintptr_t>(a.o_d) | reinterpret_cast<uintptr_t>(a.o_g)) & 31) == 0;
     p.win_off = a.win_off;
     p.gwin_off = a.gwin_off;
     p.n_win = static_cast<int32_t>(a.win_off ? a.n_win : a.n_gwin);

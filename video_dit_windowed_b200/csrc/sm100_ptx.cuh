@@ -251,6 +251,21 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- global memory -------------------------------------------------------------
+// 32-byte store (the address must be 32-byte aligned): one instruction fills
+// a whole 32-byte sector.
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&r)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(dst), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]),
+                    "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+// Bring the line holding `p` into L1 (no register result, no wait).
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" :: "l"(p));
+}
+
 // ---- math --------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {
     float y;
