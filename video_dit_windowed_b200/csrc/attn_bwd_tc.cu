@@ -109,6 +109,7 @@ struct Params {
     int32_t tiles_d, tiles_g;           // 128-row tiles of one problem's detail / global rows
     int32_t n_long;                     // DKDV: units over global keys (scheduled first)
     int32_t upw;   // detail tiles per window; 0: packed tiles; -1: from the offsets
+    int32_t o_v8;  // every output 32-byte aligned: the epilogue stores 32 B at a time
 };
 
 // The unit form and counts, the same in every thread of every CTA.
@@ -734,7 +735,18 @@ __device__ void compute(const Params &p, const Sched &S, Smem<HD> &sm, uint32_t 
             for (int c = 0; c < ncol / 32; ++c) {
                 uint32_t o[32];
                 ptx::tmem_ld32(t_acc + a * HD + col0 + c * 32, o);
-                if (valid) {
+                if (valid && p.o_v8) {
+                    // two 32-byte stores per 32 columns: whole sectors
+#pragma unroll
+                    for (int v = 0; v < 2; ++v) {
+                        uint32_t w8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            w8[e] = ptx::pack_bf16x2(__uint_as_float(o[16 * v + 2 * e]) * f,
+                                                     __uint_as_float(o[16 * v + 2 * e + 1]) * f);
+                        ptx::st_global_v8(reinterpret_cast<uint8_t *>(dst) + c * 64 + v * 32, w8);
+                    }
+                } else if (valid) {
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 w;
@@ -858,6 +870,11 @@ atlas_status launch_form(Params p, const DeviceInfo &dev, cudaStream_t stream) {
         if (units > INT32_MAX) return ATLAS_ERR_SHAPE;
     }
     p.n_long = FORM == kDKDV ? p.tiles_g * p.batch * p.heads : 0;
+    uintptr_t ptr_bits = 0;
+    for (int i = 0; i < 2; ++i)
+        ptr_bits |= reinterpret_cast<uintptr_t>(p.out0[i]) |
+                    (FORM == kDKDV ? reinterpret_cast<uintptr_t>(p.out1[i]) : 0);
+    p.o_v8 = (ptr_bits & 31) == 0;
     const int grid = static_cast<int>(std::min<int64_t>(units, dev.sm_count));
     attn_bwd_tc_kernel<HD, FORM><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
