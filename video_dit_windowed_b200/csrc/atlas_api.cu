@@ -3,8 +3,14 @@
 // Every entry point checks its arguments on the host and returns a status
 // without launching anything when they are bad. See include/atlas.h for the
 // contract of each call and the passages it implements.
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -13,6 +19,41 @@
 #include "cube_geom.cuh"
 
 namespace atlas {
+
+namespace {
+bool env_flag(const char *name) {
+    const char *v = std::getenv(name);
+    return v != nullptr && v[0] != '\0' && std::strcmp(v, "0") != 0;
+}
+}  // namespace
+
+bool log_enabled() {
+    static const bool on = env_flag("ATLAS_LOG");
+    return on;
+}
+
+TraceScope::TraceScope(const char *name) {
+    static const bool nvtx = env_flag("ATLAS_NVTX");
+    on = nvtx;
+    if (on) nvtxRangePushA(name);
+}
+
+TraceScope::~TraceScope() {
+    if (on) nvtxRangePop();
+}
+
+void log_launch(const char *kernel, int grid, int block, size_t smem, const char *fmt, ...) {
+    if (!log_enabled()) return;
+    char detail[256];
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(detail, sizeof detail, fmt, ap);
+    va_end(ap);
+    int dev = -1;
+    cudaGetDevice(&dev);
+    std::fprintf(stderr, "[atlas] dev %d %s grid %d block %d smem %zu %s\n", dev, kernel, grid,
+                 block, smem, detail);
+}
 
 __device__ uint32_t g_device_error = 0;
 
@@ -188,6 +229,7 @@ ATLAS_API atlas_status atlas_cube_reorder(const void *src, void *dst, atlas_grid
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, const atlas_rope *rope,
                                           atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::reorder(src, dst, 1, grid, cube, heads, head_dim, dtype, rope, stream, false);
 }
 
@@ -196,18 +238,21 @@ ATLAS_API atlas_status atlas_cube_reorder_noalloc(const void *src, void *dst, at
                                                   int32_t head_dim, atlas_dtype dtype,
                                                   const atlas_rope *rope,
                                                   atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::reorder(src, dst, 1, grid, cube, heads, head_dim, dtype, rope, stream, true);
 }
 
 ATLAS_API atlas_status atlas_cube_unorder(const void *src, void *dst, atlas_grid3 grid,
                                           atlas_cube3 cube, int32_t heads, int32_t head_dim,
                                           atlas_dtype dtype, atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::unorder(src, dst, 1, grid, cube, heads, head_dim, dtype, nullptr, stream);
 }
 
 ATLAS_API atlas_status atlas_rope3d(const void *src, void *dst, atlas_grid3 grid, int32_t heads,
                                     int32_t head_dim, atlas_dtype dtype, const atlas_rope *rope,
                                     atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::rope3d(src, dst, 1, grid, heads, head_dim, dtype, rope, stream);
 }
 
@@ -216,6 +261,7 @@ ATLAS_API atlas_status atlas_cube_reorder_batched(const void *src, void *dst, in
                                                   int32_t heads, int32_t head_dim,
                                                   atlas_dtype dtype, const atlas_rope *rope,
                                                   atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::reorder(src, dst, batch, grid, cube, heads, head_dim, dtype, rope, stream,
                           false);
 }
@@ -224,6 +270,7 @@ ATLAS_API atlas_status atlas_cube_unorder_batched(const void *src, void *dst, in
                                                   atlas_grid3 grid, atlas_cube3 cube,
                                                   int32_t heads, int32_t head_dim,
                                                   atlas_dtype dtype, atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, nullptr, stream);
 }
 
@@ -259,6 +306,7 @@ ATLAS_API atlas_status atlas_aligned_global_reorder(const void *src, void *dst, 
                                                     int32_t head_dim, atlas_dtype dtype,
                                                     const atlas_rope *rope,
                                                     atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::aligned_perm(src, dst, batch, grid, cube, global_grid, heads, head_dim, dtype,
                                rope, stream, 5);
 }
@@ -269,6 +317,7 @@ ATLAS_API atlas_status atlas_aligned_global_unorder(const void *src, void *dst, 
                                                     int32_t head_dim, atlas_dtype dtype,
                                                     const atlas_rope *rope,
                                                     atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::aligned_perm(src, dst, batch, grid, cube, global_grid, heads, head_dim, dtype,
                                rope, stream, 6);
 }
@@ -276,6 +325,7 @@ ATLAS_API atlas_status atlas_aligned_global_unorder(const void *src, void *dst, 
 ATLAS_API atlas_status atlas_aligned_global_offsets(atlas_grid3 grid, atlas_cube3 cube,
                                                     atlas_grid3 global_grid, int32_t *offsets,
                                                     int64_t capacity, int64_t *n_windows) {
+    ATLAS_TRACE();
     if (!n_windows) return ATLAS_ERR_NULL;
     if (grid.T < 1 || grid.H < 1 || grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1 ||
         global_grid.T < 1 || global_grid.H < 1 || global_grid.W < 1)
@@ -313,6 +363,7 @@ ATLAS_API atlas_status atlas_cube_unorder_rope(const void *src, void *dst, int64
                                                int32_t heads, int32_t head_dim,
                                                atlas_dtype dtype, const atlas_rope *rope,
                                                atlas_stream_t stream) {
+    ATLAS_TRACE();
     if (!rope) return ATLAS_ERR_NULL;
     return atlas::unorder(src, dst, batch, grid, cube, heads, head_dim, dtype, rope, stream);
 }
@@ -321,6 +372,7 @@ ATLAS_API atlas_status atlas_rope3d_batched(const void *src, void *dst, int64_t 
                                             atlas_grid3 grid, int32_t heads, int32_t head_dim,
                                             atlas_dtype dtype, const atlas_rope *rope,
                                             atlas_stream_t stream) {
+    ATLAS_TRACE();
     return atlas::rope3d(src, dst, batch, grid, heads, head_dim, dtype, rope, stream);
 }
 
@@ -482,6 +534,7 @@ ATLAS_API atlas_status atlas_local_global_attn(const void *q_d, const void *k_d,
                                                int64_t n_global, int32_t heads, int32_t head_dim,
                                                float softmax_scale, atlas_dtype dtype, void *o_d,
                                                void *o_g, float *lse, atlas_stream_t stream) {
+    ATLAS_TRACE();
     atlas_attn_layout ly{1, window_len, nullptr, 0, nullptr};
     return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, ly, heads,
                                     head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
@@ -492,6 +545,7 @@ ATLAS_API atlas_status atlas_local_global_attn_windows(
     const int32_t *window_offsets, int64_t n_windows, const void *q_g, const void *k_g,
     const void *v_g, int64_t n_global, int32_t heads, int32_t head_dim, float softmax_scale,
     atlas_dtype dtype, void *o_d, void *o_g, float *lse, atlas_stream_t stream) {
+    ATLAS_TRACE();
     if (n_detail > 0 && window_offsets == nullptr) return ATLAS_ERR_NULL;
     atlas_attn_layout ly{1, 1, window_offsets, n_windows, nullptr};
     return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, ly, heads,
@@ -503,6 +557,7 @@ ATLAS_API atlas_status atlas_local_global_attn_ex(
     const void *k_g, const void *v_g, int64_t n_global, const atlas_attn_layout *layout,
     int32_t heads, int32_t head_dim, float softmax_scale, atlas_dtype dtype, void *o_d,
     void *o_g, float *lse, atlas_stream_t stream) {
+    ATLAS_TRACE();
     if (!layout) return ATLAS_ERR_NULL;
     return atlas::local_global_attn(q_d, k_d, v_d, n_detail, q_g, k_g, v_g, n_global, *layout,
                                     heads, head_dim, softmax_scale, dtype, o_d, o_g, lse, stream);
@@ -515,6 +570,7 @@ ATLAS_API atlas_status atlas_local_global_attn_bwd(
     int32_t head_dim, float softmax_scale, atlas_dtype dtype, const float *lse, float *delta,
     void *dq_d, void *dk_d, void *dv_d, void *dq_g, void *dk_g, void *dv_g,
     atlas_stream_t stream) {
+    ATLAS_TRACE();
     if (!layout) return ATLAS_ERR_NULL;
     const void *in_d[5] = {q_d, k_d, v_d, o_d, do_d};
     const void *in_g[5] = {q_g, k_g, v_g, o_g, do_g};
@@ -551,6 +607,7 @@ ATLAS_API atlas_status atlas_qkv_proj_reorder(const void *x, const void *w, int6
                                               int32_t heads, int32_t head_dim, atlas_dtype dtype,
                                               const atlas_rope *rope, void *q, void *k, void *v,
                                               atlas_stream_t stream) {
+    ATLAS_TRACE();
     atlas_status st = atlas::check_proj(x, w, batch, grid, cube, c_in, dtype);
     if (st != ATLAS_OK) return st;
     if (!q || !k || !v) return ATLAS_ERR_NULL;
@@ -575,6 +632,7 @@ ATLAS_API atlas_status atlas_out_proj_unorder(const void *o, const void *w, int6
                                               atlas_grid3 grid, atlas_cube3 cube, int32_t c_in,
                                               int32_t c_out, atlas_dtype dtype, void *y,
                                               atlas_stream_t stream) {
+    ATLAS_TRACE();
     atlas_status st = atlas::check_proj(o, w, batch, grid, cube, c_in, dtype);
     if (st != ATLAS_OK) return st;
     if (!y) return ATLAS_ERR_NULL;
@@ -593,6 +651,7 @@ ATLAS_API atlas_status atlas_out_proj_unorder(const void *o, const void *w, int6
 ATLAS_API atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 cube,
                                                  atlas_grid3 global_grid,
                                                  atlas_cube3 *global_cube) {
+    ATLAS_TRACE();
     if (!global_cube) return ATLAS_ERR_NULL;
     if (grid.T < 1 || grid.H < 1 || grid.W < 1 || global_grid.T < 1 || global_grid.H < 1 ||
         global_grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1)
@@ -614,6 +673,7 @@ ATLAS_API atlas_status atlas_aligned_global_cube(atlas_grid3 grid, atlas_cube3 c
 ATLAS_API atlas_status atlas_cube_window_offsets(atlas_grid3 grid, atlas_cube3 cube,
                                                  int32_t *offsets, int64_t capacity,
                                                  int64_t *n_windows) {
+    ATLAS_TRACE();
     if (!n_windows) return ATLAS_ERR_NULL;
     if (grid.T < 1 || grid.H < 1 || grid.W < 1 || cube.ct < 1 || cube.ch < 1 || cube.cw < 1)
         return ATLAS_ERR_SHAPE;
@@ -654,6 +714,7 @@ ATLAS_API const char *atlas_status_string(atlas_status status) {
 }
 
 ATLAS_API atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *code) {
+    ATLAS_TRACE();
     if (!code) return ATLAS_ERR_NULL;
     *code = 0;
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -666,11 +727,13 @@ ATLAS_API atlas_status atlas_last_device_error(atlas_stream_t stream, uint32_t *
     return v ? ATLAS_ERR_TIMEOUT : ATLAS_OK;
 }
 
-ATLAS_API atlas_status atlas_release_caches(void) { return release_rope_tables(); }
+ATLAS_API atlas_status atlas_release_caches(void) {
+    ATLAS_TRACE(); return release_rope_tables(); }
 
 ATLAS_API int64_t atlas_cached_rope_tables(void) { return cached_rope_tables(); }
 
 ATLAS_API atlas_status atlas_debug_stall_next_attention(void) {
+    ATLAS_TRACE();
     g_stall_request.store(1);
     return ATLAS_OK;
 }

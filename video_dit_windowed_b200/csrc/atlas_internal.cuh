@@ -53,6 +53,21 @@ struct DeviceInfo {
 // usable device or not compute capability 10.0.
 bool current_device(DeviceInfo *out);
 
+// Tracing and logging, both off by default and read once from the
+// environment: ATLAS_NVTX=1 opens an NVTX range around every C-ABI call
+// (named after the call; visible in Nsight Systems and Nsight Compute
+// timelines), ATLAS_LOG=1 prints one line per kernel launch to stderr (the
+// kernel, its grid, block and dynamic shared memory, and the work it walks).
+bool log_enabled();
+struct TraceScope {
+    bool on;
+    explicit TraceScope(const char *name);
+    ~TraceScope();
+};
+#define ATLAS_TRACE() ::atlas::TraceScope atlas_trace_scope_(__func__)
+void log_launch(const char *kernel, int grid, int block, size_t smem, const char *fmt, ...)
+    __attribute__((format(printf, 5, 6)));
+
 // Raise `func`'s dynamic shared-memory limit to `bytes` on the current
 // device, once per (device, function): the attribute belongs to the device's
 // context, so a process driving several GPUs sets it on each.

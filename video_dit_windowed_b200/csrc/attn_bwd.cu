@@ -290,6 +290,10 @@ dim3 row_grid(const AttnArgs &a) {
 template <typename T, int HD>
 atlas_status delta_hd(const AttnBwdArgs &b, cudaStream_t stream) {
     const AttnArgs &a = b.fwd;
+    if (log_enabled())
+        log_launch("delta_kernel", static_cast<int>(row_grid(a).x * row_grid(a).y), kWarps * 32, 0,
+                   "head_dim %d rows %lld heads %d", HD,
+                   static_cast<long long>(a.batch * (a.n_detail + a.n_global)), a.heads);
     delta_kernel<T, HD><<<row_grid(a), kWarps * 32, 0, stream>>>(
         static_cast<const T *>(a.o_d), static_cast<const T *>(b.do_d),
         static_cast<const T *>(a.o_g), static_cast<const T *>(b.do_g), b.delta, geo_of(a));
@@ -318,6 +322,9 @@ atlas_status bwd_simt_hd(const AttnBwdArgs &b, cudaStream_t stream) {
     p.dv_g = static_cast<float *>(b.dv_g);
     p.scale = a.scale;
     const Geo g = geo_of(a);
+    if (log_enabled())
+        log_launch("dq_simt_kernel + dkdv_simt_kernel", static_cast<int>(row_grid(a).x * row_grid(a).y),
+                   kWarps * 32, 0, "head_dim %d (fp32)", HD);
     dq_simt_kernel<HD><<<row_grid(a), kWarps * 32, 0, stream>>>(p, g);
     dkdv_simt_kernel<HD><<<row_grid(a), kWarps * 32, 0, stream>>>(p, g);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;

@@ -876,6 +876,11 @@ atlas_status launch_form(Params p, const DeviceInfo &dev, cudaStream_t stream) {
                     (FORM == kDKDV ? reinterpret_cast<uintptr_t>(p.out1[i]) : 0);
     p.o_v8 = (ptr_bits & 31) == 0;
     const int grid = static_cast<int>(std::min<int64_t>(units, dev.sm_count));
+    if (log_enabled())
+        log_launch(FORM == kDQ ? "attn_bwd_tc_kernel<dQ>" : "attn_bwd_tc_kernel<dK/dV>", grid,
+                   kThreads, smem, "head_dim %d units %lld (global-key units %d) batch %d heads %d "
+                   "n_detail %d n_global %d", HD, static_cast<long long>(units), p.n_long, p.batch,
+                   p.heads, p.N, p.G);
     attn_bwd_tc_kernel<HD, FORM><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

@@ -116,6 +116,10 @@ atlas_status launch_hd(const Params &p, cudaStream_t stream) {
     const int64_t rows = p.batch * (p.N + p.G);
     if (rows == 0) return ATLAS_OK;
     dim3 grid(static_cast<unsigned>((rows + kWarps - 1) / kWarps), static_cast<unsigned>(p.heads));
+    if (log_enabled())
+        log_launch("attn_simt_kernel", static_cast<int>(grid.x * grid.y), kWarps * 32, 0,
+                   "head_dim %d rows %lld heads %d (fp32)", HD, static_cast<long long>(rows),
+                   p.heads);
     attn_simt_kernel<HD><<<grid, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

@@ -892,6 +892,11 @@ atlas_status launch_hd(const AttnArgs &a, const DeviceInfo &dev, cudaStream_t st
     const size_t smem = sizeof(Smem<HD>) + 1024;
     if (!set_smem_limit(fn, static_cast<int>(smem))) return ATLAS_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(n_units, dev.sm_count));
+    if (log_enabled())
+        log_launch(narrow ? "attn_tc_kernel<NARROW>" : "attn_tc_kernel", grid, kThreads, smem,
+                   "head_dim %d units %lld batch %d heads %d n_detail %d window %d n_global %d "
+                   "offsets %s global_ranges %s", HD, static_cast<long long>(n_units), p.batch,
+                   p.heads, p.N, p.L, p.G, p.win_off ? "yes" : "no", p.gwin_off ? "yes" : "no");
     if (narrow)
         attn_tc_kernel<HD, true><<<grid, kThreads, smem, stream>>>(p);
     else

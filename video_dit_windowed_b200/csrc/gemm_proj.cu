@@ -346,6 +346,10 @@ atlas_status launch(Params &p, const void *a, const void *b, const DeviceInfo &d
                         static_cast<int>(smem)))
         return ATLAS_ERR_CUDA;
     const int grid = static_cast<int>(std::min<int64_t>(total, dev.sm_count));
+    if (log_enabled())
+        log_launch("gemm_proj_kernel", grid, kThreads, smem,
+                   "M %d N %d K %d tiles %d (128x256, groups of %d column tiles)%s", p.M, p.N,
+                   p.K, p.n_tile_total, kGroupN, p.tab ? " rope" : "");
     gemm_proj_kernel<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }

@@ -278,6 +278,10 @@ atlas_status launch_g(const Params &p, const DeviceInfo &dev, cudaStream_t strea
     uint32_t blocks_needed = (p.total_rows + kGroups - 1) / kGroups;
     uint32_t grid = std::min<uint32_t>(blocks_needed, static_cast<uint32_t>(dev.sm_count) * 8u);
     if (grid == 0) return ATLAS_OK;
+    if (log_enabled())
+        log_launch("permute_rope_kernel", static_cast<int>(grid), kThreads, 0,
+                   "mode %d rope %d elem_bytes %d row_group %d rows %u row_bytes %u", MODE,
+                   ROPE ? 1 : 0, EB, G, p.total_rows, p.row_vecs * 16u);
     permute_rope_kernel<EB, ROPE, MODE, G><<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? ATLAS_OK : ATLAS_ERR_CUDA;
 }
