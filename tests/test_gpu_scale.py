@@ -13,7 +13,7 @@ EVERY row with the fp64 oracle:
   * the NARROW form with partial cubes (variable windows from offsets) and
     with the "aligned proxy tokens only" ranges;
   * the backward, both unit forms (dQ with query rows resident, dK/dV with
-    key rows resident), fixed and variable windows.
+    key rows resident), fixed and variable windows and the aligned ranges.
 
 Then the indicator-V mask probe on every row of the full-size workloads (720p,
 4k, 4k_long with fixed windows; 8k29 with partial cubes, all global keys and
@@ -192,6 +192,29 @@ def test_every_row_backward_partial_cubes():
                                    f64(t["q_g"]), f64(t["k_g"]), f64(t["v_g"]), f64(t["do_d"]),
                                    f64(t["do_g"]), hd ** -0.5, n_threads(), win_off=off)
     assert_grads_close([f64(g) for g in got], ref, "bf16", "backward, partial cubes")
+
+
+def test_every_row_backward_aligned_ranges():
+    """Aligned proxy tokens only (9x48x80 grid, 3x16x16 cubes, 9x12x20 proxy
+    grid), 4 heads: 1148 units in each form. The GPU takes the global tokens
+    in the aligned order, the oracle in raster order."""
+    grid, cube, gg, heads, hd = (9, 48, 80), (3, 16, 16), (9, 12, 20), 4, 128
+    N, G = 9 * 48 * 80, 9 * 12 * 20
+    assert ceil_div(N + G, TILE_ROWS_BWD) * heads >= 7 * n_sm()
+    t = bwd_inputs(1, N, G, heads, hd, "bf16", seed=37)
+    pos_t = torch.as_tensor(aligned_positions(grid, cube, gg), device=DEV)
+    y = dict(t)
+    for s in ("q_g", "k_g", "v_g", "do_g"):      # raster -> aligned order
+        y[s] = torch.empty_like(t[s])
+        y[s][pos_t] = t[s]
+    got = bwd_run_gpu(y, 1, heads, N, G,
+                      window_offsets=atlas.cube_window_offsets(grid, cube).to(DEV),
+                      global_window_offsets=atlas.aligned_global_offsets(grid, cube, gg).to(DEV))
+    got = [f64(g) for g in got[:3]] + [f64(g[pos_t]) for g in got[3:]]   # back to raster
+    ref = orc().attention_bwd_full_aligned(
+        f64(t["q_d"]), f64(t["k_d"]), f64(t["v_d"]), grid, cube, f64(t["q_g"]), f64(t["k_g"]),
+        f64(t["v_g"]), gg, f64(t["do_d"]), f64(t["do_g"]), hd ** -0.5, n_threads())
+    assert_grads_close(got, ref, "bf16", "backward, aligned ranges")
 
 
 # ---------------------------------------------------------------------------
