@@ -250,3 +250,25 @@ def test_head_shards_equal_the_full_call():
         for a, b in zip(full[:3], part[:3]):
             assert torch.equal(a[:, h0:h1].contiguous().view(torch.int16), b.view(torch.int16))
         assert torch.equal(full[3][h0:h1], part[3])
+
+
+def test_outputs_only_16_byte_aligned():
+    """The C-ABI promises outputs 16-byte alignment only; with both outputs
+    32-byte aligned the epilogue stores 32 bytes at a time, otherwise 16.
+    Outputs that start 16 bytes into a buffer take the 16-byte path and
+    must give the same bits."""
+    N, L, G, heads, hd = 1536, 768, 300, 2, 128
+    q_d, k_d, v_d, q_g, k_g, v_g = inputs(N, G, heads, hd, "bf16", seed=6)
+    ref_d, ref_g, ref_l = attention_gpu(q_d, k_d, v_d, L, q_g, k_g, v_g)
+    buf_d = torch.zeros(N * heads * hd + 8, dtype=torch.bfloat16, device=DEV)
+    buf_g = torch.zeros(G * heads * hd + 8, dtype=torch.bfloat16, device=DEV)
+    o_d = buf_d[8:].view(N, heads, hd)          # 16 bytes past a 512-byte boundary
+    o_g = buf_g[8:].view(G, heads, hd)
+    assert o_d.data_ptr() % 32 == 16 and o_g.data_ptr() % 32 == 16
+    lse = torch.empty_like(ref_l)
+    atlas.local_global_attn(q_d, k_d, v_d, L, q_g, k_g, v_g, o_d, o_g, lse)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    assert torch.equal(o_d.view(torch.int16), ref_d.view(torch.int16))
+    assert torch.equal(o_g.view(torch.int16), ref_g.view(torch.int16))
+    assert torch.equal(lse, ref_l)

@@ -295,3 +295,28 @@ def test_backward_window_forms(offsets):
                                    f64(t["do_g"]), hd ** -0.5, n_threads(),
                                    win_off=np.asarray(offsets, dtype=np.int64))
     assert_grads_close([f64(g) for g in got], ref, "bf16", f"offsets {offsets[:4]}")
+
+
+def test_gradients_only_16_byte_aligned():
+    """Gradient outputs that start 16 bytes into a buffer (the C-ABI's
+    minimum alignment) take the 16-byte store path: same bits as aligned
+    outputs."""
+    N, L, G, heads, hd = 1536, 768, 300, 2, 128
+    t = inputs(1, N, G, heads, hd, "bf16", seed=24)
+    ref = run_gpu(t, 1, heads, N, G, window_len=L)
+    o_d, o_g = torch.empty_like(t["q_d"]), torch.empty_like(t["q_g"])
+    lse = torch.empty(1, heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_ex(t["q_d"], t["k_d"], t["v_d"], t["q_g"], t["k_g"], t["v_g"], o_d,
+                               o_g, lse, window_len=L)
+    grads = []
+    for name in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g"):
+        buf = torch.zeros(t[name].numel() + 8, dtype=torch.bfloat16, device=DEV)
+        g = buf[8:].view(t[name].shape)
+        assert g.data_ptr() % 32 == 16
+        grads.append(g)
+    atlas.local_global_attn_bwd(t["q_d"], t["k_d"], t["v_d"], o_d, t["do_d"], t["q_g"],
+                                t["k_g"], t["v_g"], o_g, t["do_g"], lse, *grads, window_len=L)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    for a, b in zip(grads, ref):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
