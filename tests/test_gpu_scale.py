@@ -9,7 +9,8 @@ units outnumber the SMs several times over, so the cases here are sized for
 that (the unit count is asserted against the device's SM count) and compare
 EVERY row with the fp64 oracle:
   * the fixed-window form at the 720p geometry (21x48x80 grid, 3x16x16
-    cubes, 21x12x20 proxy grid) with 4 heads;
+    cubes, 21x12x20 proxy grid) with 4 heads, and on a smaller grid with a
+    batch of two problems and with head_dim 64;
   * the NARROW form with partial cubes (variable windows from offsets) and
     with the "aligned proxy tokens only" ranges;
   * the backward, both unit forms (dQ with query rows resident, dK/dV with
@@ -101,6 +102,31 @@ def test_every_row_fixed_windows_720p_geometry():
         f64(x["q_d"]), f64(x["k_d"]), f64(x["v_d"]), L, f64(x["q_g"]), f64(x["k_g"]),
         f64(x["v_g"]), w.softmax_scale, n_threads())
     compare_all_rows(o_d, o_g, lse, ref_d, ref_g, ref_l, "720p geometry, 4 heads")
+
+
+@pytest.mark.parametrize("B,heads,hd", [(2, 4, 128), (1, 8, 64)])
+def test_every_row_batch_and_head_dim_64(B, heads, hd):
+    """Fixed windows on a 9x48x80 grid (3x16x16 cubes, 9x12x20 proxy grid):
+    two problems stacked along the rows with 4 heads, and head_dim 64 with 8
+    heads; 1152 units either way."""
+    grid, gg, L = (9, 48, 80), (9, 12, 20), 768
+    N, G = 9 * 48 * 80, 9 * 12 * 20
+    assert fwd_units([L] * (N // L), G, heads) * B >= 7 * n_sm()
+    x = {s: mk(B * (N if s.endswith("_d") else G), heads, hd, s, seed=38)
+         for s in ("q_d", "k_d", "v_d", "q_g", "k_g", "v_g")}
+    o_d, o_g = torch.empty_like(x["q_d"]), torch.empty_like(x["q_g"])
+    lse = torch.empty(B, heads, N + G, dtype=torch.float32, device=DEV)
+    atlas.local_global_attn_ex(x["q_d"], x["k_d"], x["v_d"], x["q_g"], x["k_g"], x["v_g"], o_d,
+                               o_g, lse, batch=B, window_len=L)
+    torch.cuda.synchronize()
+    check_no_device_error()
+    for b in range(B):
+        sd, sg = slice(b * N, (b + 1) * N), slice(b * G, (b + 1) * G)
+        ref_d, ref_g, ref_l = orc().attention_full(
+            f64(x["q_d"][sd]), f64(x["k_d"][sd]), f64(x["v_d"][sd]), L, f64(x["q_g"][sg]),
+            f64(x["k_g"][sg]), f64(x["v_g"][sg]), hd ** -0.5, n_threads())
+        compare_all_rows(o_d[sd], o_g[sg], lse[b], ref_d, ref_g, ref_l,
+                         f"problem {b}, {heads} heads, head_dim {hd}")
 
 
 def test_every_row_partial_cubes_narrow_form():
