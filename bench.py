@@ -568,6 +568,14 @@ def time_oracle(w, budget_s=15.0, seed=0):
     return flops / t_total / 1e12, cores, sample, t_total
 
 
+def prep_phase_bytes(w):
+    """Algorithmic bytes of one problem's reorder+RoPE phase (bf16 I/O, every
+    head), the figure the GPU phase's GB/s counts; used to extrapolate the
+    oracle's sampled rate to the whole configuration."""
+    row = w.heads * w.head_dim * w.elem_bytes
+    return 2 * (3 * w.n_detail + 2 * w.n_global) * row
+
+
 def time_oracle_prep(w, heads=4):
     """Time the fp64 oracle's reorder + RoPE phase: RoPE then cube reorder of
     detail Q and K, byte reorder of detail V (bf16 rows), RoPE of global Q
@@ -858,10 +866,12 @@ def run_atlas(args, world, rank, local):
     if not args.no_cpu_baseline and world == 1 and args.mask == "all" and not args.backward:
         tf, cores, sample, _ = time_oracle(w, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": sample}
+                               "sample": sample,
+                               "extrapolated_full_config_s": flops / (tf * 1e12)}
         gbs, pcores, psample, _ = time_oracle_prep(w, heads=8)
-        out["cpu_baseline_reorder_rope"] = {"value": gbs, "unit": "GB/s", "cores": pcores,
-                                            "kind": "oracle", "sample": psample}
+        out["cpu_baseline_reorder_rope"] = {
+            "value": gbs, "unit": "GB/s", "cores": pcores, "kind": "oracle", "sample": psample,
+            "extrapolated_full_config_s": prep_phase_bytes(w) / (gbs * 1e9)}
     extra = (world == 1 and not args.no_workloads and args.workload == "720p" and
              args.mask == "all" and args.batch == 1 and not args.backward and not args.graph
              and not args.heads)
@@ -938,10 +948,12 @@ def run_workload_line(args, w, dev, stream, steps, pk, pk_kind, cpu_budget):
     if not args.no_cpu_baseline:
         tf, cores, sample, _ = time_oracle(w, budget_s=cpu_budget)
         line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample,
+                                "extrapolated_full_config_s": flops / (tf * 1e12)}
         gbs, pcores, psample, _ = time_oracle_prep(w)
-        line["cpu_baseline_reorder_rope"] = {"value": gbs, "unit": "GB/s", "cores": pcores,
-                                             "kind": "oracle", "sample": psample}
+        line["cpu_baseline_reorder_rope"] = {
+            "value": gbs, "unit": "GB/s", "cores": pcores, "kind": "oracle", "sample": psample,
+            "extrapolated_full_config_s": prep_phase_bytes(w) / (gbs * 1e9)}
     return line
 
 
