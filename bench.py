@@ -568,6 +568,127 @@ def time_oracle(w, budget_s=15.0, seed=0):
     return flops / t_total / 1e12, cores, sample, t_total
 
 
+def time_oracle_aligned(w, budget_s=10.0, seed=0):
+    """Time the fp64 oracle of the "aligned proxy tokens only" variant on a
+    bounded sample of one head: whole windows of detail rows, picked at
+    random, each against its own window and its aligned global keys, then a
+    128-row block of global rows, until about ``budget_s`` of work. FLOPs
+    count the pairs the mask allows (4*D per pair). Returns (TFLOP/s, cores,
+    sample, seconds)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    orc = oracle.Oracle()
+    cores = orc.max_threads()
+    rng = np.random.default_rng(seed)
+    D, G, N = w.head_dim, w.n_global, w.n_detail
+    off = orc.cube_windows(w.grid, w.cube)
+    n_win = off.size - 1
+    boxes = [w.aligned_boxes(a) for a in range(3)]
+    nb = [-(-E // c) for E, c in zip(w.grid, w.cube)]
+    kg, vg = rng.standard_normal((G, D)), rng.standard_normal((G, D))
+    flops, t, det, glob = 0, 0.0, 0, 0
+    for wi in rng.permutation(n_win):
+        if t >= budget_s:
+            break
+        lo, hi = int(off[wi]), int(off[wi + 1])
+        n = hi - lo
+        k, v, q = (rng.standard_normal((n, D)) for _ in range(3))
+        t0 = time.perf_counter()
+        orc.attention_head_aligned(w.grid, w.cube, w.global_grid, w.softmax_scale, k, v, lo, kg,
+                                   vg, np.arange(lo, hi, dtype=np.int64), q, cores)
+        t += time.perf_counter() - t0
+        bt, rest = divmod(int(wi), nb[1] * nb[2])
+        bh, bw = divmod(rest, nb[2])
+        flops += 4 * D * n * (n + boxes[0][bt] * boxes[1][bh] * boxes[2][bw])
+        det += n
+    if G:
+        rows = min(128, G)
+        q = rng.standard_normal((rows, D))
+        t0 = time.perf_counter()
+        orc.attention_head_aligned(w.grid, w.cube, w.global_grid, w.softmax_scale, None, None, 0,
+                                   kg, vg, N + np.arange(rows, dtype=np.int64), q, cores)
+        t += time.perf_counter() - t0
+        flops += 4 * D * rows * G
+        glob = rows
+    sample = (f"{det} detail rows (whole windows, random) + {glob} global rows of one head, "
+              f"aligned mask, {t:.1f} s of fp64 oracle work")
+    return flops / t / 1e12, cores, sample, t
+
+
+def slab_workload(w, mask):
+    """One head of the workload cut to its first slab of cubes along time
+    (the first ct frames of the detail grid); the global grid stays whole for
+    the method's mask and is cut to the frames aligned with the slab for the
+    aligned mask."""
+    import dataclasses
+    grid = (min(w.grid[0], w.cube[0]), w.grid[1], w.grid[2])
+    gg = w.global_grid
+    if mask == "aligned" and w.n_global:
+        gg = (max(1, -(-grid[0] * gg[0] // w.grid[0])), gg[1], gg[2])
+    return dataclasses.replace(w, grid=grid, global_grid=gg, heads=1)
+
+
+def time_oracle_bwd(w, mask="all", seed=0):
+    """Time the fp64 oracle's backward (softmax-Jacobian definition: every
+    row's statistics, then dQ over query rows and dK, dV over key rows), in
+    full, on one head of the workload's first slab of cubes along time
+    (slab_workload). FLOPs: 2.5x the forward's allowed-pair FLOPs, the count
+    the GPU's training-step line uses. Returns (TFLOP/s, cores, sample, s)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    orc = oracle.Oracle()
+    cores = orc.max_threads()
+    rng = np.random.default_rng(seed)
+    s = slab_workload(w, mask)
+    N, G, D = s.n_detail, s.n_global, s.head_dim
+    q_d, k_d, v_d, do_d = (rng.standard_normal((N, 1, D)) for _ in range(4))
+    q_g, k_g, v_g, do_g = (rng.standard_normal((G, 1, D)) for _ in range(4))
+    t0 = time.perf_counter()
+    if mask == "aligned":
+        orc.attention_bwd_full_aligned(q_d, k_d, v_d, s.grid, s.cube, q_g, k_g, v_g,
+                                       s.global_grid, do_d, do_g, s.softmax_scale, cores)
+    else:
+        off = orc.cube_windows(s.grid, s.cube) if s.partial else None
+        orc.attention_bwd_full(q_d, k_d, v_d, s.window_len, q_g, k_g, v_g, do_d, do_g,
+                               s.softmax_scale, cores, win_off=off)
+    t = time.perf_counter() - t0
+    flops = s.unmasked_flops(mask) * 5 // 2
+    sample = (f"one head, detail {s.grid[0]}x{s.grid[1]}x{s.grid[2]} (first slab of cubes), "
+              f"global {s.global_grid[0]}x{s.global_grid[1]}x{s.global_grid[2]}, {mask} mask, "
+              f"full backward, {t:.1f} s of fp64 oracle work")
+    return flops / t / 1e12, cores, sample, t
+
+
+def time_oracle_proj(w, seed=0):
+    """Time the oracle's projections (fp64 matmul composed with its RoPE and
+    cube reorder for Q, K, V; its unorder composed with the output matmul)
+    on a corner of the workload's grid two cubes wide (ct x ch x 2cw tokens),
+    model width heads*head_dim, random weights. FLOPs 2*rows*C*3C + 2*rows*C*C. Returns
+    (TFLOP/s, cores, sample, seconds)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    orc = oracle.Oracle()
+    rng = np.random.default_rng(seed)
+    grid = (min(w.grid[0], w.cube[0]), min(w.grid[1], w.cube[1]),
+            min(w.grid[2], 2 * w.cube[2]))
+    rows = grid[0] * grid[1] * grid[2]
+    C = w.heads * w.head_dim
+    x = rng.standard_normal((rows, C))
+    w_qkv = rng.standard_normal((3 * C, C)) / C ** 0.5
+    w_o = rng.standard_normal((C, C)) / C ** 0.5
+    t0 = time.perf_counter()
+    q, _, _ = orc.qkv_proj_reorder(x, w_qkv, grid, w.cube, w.heads, w.head_dim, w.theta,
+                                   w.split, w.detail_scales)
+    orc.out_proj_unorder(q.reshape(rows, C), w_o, grid, w.cube)
+    t = time.perf_counter() - t0
+    flops = 2 * rows * C * 3 * C + 2 * rows * C * C
+    cores = os.cpu_count() or 1
+    sample = (f"detail {grid[0]}x{grid[1]}x{grid[2]} ({rows} rows, two cubes), width "
+              f"{C}: QKV projection + RoPE + reorder and unorder + output projection, "
+              f"{t:.1f} s (numpy fp64 matmul on up to {cores} threads)")
+    return flops / t / 1e12, cores, sample, t
+
+
 def prep_phase_bytes(w):
     """Algorithmic bytes of one problem's reorder+RoPE phase (bf16 I/O, every
     head), the figure the GPU phase's GB/s counts; used to extrapolate the
@@ -863,6 +984,16 @@ def run_atlas(args, world, rank, local):
                          "peak_kind": peak_kind}}
     if e2e:
         out["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1 and args.backward and args.mask in ("all",
+                                                                                  "aligned"):
+        tf, cores, sample, _ = time_oracle_bwd(w, args.mask)
+        out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample, "counts": "backward as 2.5x the forward"}
+    if not args.no_cpu_baseline and world == 1 and args.mask == "aligned" and not args.backward:
+        tf, cores, sample, _ = time_oracle_aligned(w, budget_s=min(args.cpu_budget, 10.0))
+        out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample,
+                               "extrapolated_full_config_s": flops / (tf * 1e12)}
     if not args.no_cpu_baseline and world == 1 and args.mask == "all" and not args.backward:
         tf, cores, sample, _ = time_oracle(w, budget_s=args.cpu_budget)
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -994,6 +1125,10 @@ def report_proj(args, world, rank, path, elapsed, phases, clk):
         "gpu_launches": path.launches_per_step() * args.steps,
         "clocks": clk,
     }
+    if not args.no_cpu_baseline and world == 1:
+        tf, cores, sample, _ = time_oracle_proj(path.w)
+        out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample, "counts": "projection FLOPs only"}
     print(json.dumps(out), flush=True)
 
 
