@@ -538,8 +538,10 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
     // P = exp2(S*scale*log2e - m) of the NC columns in `sr`, as bf16 pairs
     // into tensor memory (stores of 32 packed columns; one of 16 for a
     // 32-column tile); returns the row sum of the fp32 P. WithMax: the row
-    // maximum of the raw S is taken in the same pass, into mx.
-    auto exp_store = [&](auto with_max, const auto &sr, float m, float &mx) -> float {
+    // maximum of the raw S is taken in the same pass, into mx. `between` runs
+    // after the first group's store, before the second group is read.
+    auto exp_store = [&](auto with_max, const auto &sr, float m, float &mx,
+                         auto &&between) -> float {
         constexpr bool kWithMax = decltype(with_max)::value;
         constexpr int NC = static_cast<int>(sizeof(sr) / sizeof(uint32_t));
         constexpr int kPer = NC >= 64 ? 32 : 16;
@@ -566,6 +568,7 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
                 ptx::tmem_st32_nowait(t_s + g * 32, pk);
             else
                 ptx::tmem_st16_nowait(t_s + g * 16, pk);
+            if (g == 0) between();
         }
         ptx::tmem_wait_st();
 #pragma unroll
@@ -643,20 +646,30 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
             // narrow tile: the others hold no allowed key of any row).
             auto tile = [&](auto ncw) -> float {
                 constexpr int NC = decltype(ncw)::value;
+                // A full tile loads its second 64 columns while the first
+                // 64 are exponentiated (fast path), else before anything.
                 uint32_t sr[NC];
-                if constexpr (NC == 128)
-                    ptx::tmem_ld128(t_s, sr);
-                else if constexpr (NC == 64)
+                auto &sr_hi = *reinterpret_cast<uint32_t(*)[64]>(&sr[NC > 64 ? 64 : 0]);
+                if constexpr (NC == 128) {
+                    ptx::tmem_ld64(t_s, *reinterpret_cast<uint32_t(*)[64]>(&sr[0]));
+                    ptx::tmem_ld64_nowait(t_s + 64, sr_hi);
+                } else if constexpr (NC == 64) {
                     ptx::tmem_ld64(t_s, sr);
-                else
+                } else {
                     ptx::tmem_ld32(t_s, sr);
-                if (row_masked) {
-#pragma unroll
-                    for (int c = 0; c < NC; ++c)
-                        if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
                 }
+                auto wait_hi = [&] {
+                    if constexpr (NC == 128) ptx::tmem_wait_ld(sr_hi);
+                };
+                auto nothing = [] {};
                 float sum, mx;
                 if (__any_sync(kAll, m_run == kNegInf || row_masked)) {
+                    wait_hi();
+                    if (row_masked) {
+#pragma unroll
+                        for (int c = 0; c < NC; ++c)
+                            if (k0 + c < klo || k0 + c >= khi) sr[c] = __float_as_uint(kNegInf);
+                    }
                     // No reference yet, or masked keys: row max first. The
                     // reference moves only when the tile's max exceeds it by
                     // more than the threshold (exact either way: O and l
@@ -671,12 +684,13 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
                     }
                     l_run *= alpha;
                     if (j > 0) rescale_o(need, alpha);
-                    sum = exp_store(std::false_type{}, sr, m_run == kNegInf ? 0.f : m_run, mx);
+                    sum = exp_store(std::false_type{}, sr, m_run == kNegInf ? 0.f : m_run, mx,
+                                    nothing);
                 } else {
                     // Exponentials against the running reference right away,
                     // the tile max in the same pass; redo the (rare) rows
                     // whose max moved past the threshold.
-                    sum = exp_store(std::true_type{}, sr, m_run, mx);
+                    sum = exp_store(std::true_type{}, sr, m_run, mx, wait_hi);
                     const float mx2 = mx * sc;
                     const bool need = mx2 > m_run + kRescaleThreshold;
                     if (__any_sync(kAll, need)) {
@@ -684,7 +698,7 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
                         if (need) m_run = mx2;
                         l_run *= alpha;
                         rescale_o(need, alpha);
-                        sum = exp_store(std::false_type{}, sr, m_run, mx);
+                        sum = exp_store(std::false_type{}, sr, m_run, mx, nothing);
                     }
                 }
                 return sum;
