@@ -725,35 +725,36 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
         __nv_bfloat16 *out = U.detail ? p.o_d : p.o_g;
         uint4 *dst = reinterpret_cast<uint4 *>(
             out + (static_cast<int64_t>(U.row0 + (row_valid ? q : 0)) * p.heads + U.head) * HD);
-#pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-            uint32_t o[32];
-            ptx::tmem_ld32(t_o + c * 32, o);
-            if (row_valid && p.o_v8) {
-                // two 32-byte stores per 32 columns: whole sectors
+        // The whole O row in one load and one wait, then bf16 stores.
+        uint32_t o[HD];
+        if constexpr (HD == 128)
+            ptx::tmem_ld128(t_o, o);
+        else
+            ptx::tmem_ld64(t_o, o);
+        if (row_valid && p.o_v8) {
+            // 32-byte stores: whole sectors
 #pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                    uint32_t w8[8];
+            for (int v = 0; v < HD / 16; ++v) {
+                uint32_t w8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        w8[e] = ptx::pack_bf16x2(__uint_as_float(o[16 * v + 2 * e]) * inv_l,
-                                                 __uint_as_float(o[16 * v + 2 * e + 1]) * inv_l);
-                    ptx::st_global_v8(reinterpret_cast<uint8_t *>(dst) + c * 64 + v * 32, w8);
-                }
-            } else if (row_valid) {
+                for (int e = 0; e < 8; ++e)
+                    w8[e] = ptx::pack_bf16x2(__uint_as_float(o[16 * v + 2 * e]) * inv_l,
+                                             __uint_as_float(o[16 * v + 2 * e + 1]) * inv_l);
+                ptx::st_global_v8(reinterpret_cast<uint8_t *>(dst) + v * 32, w8);
+            }
+        } else if (row_valid) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    uint4 w;
-                    w.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
-                                           __uint_as_float(o[8 * v + 1]) * inv_l);
-                    w.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
-                                           __uint_as_float(o[8 * v + 3]) * inv_l);
-                    w.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
-                                           __uint_as_float(o[8 * v + 5]) * inv_l);
-                    w.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
-                                           __uint_as_float(o[8 * v + 7]) * inv_l);
-                    dst[c * 4 + v] = w;
-                }
+            for (int v = 0; v < HD / 8; ++v) {
+                uint4 w;
+                w.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                       __uint_as_float(o[8 * v + 1]) * inv_l);
+                w.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                       __uint_as_float(o[8 * v + 3]) * inv_l);
+                w.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                       __uint_as_float(o[8 * v + 5]) * inv_l);
+                w.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                       __uint_as_float(o[8 * v + 7]) * inv_l);
+                dst[v] = w;
             }
         }
         if (p.lse != nullptr && row_valid) {
