@@ -649,17 +649,17 @@ __device__ void softmax_epilogue(const Params &p, const Sched &S, Smem<HD> &sm, 
                 // A full tile loads its second 64 columns while the first
                 // 64 are exponentiated (fast path), else before anything.
                 uint32_t sr[NC];
-                auto &sr_hi = *reinterpret_cast<uint32_t(*)[64]>(&sr[NC > 64 ? 64 : 0]);
                 if constexpr (NC == 128) {
                     ptx::tmem_ld64(t_s, *reinterpret_cast<uint32_t(*)[64]>(&sr[0]));
-                    ptx::tmem_ld64_nowait(t_s + 64, sr_hi);
+                    ptx::tmem_ld64_nowait(t_s + 64, *reinterpret_cast<uint32_t(*)[64]>(&sr[64]));
                 } else if constexpr (NC == 64) {
                     ptx::tmem_ld64(t_s, sr);
                 } else {
                     ptx::tmem_ld32(t_s, sr);
                 }
                 auto wait_hi = [&] {
-                    if constexpr (NC == 128) ptx::tmem_wait_ld(sr_hi);
+                    if constexpr (NC == 128)
+                        ptx::tmem_wait_ld(*reinterpret_cast<uint32_t(*)[64]>(&sr[64]));
                 };
                 auto nothing = [] {};
                 float sum, mx;
